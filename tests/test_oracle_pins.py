@@ -1,0 +1,422 @@
+"""Pins for the f64 oracle: closed forms, invariants, brute force and library
+routines that do not share the oracle's own formulas.
+
+Every pin is a function of the oracle module, so the same pins also run
+against mutated copies of the oracle (a sign flipped, a term dropped, an
+index moved): each planted mistake must make at least one pin fail.
+"""
+import importlib.util
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle.kld_oracle as ORACLE
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ORACLE_SRC = os.path.join(ROOT, "oracle", "kld_oracle.py")
+
+
+def _close(a, b, rtol=1e-10, atol=1e-12):
+    return abs(a - b) <= atol + rtol * abs(b)
+
+
+# ---------------------------------------------------------------------------
+# full-vocabulary pins
+# ---------------------------------------------------------------------------
+
+def pin_self_is_zero(O):
+    rng = np.random.default_rng(1)
+    for V in (2, 7, 1000):
+        x = rng.normal(0, 3, V)
+        r = O.full_vocab_row(x, x.copy(), 0)
+        assert r["kl"] == 0.0
+        assert r["ref_argmax"] == r["cand_argmax"] == int(np.argmax(x))
+
+
+def pin_nonnegative(O):
+    rng = np.random.default_rng(2)
+    for _ in range(50):
+        V = int(rng.integers(2, 300))
+        x = rng.normal(0, 2, V)
+        y = x + rng.normal(0, rng.uniform(0.01, 3), V)
+        assert O.full_vocab_row(x, y)["kl"] >= -1e-14
+
+
+def pin_one_hot_vs_uniform(O):
+    for V in (2, 10, 4096, 248_320):
+        x = np.full(V, -np.inf)
+        x[V // 3] = 0.0
+        r = O.full_vocab_row(x, np.zeros(V), V // 3)
+        assert _close(r["kl"], math.log(V), rtol=1e-13)
+        assert r["ref_argmax"] == V // 3 and r["cand_argmax"] == 0
+        assert r["ref_target_lp"] == 0.0
+        assert _close(r["cand_target_lp"], -math.log(V), rtol=1e-13)
+
+
+def pin_two_point(O):
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        a, b, c, d = rng.normal(0, 2, 4)
+        p = 1.0 / (1.0 + math.exp(b - a))
+        q = 1.0 / (1.0 + math.exp(d - c))
+        want = p * math.log(p / q) + (1 - p) * math.log((1 - p) / (1 - q))
+        got = O.full_vocab_row(np.array([a, b]), np.array([c, d]))["kl"]
+        assert _close(got, want, rtol=1e-9, atol=1e-15)
+
+
+def pin_geometric(O):
+    # x_i = a i, y_i = b i: truncated geometric distributions with ratio
+    # r = e^a; Z(a) = (1 - r^V) / (1 - r), E_p[i] = r/(1-r) - V r^V/(1-r^V),
+    # KL = (a - b) E_p[i] - ln Z(a) + ln Z(b).
+    for (a, b, V) in ((-0.3, -0.25, 50), (-0.05, -0.2, 400), (0.1, -0.1, 30)):
+        i = np.arange(V, dtype=np.float64)
+        ra, rb = math.exp(a), math.exp(b)
+        Za = (1 - ra ** V) / (1 - ra)
+        Zb = (1 - rb ** V) / (1 - rb)
+        Ei = ra / (1 - ra) - V * ra ** V / (1 - ra ** V)
+        want = (a - b) * Ei - math.log(Za) + math.log(Zb)
+        r = O.full_vocab_row(a * i, b * i, V - 1)
+        assert _close(r["kl"], want, rtol=1e-10)
+        # log p_{V-1} = a (V-1) - ln Z(a); log q_{V-1} = b (V-1) - ln Z(b)
+        assert _close(r["ref_target_lp"], a * (V - 1) - math.log(Za), rtol=1e-12)
+        assert _close(r["cand_target_lp"], b * (V - 1) - math.log(Zb), rtol=1e-12)
+
+
+def pin_single_logit_shift(O):
+    # y = x + c e_j  =>  KL(p || q) = ln(1 - p_j + p_j e^c) - c p_j
+    rng = np.random.default_rng(4)
+    for _ in range(20):
+        V = int(rng.integers(3, 500))
+        x = rng.normal(0, 1.5, V)
+        j = int(rng.integers(0, V))
+        c = float(rng.normal(0, 2))
+        y = x.copy()
+        y[j] += c
+        e = np.exp(x - x.max())
+        pj = e[j] / e.sum()
+        want = math.log(1 - pj + pj * math.exp(c)) - c * pj
+        assert _close(O.full_vocab_row(x, y)["kl"], want, rtol=1e-9, atol=1e-15)
+
+
+def pin_shift_and_permutation(O):
+    rng = np.random.default_rng(5)
+    V = 777
+    x = rng.normal(0, 2, V)
+    y = x + rng.normal(0, 0.3, V)
+    base = O.full_vocab_row(x, y, 5)
+    sh = O.full_vocab_row(x + 3.7, y - 2.1, 5)
+    assert _close(sh["kl"], base["kl"], rtol=1e-10)
+    assert _close(sh["ref_target_lp"], base["ref_target_lp"], rtol=1e-12)
+    perm = rng.permutation(V)
+    pr = O.full_vocab_row(x[perm], y[perm], int(np.argmax(perm == 5)))
+    assert _close(pr["kl"], base["kl"], rtol=1e-10)
+    assert perm[pr["ref_argmax"]] == base["ref_argmax"]
+    assert _close(pr["ref_target_lp"], base["ref_target_lp"], rtol=1e-12)
+
+
+def pin_argmax_lowest_index(O):
+    x = np.array([1.0, 3.0, 2.0, 3.0, 3.0])
+    y = np.array([5.0, 0.0, 5.0, 5.0, -1.0])
+    r = O.full_vocab_row(x, y)
+    assert r["ref_argmax"] == 1 and r["cand_argmax"] == 0
+
+
+def pin_uniform_target(O):
+    for V in (3, 4096):
+        r = O.full_vocab_row(np.zeros(V), np.full(V, 2.5), 1)
+        assert _close(r["ref_target_lp"], -math.log(V), rtol=1e-13)
+        assert abs(r["kl"]) < 1e-15
+
+
+def pin_non_finite(O):
+    V = 16
+    x = np.linspace(-2, 2, V)
+    bad = x.copy()
+    bad[3] = np.nan
+    for a, b in ((bad, x), (x, bad)):
+        r = O.full_vocab_row(a, b, 1)
+        assert math.isnan(r["kl"]) and r["ref_argmax"] == -1 and math.isnan(r["ref_target_lp"])
+    pinf = x.copy()
+    pinf[0] = np.inf
+    assert math.isnan(O.full_vocab_row(pinf, x)["kl"])
+    assert math.isnan(O.full_vocab_row(np.full(V, -np.inf), x)["kl"])
+    # a masked reference id (x = -inf) contributes nothing, even against -inf
+    xm = x.copy()
+    xm[2] = -np.inf
+    ym = x.copy()
+    ym[2] = -np.inf
+    assert abs(O.full_vocab_row(xm, ym)["kl"]) < 1e-15
+    # the candidate gives zero mass where the reference has some: KL = +inf
+    yz = x.copy()
+    yz[7] = -np.inf
+    assert O.full_vocab_row(x, yz)["kl"] == math.inf
+
+
+def pin_bf16_conversion(O):
+    # bf16 bit patterns of a few exactly known values
+    bits = np.array([0x3F80, 0xC000, 0x0000, 0x7F80, 0xFF80, 0x3E80, 0x4049], dtype=np.uint16)
+    want = [1.0, -2.0, 0.0, math.inf, -math.inf, 0.25, 3.140625]
+    assert list(O.bf16_bits_to_f64(bits)) == want
+
+
+# ---------------------------------------------------------------------------
+# top-k + tail bucket pins
+# ---------------------------------------------------------------------------
+
+def _brute_force_tail_kl(ref_ids, ref_lp, cand_ids, cand_lp, V):
+    """Materialise the candidate's distribution over all V ids from the
+    rule (listed ids keep their mass, the leftover is spread evenly over the
+    other V - k ids), then coarsen both sides onto the reference's k cells
+    plus one cell holding every other id, by enumeration."""
+    k = len(ref_ids)
+    q_full = [None] * V
+    for s, cid in enumerate(cand_ids):
+        if q_full[cid] is None:
+            q_full[cid] = math.exp(cand_lp[s])
+    listed = sum(math.exp(v) for v in cand_lp)
+    fill = max(1.0 - listed, 0.0) / (V - k)
+    q_full = [fill if v is None else v for v in q_full]
+    p_cells = [math.exp(v) for v in ref_lp]
+    q_cells = [q_full[r] for r in ref_ids]
+    p_rest = 1.0 - sum(p_cells)
+    q_rest = sum(q_full[v] for v in range(V) if v not in set(ref_ids))
+    kl = 0.0
+    for p, q in zip(p_cells, q_cells):
+        kl += p * math.log(p / q)
+    if p_rest > 0:
+        kl += p_rest * math.log(p_rest / q_rest)
+    return kl
+
+
+def pin_tail_brute_force(O):
+    rng = np.random.default_rng(6)
+    for _ in range(300):
+        V = int(rng.integers(3, 17))
+        k = int(rng.integers(1, min(8, V - 1) + 1))
+        # full distributions so that every listed mass is consistent
+        p = rng.dirichlet(np.full(V, 0.7))
+        q = rng.dirichlet(np.full(V, 0.7))
+        ref_ids = rng.permutation(V)[:k]
+        cand_ids = rng.permutation(V)[:k]
+        ref_lp = np.log(p[ref_ids])
+        cand_lp = np.log(q[cand_ids])
+        want = _brute_force_tail_kl(list(ref_ids), list(ref_lp), list(cand_ids), list(cand_lp), V)
+        got = O.topk_tail_row(ref_ids, ref_lp, cand_ids, cand_lp, V)
+        assert _close(got["kl"], want, rtol=1e-9, atol=1e-13), (V, k, got, want)
+        assert got["n_matched"] == len(set(ref_ids) & set(cand_ids))
+        assert got["top1"] == int(ref_ids[0] == cand_ids[0])
+        vec = O.topk_tail(ref_ids[None], ref_lp[None], cand_ids[None], cand_lp[None], V)
+        assert _close(vec["kl"][0], want, rtol=1e-9, atol=1e-13)
+        assert vec["n_matched"][0] == got["n_matched"]
+
+
+def pin_tail_lower_bound(O):
+    # "The score": coarsening onto cells gives a lower bound on the full KL.
+    # When the candidate's top-k holds every reference top-k id, the tail
+    # rule is an exact coarsening, so tail KL <= full KL must hold.
+    rng = np.random.default_rng(7)
+    hits = 0
+    for _ in range(200):
+        V = int(rng.integers(20, 200))
+        k = int(rng.integers(2, 12))
+        x = rng.normal(0, 2, V)
+        y = x + rng.normal(0, 0.05, V)
+        lp = x - (x.max() + math.log(np.exp(x - x.max()).sum()))
+        lq = y - (y.max() + math.log(np.exp(y - y.max()).sum()))
+        R = np.argsort(-lp, kind="stable")[:k]
+        C = np.argsort(-lq, kind="stable")[:k]
+        if not set(R) <= set(C):
+            continue
+        hits += 1
+        t = O.topk_tail_row(R, lp[R], C, lq[C], V)["kl"]
+        f = O.full_vocab_row(x, y)["kl"]
+        assert t <= f + 1e-13
+        # with the ids equal the tail rule is the exact two-level coarsening
+        pr = 1 - np.exp(lp[R]).sum()
+        qr = 1 - np.exp(lq[R]).sum()
+        exact = float(np.sum(np.exp(lp[R]) * (lp[R] - lq[R]))) + pr * math.log(pr / qr)
+        assert _close(t, exact, rtol=1e-9, atol=1e-14)
+    assert hits > 20
+
+
+def pin_tail_spread_cases(O):
+    # one unmatched id: q = leftover / (V - k), exactly
+    V, k = 10, 2
+    ref_ids = np.array([0, 1])
+    cand_ids = np.array([0, 5])
+    ref_lp = np.log(np.array([0.5, 0.25]))
+    cand_lp = np.log(np.array([0.4, 0.2]))
+    spread = 0.4 / 8
+    want = 0.5 * math.log(0.5 / 0.4) + 0.25 * math.log(0.25 / spread) \
+        + 0.25 * math.log(0.25 / (1 - 0.4 - spread))
+    assert _close(O.topk_tail_row(ref_ids, ref_lp, cand_ids, cand_lp, V)["kl"], want, rtol=1e-12)
+    # duplicate candidate id: the first slot is the match
+    r = O.topk_tail_row(np.array([3, 1]), np.log([0.5, 0.1]), np.array([3, 3]),
+                        np.log([0.3, 0.2]), 20)
+    assert r["n_matched"] == 1
+    q_tail = 1 - 0.3 - 0.5 / 18
+    want = 0.5 * math.log(0.5 / 0.3) + 0.1 * math.log(0.1 / (0.5 / 18)) + 0.4 * math.log(0.4 / q_tail)
+    assert _close(r["kl"], want, rtol=1e-12)
+
+
+def pin_tail_self(O):
+    rng = np.random.default_rng(8)
+    ids = np.stack([rng.permutation(1000)[:64] for _ in range(50)])
+    lp = np.sort(np.log(rng.dirichlet(np.ones(80), 50)[:, :64]), axis=1)[:, ::-1].astype(np.float16)
+    r = O.topk_tail(ids, lp, ids, lp, 1000)
+    assert np.all(r["kl"] == 0.0) and np.all(r["top1"] == 1) and np.all(r["n_matched"] == 64)
+
+
+# ---------------------------------------------------------------------------
+# reductions
+# ---------------------------------------------------------------------------
+
+def pin_quantiles(O):
+    rng = np.random.default_rng(9)
+    for n in (1, 2, 3, 10, 1001, 2047):
+        kl = rng.exponential(1e-3, n).astype(np.float32)
+        qs = (0.0, 0.5, 0.9, 0.99, 0.999, 1.0)
+        st = O.reduce_stats(kl, quantiles=qs)
+        want = np.quantile(kl.astype(np.float64), qs, method="linear")
+        for got, w in zip(st["q_value"], want):
+            assert _close(got, float(w), rtol=1e-15, atol=0)
+        s = sorted(kl.tolist())
+        for q, lo, hi in zip(qs, st["q_lo"], st["q_hi"]):
+            h = (n - 1) * q
+            assert lo == s[int(math.floor(h))]
+            assert hi == s[min(int(math.floor(h)) + 1, n - 1)]
+
+
+def pin_mean_and_counts(O):
+    rng = np.random.default_rng(10)
+    n = 3000
+    kl = rng.exponential(0.01, n).astype(np.float32)
+    kl[::97] = np.nan
+    mask = rng.random(n) < 0.8
+    ra = rng.integers(0, 5, n)
+    ca = rng.integers(0, 5, n)
+    rt = -rng.exponential(2.0, n).astype(np.float32)
+    ct = -rng.exponential(2.1, n).astype(np.float32)
+    thr = (0.0, 0.01, 0.05)
+    st = O.reduce_stats(kl, ra, ca, None, rt, ct, mask, quantiles=(0.5,), thresholds=thr)
+    sel = [i for i in range(n) if mask[i] and not math.isnan(kl[i])]
+    assert st["n"] == len(sel)
+    assert st["n_nan"] == sum(1 for i in range(n) if mask[i] and math.isnan(kl[i]))
+    exact = sum((Fraction(float(kl[i])) for i in sel), Fraction(0)) / len(sel)
+    assert st["mean_kl"] == float(exact)
+    assert st["top1_agree"] == sum(1 for i in sel if ra[i] == ca[i])
+    for t, c in zip(thr, st["exceed"]):
+        assert c == sum(1 for i in sel if kl[i] > np.float32(t))
+    nll_r = float(sum((Fraction(-float(rt[i])) for i in sel), Fraction(0)) / len(sel))
+    assert _close(st["ref_ppl"], math.exp(nll_r), rtol=1e-15)
+
+
+def pin_uniform_perplexity(O):
+    # A uniform reference over V ids has perplexity V.
+    V = 4096
+    res = O.full_vocab(np.zeros((5, V)), np.zeros((5, V)), np.arange(5))
+    st = O.reduce_stats(res["kl"], res["ref_argmax"], res["cand_argmax"], None,
+                        res["ref_target_lp"], res["cand_target_lp"])
+    assert _close(st["ref_ppl"], V, rtol=1e-6)
+    assert st["top1_rate"] == 1.0 and st["ppl_ratio"] == 1.0
+
+
+# ---------------------------------------------------------------------------
+# shared head
+# ---------------------------------------------------------------------------
+
+def pin_shared_head_matmul(O):
+    rng = np.random.default_rng(11)
+    n, K, V = 3, 5, 7
+    H = rng.normal(size=(n, K))
+    W = rng.normal(size=(V, K))
+    L = O.shared_head_logits(H, W)
+    for i in range(n):
+        for v in range(V):
+            acc = 0.0
+            for k in range(K):
+                acc += H[i, k] * W[v, k]
+            assert _close(L[i, v], acc, rtol=1e-12, atol=1e-14)
+    res = O.shared_head(H, H.copy(), W, np.zeros(n, dtype=np.int64), v_chunk=3)
+    assert np.all(res["kl"] == 0.0)
+    res2 = O.shared_head(H, H + 0.1, W, np.zeros(n, dtype=np.int64), v_chunk=3)
+    for i in range(n):
+        assert _close(res2["kl"][i], O.full_vocab_row(H[i] @ W.T, (H[i] + 0.1) @ W.T)["kl"], rtol=1e-12)
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
+
+
+@pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
+def test_pin(pin):
+    pin(ORACLE)
+
+
+def test_golden_bf16_self_scores():
+    """Reference vs itself: mean KLD 0 and top-1 agreement 100% (golden)."""
+    path = os.path.join(ROOT, "tests", "golden", "bf16_self_scores.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    mean_kld, top1 = float(rows[0][0]), float(rows[0][1])
+    rng = np.random.default_rng(12)
+    X = rng.normal(0, 2, (16, 4096))
+    res = ORACLE.full_vocab(X, X.copy(), rng.integers(0, 4096, 16))
+    st = ORACLE.reduce_stats(res["kl"], res["ref_argmax"], res["cand_argmax"])
+    assert st["mean_kl"] == mean_kld and st["top1_rate"] == top1
+    ids = np.stack([rng.permutation(4096)[:64] for _ in range(16)])
+    lp = np.sort(np.log(rng.dirichlet(np.ones(100), 16)[:, :64]), axis=1)[:, ::-1]
+    tr = ORACLE.topk_tail(ids, lp, ids, lp, 4096)
+    st2 = ORACLE.reduce_stats(tr["kl"], top1=tr["top1"])
+    assert st2["mean_kl"] == mean_kld and st2["top1_rate"] == top1
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: each must be caught by at least one pin
+# ---------------------------------------------------------------------------
+
+MUTANTS = [
+    ("KL direction reversed", "terms = p[live] * (lp[live] - lq[live])",
+     "terms = np.exp(lq[live]) * (lq[live] - lp[live])"),
+    ("log-softmax sign", "return z - lse", "return z + lse"),
+    ("normaliser without max", "lse = m + math.log(float(np.sum(np.exp(z - m))))",
+     "lse = math.log(float(np.sum(np.exp(z - m))))"),
+    ("argmax picks the last tie", "out[\"ref_argmax\"] = int(np.argmax(x))",
+     "out[\"ref_argmax\"] = int(x.shape[0] - 1 - np.argmax(x[::-1]))"),
+    ("candidate target from the reference", "out[\"cand_target_lp\"] = float(lq[t])",
+     "out[\"cand_target_lp\"] = float(lp[t])"),
+    ("spread over V instead of V - k", "spread = leftover / (vocab - k)\n    log_spread",
+     "spread = leftover / vocab\n    log_spread"),
+    ("tail term dropped", "kl += p_tail * (math.log(p_tail) - math.log(max(q_tail, Q_FLOOR)))",
+     "kl += 0.0"),
+    ("unmatched ids get the whole leftover", "            q[j] = spread\n            logq[j] = log_spread",
+     "            q[j] = leftover\n            logq[j] = math.log(max(leftover, Q_FLOOR))"),
+    ("q_tail from the reference side", "q_tail = 1.0 - float(np.sum(q))", "q_tail = 1.0 - float(np.sum(p))"),
+    ("percentile index n q", "h = (n - 1) * float(q)", "h = n * float(q) - 0.5"),
+    ("mean over all positions", "out[\"mean_kl\"] = math.fsum(vals.tolist()) / n if n else math.nan",
+     "out[\"mean_kl\"] = math.fsum(vals.tolist()) / max(n_all, 1)"),
+    ("transposed head", "return np.asarray(H, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T",
+     "return (np.asarray(W, dtype=np.float64) @ np.asarray(H, dtype=np.float64).T).T[:, ::-1]"),
+]
+
+
+def _load_mutant(old, new):
+    src = open(ORACLE_SRC).read()
+    assert src.count(old) == 1, f"mutant anchor not unique / missing: {old!r}"
+    spec = importlib.util.spec_from_loader("oracle_mutant", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(name, old, new):
+    mod = _load_mutant(old, new)
+    failures = 0
+    for pin in PINS:
+        try:
+            pin(mod)
+        except Exception:
+            failures += 1
+    assert failures > 0, f"no pin catches: {name}"
