@@ -1,0 +1,414 @@
+"""Throughput of teacher-forced KL scoring on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step scores one window of full-vocabulary logits (2047 positions x
+248,320 vocabulary ids, bf16, seeded synthetic Zipf/Gumbel rows) with
+kld_full_vocab and reduces it with kld_reduce_stats (mean, median, p99,
+p99.9, top-1, perplexity).  Inputs are resident in HBM and larger than L2
+(2.03 GB per step).  With N GPUs (torchrun) every rank scores its own window:
+weak scaling, no collective on the data path; the timing is the max over
+ranks.  Rank 0 prints one JSON line.
+
+--impl reference times the f64 CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "scored positions/sec at V=248,320 (KL+top-1)"
+UNIT = "positions/s"
+N_ROWS = 2047
+VOCAB = 248_320
+QUANTILES = (0.5, 0.99, 0.999)
+WORKLOAD = "one-window full-vocabulary scoring: 2047 positions x 248,320 vocab, bf16 logits"
+PROFILE = os.path.join(ROOT, "profiles", "full_vocab_kernel_window_bf16.txt")
+KERNEL_SOURCES = [os.path.join(ROOT, "quantization_fidelity_scoring_b200", "csrc", f)
+                  for f in ("full_vocab.cu", "kld_common.cuh")]
+
+
+def kernel_digest() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    if not os.path.exists(PROFILE):
+        return None
+    vals = {}
+    for line in open(PROFILE):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_digest") != kernel_digest():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """NVML clock / throttle-reason sampling on a background thread (read only)."""
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples = []  # (t, sm_mhz, reasons_bitmask)
+        self._stop = threading.Event()
+        self._th = None
+        self.max_mhz = None
+        self.ok = False
+
+    def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._th = threading.Thread(target=self._run, daemon=True)
+        self._th.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self._th:
+            self._th.join()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        use = inside if inside else self.samples
+        names = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+        seen = set()
+        for _, _, rs in use:
+            for bit, name in names.items():
+                if rs & bit:
+                    seen.add(name)
+        return {"sm_mhz": statistics.median([s[1] for s in use]) if use else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(seen),
+                "samples_in_timed_region": len(inside), "samples": len(use)}
+
+
+def oracle_rows(ref, cand, targets, rows):
+    """Run the f64 oracle on the given row indices (host copies); returns seconds."""
+    import numpy as np
+    import torch
+    from oracle import kld_oracle as O
+    idx = torch.as_tensor(rows, device=ref.device)
+    X = O.bf16_bits_to_f64(ref[idx].cpu().view(torch.int16).numpy().view(np.uint16))
+    Y = O.bf16_bits_to_f64(cand[idx].cpu().view(torch.int16).numpy().view(np.uint16))
+    T = targets[idx].cpu().numpy()
+    t0 = time.perf_counter()
+    res = O.full_vocab(X, Y, T)
+    O.reduce_stats(res["kl"], res["ref_argmax"], res["cand_argmax"], None, res["ref_target_lp"],
+                   res["cand_target_lp"], quantiles=QUANTILES)
+    return time.perf_counter() - t0
+
+
+def cpu_sample_stats(seconds_per_row: float, rows: int, dt: float) -> dict:
+    return {"value": rows / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of the {N_ROWS} rows of one window (f64 numpy oracle: full-vocabulary "
+                      f"scoring + reductions), single thread; host has {os.cpu_count()} cores"}
+
+
+def run_reference(args) -> int:
+    """Reference arm: the f64 oracle on host cores, bounded samples per step."""
+    import numpy as np
+    import torch
+    from oracle import kld_oracle as O
+    from synth import workloads as W
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    # inputs drawn on the GPU when there is one (same bytes as our arm), else on the host
+    dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
+    budget_s = 90.0
+    per_row_s = 0.02
+    rows_per_step = max(1, min(256, int(budget_s / ((args.steps + args.warmup) * per_row_s))))
+    d = W.window_full_vocab(seed=W.seed_for(2), device=dev, n_rows=min(N_ROWS, max(2 * rows_per_step, 64)))
+    X = O.bf16_bits_to_f64(d["ref"].cpu().view(torch.int16).numpy().view(np.uint16))
+    Y = O.bf16_bits_to_f64(d["cand"].cpu().view(torch.int16).numpy().view(np.uint16))
+    T = d["targets"].cpu().numpy()
+    del d
+
+    def step(i):
+        a = (i * rows_per_step) % (X.shape[0] - rows_per_step + 1)
+        sl = slice(a, a + rows_per_step)
+        res = O.full_vocab(X[sl], Y[sl], T[sl])
+        O.reduce_stats(res["kl"], res["ref_argmax"], res["cand_argmax"], None, res["ref_target_lp"],
+                       res["cand_target_lp"], quantiles=QUANTILES)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    value = rows_per_step * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Zipf/Gumbel logits; no corpus or model)",
+        "config": config_dict(),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{rows_per_step} rows of the window per step, f64 numpy oracle, "
+                                   f"single thread; host has {os.cpu_count()} cores"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict() -> dict:
+    return {"workload": WORKLOAD, "n_rows": N_ROWS, "vocab": VOCAB, "input_dtype": "bf16",
+            "step": "kld_full_vocab + kld_reduce_stats (mean, p50, p99, p99.9, top-1, ppl)",
+            "l2": "inputs larger than L2: 2.03 GB of logits per step",
+            "parallelism": "dp (each rank scores its own window)"}
+
+
+def run_ours(args) -> int:
+    import torch
+    import torch.distributed as dist
+
+    import quantization_fidelity_scoring_b200 as kq
+    from synth import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    kq.load_library()
+
+    d = W.window_full_vocab(seed=W.seed_for(2) + 1000 * rank, device=dev)
+    ref, cand, targets = d["ref"], d["cand"], d["targets"]
+    n = ref.shape[0]
+    stream = torch.cuda.current_stream()
+    kl = torch.empty(n, dtype=torch.float32, device=dev)
+    ra = torch.empty(n, dtype=torch.int32, device=dev)
+    ca = torch.empty(n, dtype=torch.int32, device=dev)
+    lpr = torch.empty(n, dtype=torch.float32, device=dev)
+    lpc = torch.empty(n, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    stats_buf = torch.empty(280, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kq.kld_full_vocab(ref, cand, targets, kl=kl, ref_argmax=ra, cand_argmax=ca, ref_target_lp=lpr,
+                          cand_target_lp=lpc, dev_status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf,
+                            workspace=ws, dev_status=status, stream=stream, to_host=False)
+
+    sampler = ClockSampler(local).start()
+    # warm-up: at least W steps and about a second of load so the clocks settle
+    t_w = time.perf_counter()
+    i = 0
+    while i < args.warmup or time.perf_counter() - t_w < 1.0:
+        step()
+        i += 1
+        if i % 50 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    start.record(stream)
+    for s in range(args.steps):
+        step(kev[s])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ms = start.elapsed_time(stop)
+    k_ms = [a.elapsed_time(b) for a, b in kev]
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    assert status.item() == 0, f"device status {status.item()}"
+
+    positions = n * world * args.steps
+    value = positions / (ms / 1e3)
+
+    # roofline of the dominant kernel (full-vocabulary pass)
+    alg_bytes = 2 * n * VOCAB * 2 + n * (4 + 4 * 5)   # both logit rows, targets, five outputs
+    k_avg_s = statistics.mean(k_ms) / 1e3
+    achieved = alg_bytes / k_avg_s / 1e9
+    peak, peak_kind = measured_peaks()
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(),
+                "kernel": "kld::full_vocab_kernel<bf16>", "kernel_ms": statistics.mean(k_ms),
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s"}
+
+    e2e = measure_e2e(args, kq, d, dev, world)
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded Zipf/Gumbel logits; no corpus or model)",
+            "config": config_dict(), "roofline": roofline,
+            "clocks": sampler.summary(t0, t1), "gpu_launches": 2 * args.steps, "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            rows = list(range(0, n, max(1, n // args.cpu_rows)))[:args.cpu_rows]
+            dt = oracle_rows(ref, cand, targets, rows)
+            line["cpu_baseline"] = cpu_sample_stats(dt / len(rows), len(rows), dt)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_e2e(args, kq, d, dev, world) -> dict:
+    """The same step from pinned host buffers: per step the logits and targets
+    are copied host -> device in row chunks on a copy stream, overlapped with
+    scoring of the previous chunk, and the stats struct is read back."""
+    import torch
+    import torch.distributed as dist
+    n = d["ref"].shape[0]
+    chunk = 256
+    h_ref = d["ref"].cpu().pin_memory()
+    h_cand = d["cand"].cpu().pin_memory()
+    h_t = d["targets"].cpu().pin_memory()
+    d_ref = torch.empty_like(d["ref"])
+    d_cand = torch.empty_like(d["cand"])
+    d_t = torch.empty_like(d["targets"])
+    kl = torch.empty(n, dtype=torch.float32, device=dev)
+    ra = torch.empty(n, dtype=torch.int32, device=dev)
+    ca = torch.empty(n, dtype=torch.int32, device=dev)
+    lpr = torch.empty(n, dtype=torch.float32, device=dev)
+    lpc = torch.empty(n, dtype=torch.float32, device=dev)
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    stats_buf = torch.empty(280, dtype=torch.uint8, device=dev)
+    h_stats = torch.empty(280, dtype=torch.uint8).pin_memory()
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=dev)
+    chunks = [(a, min(n, a + chunk)) for a in range(0, n, chunk)]
+
+    def step():
+        evs = []
+        with torch.cuda.stream(copy):
+            for a, b in chunks:
+                d_ref[a:b].copy_(h_ref[a:b], non_blocking=True)
+                d_cand[a:b].copy_(h_cand[a:b], non_blocking=True)
+                d_t[a:b].copy_(h_t[a:b], non_blocking=True)
+                e = torch.cuda.Event()
+                e.record(copy)
+                evs.append(e)
+        for (a, b), e in zip(chunks, evs):
+            comp.wait_event(e)
+            kq.kld_full_vocab(d_ref[a:b], d_cand[a:b], d_t[a:b], kl=kl[a:b], ref_argmax=ra[a:b],
+                              cand_argmax=ca[a:b], ref_target_lp=lpr[a:b], cand_target_lp=lpc[a:b],
+                              stream=comp)
+        kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf, workspace=ws,
+                            stream=comp, to_host=False)
+        h_stats.copy_(stats_buf, non_blocking=True)
+        comp.synchronize()
+
+    steps = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(3):
+        step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = time.perf_counter() - t0
+    if world > 1:
+        tt = torch.tensor([dt], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        dt = float(tt.item())
+    h2d = h_ref.numel() * 2 + h_cand.numel() * 2 + h_t.numel() * 4
+    return {"value": n * world * steps / dt, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": 280, "steps": steps,
+            "how": "pinned host logits copied in 256-row chunks on a copy stream, overlapped with "
+                   "scoring of earlier chunks; stats struct read back each step; wall clock"}
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,219 @@
+/*
+ * kld.h - C ABI of libkld: teacher-forced KL(reference || candidate) scoring
+ * of next-token distributions on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (sources are web pages, cited by title and section):
+ *
+ *  - Per scored position, KL(p || q) = sum_i p_i (log p_i - log q_i) where p
+ *    and q are the softmax of the reference and candidate logits over the
+ *    whole vocabulary ("Qwen3.8-27B Quantization Challenge", sections "How
+ *    the references were made" and "The score"), the exact argmax of each
+ *    side for top-1 agreement and the log-probability of the true next token
+ *    for perplexity ("Qwopus3.8-27B-Coder-Flash: quality-eval reference",
+ *    section "Method").
+ *  - The top-64 + one tail bucket approximation of that KL from stored top-k
+ *    lists ("Qwopus3.8-27B-Coder-Flash: quality-eval reference", "Method"
+ *    and "Files").
+ *  - The same full-vocabulary scores from final hidden states pushed through
+ *    one shared BF16 LM head ("Qwen3.8-27B fidelity suite v5", opening
+ *    paragraph).
+ *  - Mean / percentile / top-1 / perplexity / exceedance reductions
+ *    ("Qwen3.8-27B Quantization Challenge", "The score"; "Qwen3.8-27B IQ8R
+ *    ... radiance container", "Quality"; "Qwen3.8-27B fidelity suite v5",
+ *    "What is in here").
+ *
+ * Conventions shared by every entry point:
+ *
+ *  - Memory.  Every pointer argument is a DEVICE pointer unless its comment
+ *    says "host".  The caller owns all memory; the library allocates nothing
+ *    and keeps no state between calls.
+ *  - Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *    default stream).  Every call only enqueues work on that stream and
+ *    returns without synchronising.
+ *  - Errors detectable on the host (bad sizes, null or misaligned pointers,
+ *    unsupported dtype, workspace too small) are returned synchronously and
+ *    nothing is launched.  KLD_ERR_CUDA means a CUDA launch failed; the
+ *    stream may then hold partial results.
+ *  - Errors found on the device are OR-ed into *dev_status as KLD_DEV_* bits
+ *    (dev_status may be NULL to ignore them).  The caller zeroes the word
+ *    before the call and reads it after synchronising.  The library never
+ *    traps or asserts on the device.
+ *  - Determinism.  For a given shape every output is bitwise identical from
+ *    run to run: all reductions use fixed trees and fixed orders, never
+ *    floating-point atomics.
+ *  - Thread safety.  Calls are reentrant; concurrent calls on different
+ *    streams must not share output, workspace or dev_status buffers.
+ */
+#ifndef KLD_H_
+#define KLD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kld_status {
+  KLD_OK = 0,
+  KLD_ERR_INVALID_ARG = 1, /* null required pointer, bad size or bad combination */
+  KLD_ERR_ALIGNMENT = 2,   /* a pointer or leading dimension breaks the alignment rules */
+  KLD_ERR_UNSUPPORTED = 3, /* dtype or size outside what the kernels implement */
+  KLD_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than the *_workspace_size query */
+  KLD_ERR_CUDA = 5         /* a CUDA runtime call or kernel launch failed */
+} kld_status;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define KLD_DEV_BAD_TARGET 0x1 /* a target id was outside [0, vocab): that row's target lps are NaN */
+#define KLD_DEV_BAD_ID 0x2     /* a top-k id was outside [0, vocab): that row's KL is NaN */
+#define KLD_DEV_TIMEOUT 0x4    /* a bounded wait inside a kernel gave up; outputs are invalid */
+
+typedef enum kld_dtype {
+  KLD_F32 = 0,  /* IEEE binary32 logits */
+  KLD_BF16 = 1  /* bfloat16 logits (upper half of a binary32) */
+} kld_dtype;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int kld_version(void);
+
+/* Static, NUL-terminated description of a status code. */
+const char* kld_status_string(kld_status s);
+
+/*
+ * kld_full_vocab - full-vocabulary scoring of n_rows positions.
+ *
+ * Defines ("Qwen3.8-27B Quantization Challenge", "How the references were
+ * made" / "The score"; "Qwopus3.8-27B-Coder-Flash: quality-eval reference",
+ * "Method"): for row r with reference logits x = ref_logits[r, 0:vocab] and
+ * candidate logits y = cand_logits[r, 0:vocab], p = softmax(x),
+ * q = softmax(y), computed in f32 arithmetic (f64 for the final per-row
+ * combination):
+ *    kl[r]             = sum_i p_i (log p_i - log q_i)        (nats)
+ *    ref_argmax[r]     = lowest i with x_i = max x   (cand_argmax: same on y)
+ *    ref_target_lp[r]  = log p_t,  cand_target_lp[r] = log q_t,  t = target_ids[r]
+ *
+ * Each logit is read from HBM exactly once (single streaming pass).
+ *
+ * Arguments:
+ *   ref_logits, cand_logits  [n_rows, ld_*] row-major, element type `dtype`.
+ *                            16-byte aligned; ld_* * sizeof(element) must be
+ *                            a multiple of 16 bytes, ld_* >= vocab.
+ *   n_rows                   >= 0 (0 launches nothing).
+ *   vocab                    1 .. 2^31 - 1.
+ *   target_ids               int32 [n_rows], or NULL.  When NULL both
+ *                            *_target_lp outputs must be NULL.
+ *   kl                       f32 [n_rows], required.
+ *   ref_argmax, cand_argmax  int32 [n_rows], each may be NULL.
+ *   ref_target_lp, cand_target_lp  f32 [n_rows], each may be NULL.
+ *   dev_status               int32 device word, may be NULL.
+ *
+ * Non-finite input: -inf logits are allowed (an id with p_i = 0 contributes
+ * nothing; p_i > 0 against a candidate -inf gives kl = +inf).  A row holding
+ * NaN or +inf, or no finite logit, gives kl = NaN, argmax = -1 and NaN
+ * target lps.  A target id outside [0, vocab) gives NaN target lps and sets
+ * KLD_DEV_BAD_TARGET.
+ */
+kld_status kld_full_vocab(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
+                          int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
+                          const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                          int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
+                          int32_t* dev_status, void* stream);
+
+/*
+ * kld_topk_tail - KL over the reference's top-k ids plus one tail bucket.
+ *
+ * Defines ("Qwopus3.8-27B-Coder-Flash: quality-eval reference", "Method";
+ * list layout from "Files"): per position, with reference list (R ids,
+ * log-probs a_j) and candidate list (C ids, log-probs b_s), k entries each,
+ * both sorted by descending probability:
+ *    c_s      = exp(b_s);  leftover = max(0, 1 - sum_s c_s)
+ *    spread   = leftover / (vocab - k)          (mass of each id outside C)
+ *    q_j      = c_s and log q_j = b_s   if R_j = C_s (first such s)
+ *             = spread, log q_j = log max(spread, 1e-12)   otherwise
+ *    p_j      = exp(a_j);  p_tail = 1 - sum_j p_j;  q_tail = 1 - sum_j q_j
+ *    kl       = sum_j p_j (a_j - log q_j)
+ *             + [p_tail > 0] p_tail (log p_tail - log max(q_tail, 1e-12))
+ *    top1     = (R_0 == C_0)
+ * The two mass sums are accumulated in f64.
+ *
+ * Arguments:
+ *   ref_ids, cand_ids    int32 [n_rows, k] row-major (row stride k), ids in [0, vocab).
+ *   ref_lp, cand_lp      IEEE binary16 bit patterns [n_rows, k] (row stride k).
+ *   k                    1 .. 64;  vocab: k < vocab < 2^25.
+ *   kl                   f32 [n_rows], required.
+ *   top1                 uint8 [n_rows] (0/1), may be NULL.
+ *   n_matched            int32 [n_rows] (ids of R found in C), may be NULL.
+ * All arrays need only their natural alignment.  An id outside [0, vocab)
+ * makes that row's kl NaN and sets KLD_DEV_BAD_ID.
+ */
+kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp,
+                         const int32_t* cand_ids, const uint16_t* cand_lp,
+                         int64_t n_rows, int32_t k, int64_t vocab,
+                         float* kl, uint8_t* top1, int32_t* n_matched,
+                         int32_t* dev_status, void* stream);
+
+/*
+ * Result of kld_reduce_stats, written to DEVICE memory.  Plain C layout:
+ * 8-byte fields first, then 4-byte fields; sizeof = 360 on LP64.
+ */
+#define KLD_MAX_QUANTILES 8
+#define KLD_MAX_THRESHOLDS 8
+typedef struct kld_stats {
+  int64_t n;                 /* positions scored: mask set and kl not NaN */
+  int64_t n_nan;             /* masked-in positions whose kl is NaN (excluded) */
+  int64_t top1_agree;        /* agreeing scored positions, -1 if no agreement input */
+  int64_t exceed[KLD_MAX_THRESHOLDS]; /* count of scored kl > thresholds[i] (f32 compare) */
+  double mean_kl;            /* sum of scored kl / n (NaN if n == 0) */
+  double top1_rate;          /* top1_agree / n (NaN if unavailable) */
+  double ref_mean_nll, cand_mean_nll; /* mean of -target lp over scored positions (NaN if absent) */
+  double ref_ppl, cand_ppl;  /* exp(mean NLL) */
+  double ppl_ratio;          /* cand_ppl / ref_ppl */
+  double q_value[KLD_MAX_QUANTILES]; /* linear-interpolated percentile of scored kl */
+  float q_lo[KLD_MAX_QUANTILES];     /* order statistic s[floor((n-1) q)] */
+  float q_hi[KLD_MAX_QUANTILES];     /* order statistic s[min(floor((n-1) q) + 1, n - 1)] */
+  int32_t nq, nt;            /* echo of the counts requested */
+} kld_stats;
+
+/* Workspace bytes kld_reduce_stats needs for n positions. */
+size_t kld_reduce_workspace_size(int64_t n);
+
+/*
+ * kld_reduce_stats - leaderboard reductions over per-position results.
+ *
+ * Defines ("Qwen3.8-27B Quantization Challenge", "The score": mean KL
+ * ranks, median / p99 / p99.9, top-1 agreement, perplexity ratio;
+ * "Qwen3.8-27B fidelity suite v5", "What is in here": percentiles and exact
+ * exceedance counts; "Qwopus3.8-27B-Coder-Flash: quality-eval reference",
+ * "Method": perplexity = exp(mean NLL)).  Scored positions are those with
+ * mask[i] != 0 (all when mask is NULL) and kl[i] not NaN.  Percentile q uses
+ * linear interpolation, h = (n - 1) q:
+ *    q_value = s[lo] + (s[hi] - s[lo]) (h - lo),  lo = floor h, hi = min(lo + 1, n - 1)
+ * over the ascending scored kl values s; both order statistics are exact
+ * (radix select on the f32 bit patterns).  Sums are f64 in a fixed order.
+ *
+ * Arguments:
+ *   kl                         f32 [n], required.
+ *   ref_argmax, cand_argmax    int32 [n]: agreement = (ref == cand && ref >= 0);
+ *                              both or neither.
+ *   top1                       uint8 [n] agreement flags; used when the argmax
+ *                              pair is NULL.  All three NULL: top1_agree = -1.
+ *   ref_target_lp, cand_target_lp  f32 [n] each, may be NULL.
+ *   mask                       uint8 [n] or NULL.
+ *   n                          0 .. 2^31 - 1.
+ *   quantiles                  HOST double[nq], each in [0, 1]; nq 0 .. 8.
+ *   thresholds                 HOST float[nt]; nt 0 .. 8.
+ *   out                        DEVICE kld_stats*, 8-byte aligned.
+ *   workspace                  DEVICE, >= kld_reduce_workspace_size(n) bytes, 256-byte aligned.
+ */
+kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
+                            const uint8_t* top1, const float* ref_target_lp,
+                            const float* cand_target_lp, const uint8_t* mask, int64_t n,
+                            const double* quantiles, int32_t nq, const float* thresholds,
+                            int32_t nt, kld_stats* out, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KLD_H_ */

@@ -1,0 +1,16 @@
+"""B200-native teacher-forced KL(reference || candidate) scoring.
+
+The compute lives in libkld.so (hand-written sm_100a kernels behind the C ABI
+of include/kld.h); this package is its Python binding.
+"""
+from . import _lib
+from .api import (KldError, kld_full_vocab, kld_reduce_stats, kld_reduce_workspace_size,
+                  kld_topk_tail, stats_to_dict)
+
+__all__ = ["KldError", "kld_full_vocab", "kld_topk_tail", "kld_reduce_stats",
+           "kld_reduce_workspace_size", "stats_to_dict", "load_library"]
+
+
+def load_library():
+    """Load libkld.so (raises ImportError when it has not been built)."""
+    return _lib.load()

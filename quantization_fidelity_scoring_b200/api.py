@@ -1,0 +1,170 @@
+"""Python binding of libkld: torch tensors in, C ABI call, tensors out.
+
+Argument marshalling only.  Every number is computed by the CUDA kernels
+behind the C ABI (include/kld.h); torch provides device memory and the
+current stream.  Functions carry the C names.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+
+class KldError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _lib.load()
+        msg = lib.kld_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != _lib.KLD_OK:
+        raise KldError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(name, t, dtype=None, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D")
+
+
+def _out(t, n, dtype, device):
+    return torch.empty(n, dtype=dtype, device=device) if t is None else t
+
+
+_DTYPES = {torch.float32: _lib.KLD_F32, torch.bfloat16: _lib.KLD_BF16}
+
+
+def kld_full_vocab(ref: torch.Tensor, cand: torch.Tensor, targets: torch.Tensor | None = None, *,
+                   argmax: bool = True, kl=None, ref_argmax=None, cand_argmax=None,
+                   ref_target_lp=None, cand_target_lp=None, dev_status=None, stream=None,
+                   ctas_per_row: int = 0) -> dict:
+    """Full-vocabulary KL / argmax / target log-probs of [n, V] logit rows
+    (f32 or bf16, unit stride along V).  Outputs are allocated when not
+    given.  ctas_per_row forces the split of a row across CTAs (tests)."""
+    _need_cuda("ref", ref, ndim=2)
+    _need_cuda("cand", cand, ndim=2)
+    if ref.dtype != cand.dtype or ref.dtype not in _DTYPES:
+        raise ValueError("ref and cand must both be float32 or both bfloat16")
+    if ref.shape != cand.shape:
+        raise ValueError("ref and cand shapes differ")
+    if ref.stride(1) != 1 or cand.stride(1) != 1:
+        raise ValueError("logit rows must be contiguous along the vocabulary")
+    n, V = ref.shape
+    dev = ref.device
+    if targets is not None:
+        _need_cuda("targets", targets, torch.int32, 1)
+    kl = _out(kl, n, torch.float32, dev)
+    if argmax:
+        ref_argmax = _out(ref_argmax, n, torch.int32, dev)
+        cand_argmax = _out(cand_argmax, n, torch.int32, dev)
+    if targets is not None:
+        ref_target_lp = _out(ref_target_lp, n, torch.float32, dev)
+        cand_target_lp = _out(cand_target_lp, n, torch.float32, dev)
+    lib = _lib.load()
+    args = (_ptr(ref), _ptr(cand), _DTYPES[ref.dtype], n, V, ref.stride(0), cand.stride(0),
+            _ptr(targets), _ptr(kl), _ptr(ref_argmax), _ptr(cand_argmax), _ptr(ref_target_lp),
+            _ptr(cand_target_lp), _ptr(dev_status), _stream_handle(stream))
+    if ctas_per_row:
+        st = lib.kld_full_vocab_cluster(*args, ctas_per_row)
+    else:
+        st = lib.kld_full_vocab(*args)
+    _check(st, "kld_full_vocab")
+    return dict(kl=kl, ref_argmax=ref_argmax, cand_argmax=cand_argmax,
+                ref_target_lp=ref_target_lp, cand_target_lp=cand_target_lp)
+
+
+def kld_topk_tail(ref_ids, ref_lp, cand_ids, cand_lp, vocab: int, *, kl=None, top1=None,
+                  n_matched=None, want_matched: bool = False, dev_status=None, stream=None) -> dict:
+    """Top-k + tail-bucket KL and top-1 of [..., k] id (int32) / log-prob
+    (float16) lists, contiguous."""
+    for name, t, dt in (("ref_ids", ref_ids, torch.int32), ("cand_ids", cand_ids, torch.int32),
+                        ("ref_lp", ref_lp, torch.float16), ("cand_lp", cand_lp, torch.float16)):
+        _need_cuda(name, t, dt)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.shape != ref_ids.shape:
+            raise ValueError("all four lists must have the same shape")
+    k = ref_ids.shape[-1]
+    n = ref_ids.numel() // k if k else 0
+    dev = ref_ids.device
+    kl = _out(kl, n, torch.float32, dev)
+    top1 = _out(top1, n, torch.uint8, dev)
+    if want_matched:
+        n_matched = _out(n_matched, n, torch.int32, dev)
+    lib = _lib.load()
+    st = lib.kld_topk_tail(_ptr(ref_ids), _ptr(ref_lp), _ptr(cand_ids), _ptr(cand_lp), n, k, vocab,
+                           _ptr(kl), _ptr(top1), _ptr(n_matched), _ptr(dev_status),
+                           _stream_handle(stream))
+    _check(st, "kld_topk_tail")
+    return dict(kl=kl, top1=top1, n_matched=n_matched)
+
+
+def kld_reduce_workspace_size(n: int) -> int:
+    return int(_lib.load().kld_reduce_workspace_size(n))
+
+
+def stats_to_dict(raw: _lib.KldStats) -> dict:
+    d = {f: getattr(raw, f) for f, _ in raw._fields_}
+    for f in ("exceed", "q_value", "q_lo", "q_hi"):
+        d[f] = list(d[f])
+    d["q_value"] = d["q_value"][:raw.nq]
+    d["q_lo"] = d["q_lo"][:raw.nq]
+    d["q_hi"] = d["q_hi"][:raw.nq]
+    d["exceed"] = d["exceed"][:raw.nt]
+    return d
+
+
+def kld_reduce_stats(kl, ref_argmax=None, cand_argmax=None, top1=None, ref_target_lp=None,
+                     cand_target_lp=None, mask=None, quantiles=(0.5, 0.99, 0.999), thresholds=(), *,
+                     out=None, workspace=None, dev_status=None, stream=None, to_host: bool = True):
+    """Mean / percentiles / top-1 / perplexity / exceedance over n positions.
+
+    Returns a dict (synchronising on the copy) when to_host, else the device
+    buffer holding the kld_stats struct."""
+    _need_cuda("kl", kl, torch.float32, 1)
+    n = kl.shape[0]
+    dev = kl.device
+    for name, t, dt in (("ref_argmax", ref_argmax, torch.int32), ("cand_argmax", cand_argmax, torch.int32),
+                        ("top1", top1, torch.uint8), ("ref_target_lp", ref_target_lp, torch.float32),
+                        ("cand_target_lp", cand_target_lp, torch.float32), ("mask", mask, torch.uint8)):
+        _need_cuda(name, t, dt, 1)
+        if t is not None and t.shape[0] != n:
+            raise ValueError(f"{name} length differs from kl")
+    lib = _lib.load()
+    if workspace is None:
+        workspace = torch.empty(lib.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty(ctypes.sizeof(_lib.KldStats), dtype=torch.uint8, device=dev)
+    qs = (ctypes.c_double * max(len(quantiles), 1))(*quantiles)
+    ts = (ctypes.c_float * max(len(thresholds), 1))(*thresholds)
+    st = lib.kld_reduce_stats(_ptr(kl), _ptr(ref_argmax), _ptr(cand_argmax), _ptr(top1),
+                              _ptr(ref_target_lp), _ptr(cand_target_lp), _ptr(mask), n,
+                              ctypes.cast(qs, ctypes.c_void_p), len(quantiles),
+                              ctypes.cast(ts, ctypes.c_void_p), len(thresholds), _ptr(out),
+                              _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                              _stream_handle(stream))
+    _check(st, "kld_reduce_stats")
+    if not to_host:
+        return out
+    host = out.cpu()
+    raw = _lib.KldStats.from_buffer_copy(bytes(host.numpy().tobytes()))
+    return stats_to_dict(raw)

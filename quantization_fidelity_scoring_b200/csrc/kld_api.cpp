@@ -1,0 +1,167 @@
+// C ABI of libkld: argument validation and kernel launch (see include/kld.h).
+//
+// Every check that can be made on the host is made here, before any CUDA
+// call, so that a rejected call launches nothing and needs no device.
+#include <cstdint>
+#include <cstring>
+
+#include <cuda_runtime.h>
+
+#include "../../include/kld.h"
+#include "launch.h"
+
+namespace {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline kld_status cuda_status(cudaError_t e) { return e == cudaSuccess ? KLD_OK : KLD_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int kld_version(void) { return 100; }
+
+const char* kld_status_string(kld_status s) {
+  switch (s) {
+    case KLD_OK: return "ok";
+    case KLD_ERR_INVALID_ARG: return "invalid argument";
+    case KLD_ERR_ALIGNMENT: return "misaligned pointer or leading dimension";
+    case KLD_ERR_UNSUPPORTED: return "unsupported dtype or size";
+    case KLD_ERR_WORKSPACE: return "workspace missing or too small";
+    case KLD_ERR_CUDA: return "CUDA launch or runtime error";
+  }
+  return "unknown status";
+}
+
+static kld_status full_vocab_impl(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
+                                  int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
+                                  const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                                  int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
+                                  int32_t* dev_status, void* stream, int ctas_per_row) {
+  if (dtype != KLD_F32 && dtype != KLD_BF16) return KLD_ERR_UNSUPPORTED;
+  if (n_rows < 0 || vocab < 1 || vocab > INT32_MAX) return KLD_ERR_INVALID_ARG;
+  if (ld_ref < vocab || ld_cand < vocab) return KLD_ERR_INVALID_ARG;
+  if (!target_ids && (ref_target_lp || cand_target_lp)) return KLD_ERR_INVALID_ARG;
+  if (ctas_per_row < 0 || ctas_per_row > 8) return KLD_ERR_INVALID_ARG;
+  if (n_rows == 0) return KLD_OK;
+  if (!ref_logits || !cand_logits || !kl) return KLD_ERR_INVALID_ARG;
+  // one cluster of up to 8 CTAs per row in a 1-D grid
+  if (n_rows > (int64_t)(INT32_MAX / 8)) return KLD_ERR_UNSUPPORTED;
+  const int64_t esize = dtype == KLD_BF16 ? 2 : 4;
+  if (!aligned(ref_logits, 16) || !aligned(cand_logits, 16)) return KLD_ERR_ALIGNMENT;
+  if ((ld_ref * esize) % 16 != 0 || (ld_cand * esize) % 16 != 0) return KLD_ERR_ALIGNMENT;
+  if (!aligned(kl, 4) || !aligned(ref_argmax, 4) || !aligned(cand_argmax, 4) ||
+      !aligned(ref_target_lp, 4) || !aligned(cand_target_lp, 4) || !aligned(target_ids, 4) ||
+      !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+
+  kld::FullVocabArgs a;
+  a.x = ref_logits;
+  a.y = cand_logits;
+  a.bf16 = dtype == KLD_BF16;
+  a.n_rows = n_rows;
+  a.vocab = vocab;
+  a.ld_x = ld_ref;
+  a.ld_y = ld_cand;
+  a.targets = target_ids;
+  a.kl = kl;
+  a.ax = ref_argmax;
+  a.ay = cand_argmax;
+  a.lpx = ref_target_lp;
+  a.lpy = cand_target_lp;
+  a.dev_status = dev_status;
+  a.cluster_override = ctas_per_row;
+  return cuda_status(kld::launch_full_vocab(a, static_cast<cudaStream_t>(stream)));
+}
+
+kld_status kld_full_vocab(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
+                          int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
+                          const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                          int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
+                          int32_t* dev_status, void* stream) {
+  return full_vocab_impl(ref_logits, cand_logits, dtype, n_rows, vocab, ld_ref, ld_cand, target_ids, kl,
+                         ref_argmax, cand_argmax, ref_target_lp, cand_target_lp, dev_status, stream, 0);
+}
+
+// kld_full_vocab with the number of CTAs per row forced to 1..8 (0 = automatic).
+// Exported for tests of the cross-CTA merge; not declared in kld.h.
+kld_status kld_full_vocab_cluster(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
+                                  int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
+                                  const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                                  int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
+                                  int32_t* dev_status, void* stream, int32_t ctas_per_row) {
+  return full_vocab_impl(ref_logits, cand_logits, dtype, n_rows, vocab, ld_ref, ld_cand, target_ids, kl,
+                         ref_argmax, cand_argmax, ref_target_lp, cand_target_lp, dev_status, stream,
+                         ctas_per_row);
+}
+
+kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp, const int32_t* cand_ids,
+                         const uint16_t* cand_lp, int64_t n_rows, int32_t k, int64_t vocab, float* kl,
+                         uint8_t* top1, int32_t* n_matched, int32_t* dev_status, void* stream) {
+  if (n_rows < 0 || k < 1 || k > 64 || vocab <= k || vocab >= (int64_t(1) << 25))
+    return KLD_ERR_INVALID_ARG;
+  if (n_rows == 0) return KLD_OK;
+  if (!ref_ids || !ref_lp || !cand_ids || !cand_lp || !kl) return KLD_ERR_INVALID_ARG;
+  if (n_rows > (int64_t(1) << 40)) return KLD_ERR_UNSUPPORTED;
+  if (!aligned(ref_ids, 4) || !aligned(cand_ids, 4) || !aligned(ref_lp, 2) || !aligned(cand_lp, 2) ||
+      !aligned(kl, 4) || !aligned(n_matched, 4) || !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+  kld::TopkTailArgs a;
+  a.ref_ids = ref_ids;
+  a.ref_lp = ref_lp;
+  a.cand_ids = cand_ids;
+  a.cand_lp = cand_lp;
+  a.n_rows = n_rows;
+  a.k = k;
+  a.vocab = vocab;
+  a.kl = kl;
+  a.top1 = top1;
+  a.n_matched = n_matched;
+  a.dev_status = dev_status;
+  return cuda_status(kld::launch_topk_tail(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kld_reduce_workspace_size(int64_t n) { return kld::reduce_workspace_bytes(n); }
+
+kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
+                            const uint8_t* top1, const float* ref_target_lp,
+                            const float* cand_target_lp, const uint8_t* mask, int64_t n,
+                            const double* quantiles, int32_t nq, const float* thresholds, int32_t nt,
+                            kld_stats* out, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
+  if (n < 0 || n > INT32_MAX) return KLD_ERR_INVALID_ARG;
+  if (nq < 0 || nq > KLD_MAX_QUANTILES || nt < 0 || nt > KLD_MAX_THRESHOLDS) return KLD_ERR_INVALID_ARG;
+  if ((nq > 0 && !quantiles) || (nt > 0 && !thresholds)) return KLD_ERR_INVALID_ARG;
+  if ((ref_argmax == nullptr) != (cand_argmax == nullptr)) return KLD_ERR_INVALID_ARG;
+  if (!out || (n > 0 && !kl)) return KLD_ERR_INVALID_ARG;
+  for (int i = 0; i < nq; ++i)
+    if (!(quantiles[i] >= 0.0 && quantiles[i] <= 1.0)) return KLD_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < kld::reduce_workspace_bytes(n)) return KLD_ERR_WORKSPACE;
+  if (!aligned(out, 8) || !aligned(workspace, 256) || !aligned(kl, 4) || !aligned(ref_argmax, 4) ||
+      !aligned(cand_argmax, 4) || !aligned(ref_target_lp, 4) || !aligned(cand_target_lp, 4) ||
+      !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+  kld::ReduceArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.kl = kl;
+  a.ref_argmax = ref_argmax;
+  a.cand_argmax = cand_argmax;
+  a.top1 = top1;
+  a.ref_lp = ref_target_lp;
+  a.cand_lp = cand_target_lp;
+  a.mask = mask;
+  a.n = n;
+  a.nq = nq;
+  a.nt = nt;
+  for (int i = 0; i < nq; ++i) a.quantiles[i] = quantiles[i];
+  for (int i = 0; i < nt; ++i) a.thresholds[i] = thresholds[i];
+  a.out = out;
+  a.workspace = workspace;
+  a.dev_status = dev_status;
+  return cuda_status(kld::launch_reduce(a, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+static_assert(sizeof(kld_stats) == 280, "kld_stats layout changed: update the Python mirror");

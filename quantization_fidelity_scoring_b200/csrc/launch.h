@@ -1,0 +1,63 @@
+// Internal launcher interface between the C ABI (kld_api.cpp) and the
+// kernels.  Arguments arrive here already validated.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/kld.h"
+
+namespace kld {
+
+struct FullVocabArgs {
+  const void* x;
+  const void* y;
+  bool bf16;
+  int64_t n_rows, vocab, ld_x, ld_y;
+  const int32_t* targets;
+  float* kl;
+  int32_t* ax;
+  int32_t* ay;
+  float* lpx;
+  float* lpy;
+  int32_t* dev_status;
+  int cluster_override;  // 0: choose from the vocabulary size
+};
+cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream);
+
+struct TopkTailArgs {
+  const int32_t* ref_ids;
+  const uint16_t* ref_lp;
+  const int32_t* cand_ids;
+  const uint16_t* cand_lp;
+  int64_t n_rows;
+  int k;
+  int64_t vocab;
+  float* kl;
+  uint8_t* top1;
+  int32_t* n_matched;
+  int32_t* dev_status;
+};
+cudaError_t launch_topk_tail(const TopkTailArgs& a, cudaStream_t stream);
+
+struct ReduceArgs {
+  const float* kl;
+  const int32_t* ref_argmax;
+  const int32_t* cand_argmax;
+  const uint8_t* top1;
+  const float* ref_lp;
+  const float* cand_lp;
+  const uint8_t* mask;
+  int64_t n;
+  int nq, nt;
+  double quantiles[KLD_MAX_QUANTILES];
+  float thresholds[KLD_MAX_THRESHOLDS];
+  kld_stats* out;
+  void* workspace;
+  int32_t* dev_status;
+};
+size_t reduce_workspace_bytes(int64_t n);
+cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream);
+
+}  // namespace kld

@@ -1,0 +1,386 @@
+// Leaderboard reductions over per-position results.
+//
+// "Qwen3.8-27B Quantization Challenge", "The score": mean KL ranks entries;
+// median, p99 and p99.9, top-1 agreement and the perplexity ratio are shown
+// beside it.  "Qwen3.8-27B fidelity suite v5", "What is in here": percentiles
+// and exact exceedance counts.  "Qwopus3.8-27B-Coder-Flash: quality-eval
+// reference", "Method": perplexity = exp(mean NLL of the true next token).
+//
+// Order statistics are exact: the f32 KL bit patterns are mapped to
+// order-preserving 32-bit keys and each requested rank is found by an
+// MSB-first radix select, 8 bits per pass (4 passes), with integer
+// histograms.  Sums are f64 in fixed orders (per-thread strided, then fixed
+// trees), so every output is bitwise reproducible.
+//
+// Small inputs (n <= kSmallN) run in one CTA with shared-memory histograms;
+// larger inputs use a grid of CTAs per pass with global integer histograms.
+#include <math_constants.h>
+
+#include "kld_common.cuh"
+#include "launch.h"
+
+namespace kld {
+namespace {
+
+constexpr int kMaxTargets = 2 * KLD_MAX_QUANTILES;
+constexpr int kBins = 256;
+constexpr int kPasses = 4;
+constexpr int64_t kSmallN = 65536;
+constexpr int kBigThreads = 256;
+constexpr int kMaxBigBlocks = 1024;
+constexpr int kSmallThreads = 1024;
+
+struct Partial {  // per-CTA sums of the first pass
+  double kl, nll_r, nll_c;
+  long long n, n_nan, agree;
+  long long exceed[KLD_MAX_THRESHOLDS];
+};
+
+struct ReduceParams {
+  const float* kl;
+  const int32_t* ra;
+  const int32_t* ca;
+  const uint8_t* top1;
+  const float* lpr;
+  const float* lpc;
+  const uint8_t* mask;
+  long long n;
+  int nq, nt;
+  double q[KLD_MAX_QUANTILES];
+  float thr[KLD_MAX_THRESHOLDS];
+  kld_stats* out;
+  unsigned* hist;     // [kPasses][kMaxTargets][kBins]
+  Partial* partials;  // [gridDim of pass 0]
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ uint32_t f2key(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;  // -0 sorts with +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key2f(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  return __uint_as_float(u);
+}
+
+// Per-target radix-select state, identical in every thread that derives it.
+struct Select {
+  int nt;                      // number of target ranks
+  long long n;                 // scored count
+  uint32_t prefix[kMaxTargets];
+  long long rem[kMaxTargets];  // rank within the current prefix group
+  int uslot[kMaxTargets];      // index of the target's prefix among the unique ones
+  uint32_t uprefix[kMaxTargets];
+  int nu;
+};
+
+__device__ __forceinline__ bool scored(const ReduceParams& p, long long i, float& v) {
+  if (p.mask && !p.mask[i]) return false;
+  v = p.kl[i];
+  return !(v != v);
+}
+
+// Targets from the scored count: for every quantile, the lower and upper
+// order statistic ranks of linear interpolation at h = (n - 1) q.
+__device__ void select_init(Select& s, const ReduceParams& p, long long n) {
+  s.n = n;
+  s.nt = (n > 0) ? 2 * p.nq : 0;
+  for (int i = 0; i < p.nq && n > 0; ++i) {
+    const double h = __dmul_rn((double)(n - 1), p.q[i]);
+    long long lo = (long long)floor(h);
+    if (lo > n - 1) lo = n - 1;
+    if (lo < 0) lo = 0;
+    const long long hi = (lo + 1 < n) ? lo + 1 : n - 1;
+    s.rem[2 * i] = lo;
+    s.rem[2 * i + 1] = hi;
+  }
+  for (int t = 0; t < s.nt; ++t) s.prefix[t] = 0u;
+}
+
+__device__ void select_unique(Select& s) {
+  s.nu = 0;
+  for (int t = 0; t < s.nt; ++t) {
+    int u = 0;
+    while (u < s.nu && s.uprefix[u] != s.prefix[t]) ++u;
+    if (u == s.nu) s.uprefix[s.nu++] = s.prefix[t];
+    s.uslot[t] = u;
+  }
+}
+
+// Advance every target by one 8-bit digit using histogram h[u][bin].
+__device__ void select_step(Select& s, const unsigned* h) {
+  for (int t = 0; t < s.nt; ++t) {
+    const unsigned* row = h + s.uslot[t] * kBins;
+    long long acc = 0;
+    int d = 0;
+    for (; d < kBins; ++d) {
+      const long long c = row[d];
+      if (s.rem[t] < acc + c) break;
+      acc += c;
+    }
+    if (d == kBins) d = kBins - 1;  // unreachable for consistent histograms
+    s.rem[t] -= acc;
+    s.prefix[t] = (s.prefix[t] << 8) | (uint32_t)d;
+  }
+}
+
+// One histogram pass over [begin, end) with stride `stride`, adding into the
+// shared-memory histogram sh[u][bin] for elements whose key matches a unique
+// prefix of this pass.  Pass 0 histograms every scored element.
+__device__ __forceinline__ void hist_pass(const ReduceParams& p, const Select& s, int pass,
+                                          long long begin, long long stride, unsigned* sh) {
+  const int shift = 24 - 8 * pass;
+  for (long long i = begin; i < p.n; i += stride) {
+    float v;
+    if (!scored(p, i, v)) continue;
+    const uint32_t key = f2key(v);
+    const uint32_t digit = (key >> shift) & 0xffu;
+    if (pass == 0) {
+      atomicAdd(&sh[digit], 1u);
+    } else {
+      const uint32_t pre = key >> (shift + 8);
+      for (int u = 0; u < s.nu; ++u) {
+        if (s.uprefix[u] == pre) {
+          atomicAdd(&sh[u * kBins + digit], 1u);
+          break;
+        }
+      }
+    }
+  }
+}
+
+// Pass-0 sums of one thread (fixed stride order).
+__device__ __forceinline__ void thread_sums(const ReduceParams& p, long long begin, long long stride,
+                                            Partial& acc) {
+  acc.kl = acc.nll_r = acc.nll_c = 0.0;
+  acc.n = acc.n_nan = acc.agree = 0;
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) acc.exceed[j] = 0;
+  for (long long i = begin; i < p.n; i += stride) {
+    if (p.mask && !p.mask[i]) continue;
+    const float v = p.kl[i];
+    if (v != v) {
+      ++acc.n_nan;
+      continue;
+    }
+    ++acc.n;
+    acc.kl += (double)v;
+    if (p.lpr) acc.nll_r -= (double)p.lpr[i];
+    if (p.lpc) acc.nll_c -= (double)p.lpc[i];
+    if (p.ra) {
+      const int a = p.ra[i];
+      acc.agree += (a >= 0 && a == p.ca[i]) ? 1 : 0;
+    } else if (p.top1) {
+      acc.agree += p.top1[i] ? 1 : 0;
+    }
+    for (int j = 0; j < p.nt; ++j) acc.exceed[j] += (v > p.thr[j]) ? 1 : 0;
+  }
+}
+
+__device__ __forceinline__ void partial_add(Partial& a, const Partial& b) {
+  a.kl += b.kl;
+  a.nll_r += b.nll_r;
+  a.nll_c += b.nll_c;
+  a.n += b.n;
+  a.n_nan += b.n_nan;
+  a.agree += b.agree;
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) a.exceed[j] += b.exceed[j];
+}
+
+// Fixed-order CTA reduction of per-thread partials: warp butterfly, then the
+// warps in order.  Result valid in thread 0.
+__device__ void block_sum(Partial& acc, Partial* sh_warp) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    Partial o;
+    o.kl = __shfl_down_sync(0xffffffffu, acc.kl, off);
+    o.nll_r = __shfl_down_sync(0xffffffffu, acc.nll_r, off);
+    o.nll_c = __shfl_down_sync(0xffffffffu, acc.nll_c, off);
+    o.n = __shfl_down_sync(0xffffffffu, acc.n, off);
+    o.n_nan = __shfl_down_sync(0xffffffffu, acc.n_nan, off);
+    o.agree = __shfl_down_sync(0xffffffffu, acc.agree, off);
+    for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) o.exceed[j] = __shfl_down_sync(0xffffffffu, acc.exceed[j], off);
+    if (lane < off) partial_add(acc, o);
+  }
+  if (lane == 0) sh_warp[w] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Partial t = sh_warp[0];
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) partial_add(t, sh_warp[i]);
+    acc = t;
+  }
+  __syncthreads();
+}
+
+__device__ void write_stats(const ReduceParams& p, const Partial& tot, const Select& s) {
+  kld_stats st;
+  const long long n = tot.n;
+  const double nan = CUDART_NAN;
+  st.n = n;
+  st.n_nan = tot.n_nan;
+  const bool have_agree = p.ra != nullptr || p.top1 != nullptr;
+  st.top1_agree = have_agree ? tot.agree : -1;
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) st.exceed[j] = (j < p.nt) ? tot.exceed[j] : 0;
+  st.mean_kl = n ? tot.kl / (double)n : nan;
+  st.top1_rate = (have_agree && n) ? (double)tot.agree / (double)n : nan;
+  st.ref_mean_nll = (p.lpr && n) ? tot.nll_r / (double)n : nan;
+  st.cand_mean_nll = (p.lpc && n) ? tot.nll_c / (double)n : nan;
+  st.ref_ppl = exp(st.ref_mean_nll);
+  st.cand_ppl = exp(st.cand_mean_nll);
+  st.ppl_ratio = st.cand_ppl / st.ref_ppl;
+  for (int i = 0; i < KLD_MAX_QUANTILES; ++i) {
+    st.q_value[i] = nan;
+    st.q_lo[i] = st.q_hi[i] = CUDART_NAN_F;
+  }
+  for (int i = 0; i < p.nq && n > 0; ++i) {
+    const float lo = key2f(s.prefix[2 * i]);
+    const float hi = key2f(s.prefix[2 * i + 1]);
+    const double h = __dmul_rn((double)(n - 1), p.q[i]);
+    const double frac = __dsub_rn(h, floor(h));
+    st.q_lo[i] = lo;
+    st.q_hi[i] = hi;
+    st.q_value[i] = __dadd_rn((double)lo, __dmul_rn(__dsub_rn((double)hi, (double)lo), frac));
+  }
+  st.nq = p.nq;
+  st.nt = p.nt;
+  *p.out = st;
+}
+
+// ---------------------------------------------------------------- one CTA
+
+__global__ void __launch_bounds__(kSmallThreads) reduce_small_kernel(const ReduceParams p) {
+  __shared__ unsigned sh[kMaxTargets * kBins];
+  __shared__ Partial sh_warp[kSmallThreads / 32];
+  __shared__ Select sel;
+  __shared__ long long n_scored;
+
+  Partial acc;
+  thread_sums(p, threadIdx.x, blockDim.x, acc);
+  block_sum(acc, sh_warp);
+  if (threadIdx.x == 0) n_scored = acc.n;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    select_init(sel, p, n_scored);
+    select_unique(sel);
+  }
+  __syncthreads();
+  for (int pass = 0; pass < kPasses; ++pass) {
+    for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) sh[i] = 0u;
+    __syncthreads();
+    if (sel.nt > 0) hist_pass(p, sel, pass, threadIdx.x, blockDim.x, sh);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      select_step(sel, sh);
+      select_unique(sel);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) write_stats(p, acc, sel);
+}
+
+// ---------------------------------------------------------------- many CTAs
+
+__global__ void reduce_zero_kernel(unsigned* hist) {
+  for (int i = threadIdx.x; i < kPasses * kMaxTargets * kBins; i += blockDim.x) hist[i] = 0u;
+}
+
+// Rebuild the select state from the histograms of passes < pass.
+__device__ void select_replay(Select& s, const ReduceParams& p, int pass) {
+  long long n = 0;
+  for (int d = 0; d < kBins; ++d) n += p.hist[d];
+  select_init(s, p, n);
+  select_unique(s);
+  for (int q = 0; q < pass; ++q) {
+    select_step(s, p.hist + q * kMaxTargets * kBins);
+    select_unique(s);
+  }
+}
+
+__global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReduceParams p, int pass) {
+  __shared__ unsigned sh[kMaxTargets * kBins];
+  __shared__ Select sel;
+  __shared__ Partial sh_warp[kBigThreads / 32];
+  for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) sh[i] = 0u;
+  if (threadIdx.x == 0) {
+    if (pass == 0) {
+      sel.nt = 1;  // histogram every scored element
+      sel.nu = 0;
+    } else {
+      select_replay(sel, p, pass);
+    }
+  }
+  __syncthreads();
+  const long long begin = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  if (sel.nt > 0) hist_pass(p, sel, pass, begin, stride, sh);
+  if (pass == 0) {
+    Partial acc;
+    thread_sums(p, begin, stride, acc);
+    block_sum(acc, sh_warp);
+    if (threadIdx.x == 0) p.partials[blockIdx.x] = acc;
+  }
+  __syncthreads();
+  unsigned* g = p.hist + pass * kMaxTargets * kBins;
+  const int used = (pass == 0) ? kBins : sel.nu * kBins;
+  for (int i = threadIdx.x; i < used; i += blockDim.x)
+    if (sh[i]) atomicAdd(&g[i], sh[i]);
+}
+
+__global__ void reduce_final_kernel(const ReduceParams p, int n_partials) {
+  if (threadIdx.x != 0) return;
+  Partial tot = p.partials[0];
+  for (int b = 1; b < n_partials; ++b) partial_add(tot, p.partials[b]);
+  Select sel;
+  select_replay(sel, p, kPasses);
+  write_stats(p, tot, sel);
+}
+
+int big_grid(long long n) {
+  long long g = (n + kBigThreads * 8 - 1) / (kBigThreads * 8);
+  if (g < 1) g = 1;
+  if (g > kMaxBigBlocks) g = kMaxBigBlocks;
+  return (int)g;
+}
+
+constexpr size_t kHistBytes = sizeof(unsigned) * kPasses * kMaxTargets * kBins;
+
+}  // namespace
+
+size_t reduce_workspace_bytes(int64_t n) {
+  (void)n;
+  return kHistBytes + sizeof(Partial) * kMaxBigBlocks;
+}
+
+cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
+  ReduceParams p;
+  p.kl = a.kl;
+  p.ra = a.ref_argmax;
+  p.ca = a.cand_argmax;
+  p.top1 = a.top1;
+  p.lpr = a.ref_lp;
+  p.lpc = a.cand_lp;
+  p.mask = a.mask;
+  p.n = a.n;
+  p.nq = a.nq;
+  p.nt = a.nt;
+  for (int i = 0; i < KLD_MAX_QUANTILES; ++i) p.q[i] = a.quantiles[i];
+  for (int i = 0; i < KLD_MAX_THRESHOLDS; ++i) p.thr[i] = a.thresholds[i];
+  p.out = a.out;
+  p.hist = reinterpret_cast<unsigned*>(a.workspace);
+  p.partials = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes);
+  p.dev_status = a.dev_status;
+
+  if (a.n <= kSmallN) {
+    reduce_small_kernel<<<1, kSmallThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+  }
+  const int grid = big_grid(a.n);
+  reduce_zero_kernel<<<1, 1024, 0, stream>>>(p.hist);
+  for (int pass = 0; pass < kPasses; ++pass) reduce_pass_kernel<<<grid, kBigThreads, 0, stream>>>(p, pass);
+  reduce_final_kernel<<<1, 32, 0, stream>>>(p, grid);
+  return cudaGetLastError();
+}
+
+}  // namespace kld

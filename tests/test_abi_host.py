@@ -1,0 +1,122 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/kld.h declares, and rejects bad arguments on the host before any
+CUDA call (so these run on a CPU-only machine)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantization_fidelity_scoring_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kld.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(kld_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from quantization_fidelity_scoring_b200 import build
+        build.build()
+    return _lib.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert {"kld_full_vocab", "kld_topk_tail", "kld_reduce_stats"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in _lib.PROTOTYPES, f"binding lacks a prototype for {name}"
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.kld_status_string(s)
+    assert lib.kld_version() >= 100
+
+
+def test_stats_struct_size_matches_header():
+    assert ctypes.sizeof(_lib.KldStats) == 280
+
+
+A16 = 1 << 20          # a fake, 16-byte aligned "device" address; never dereferenced
+MIS = A16 + 4          # 4-byte aligned only
+
+
+def fv(lib, **kw):
+    a = dict(ref=A16, cand=A16 + 4096, dtype=_lib.KLD_BF16, n=4, V=64, ldr=64, ldc=64, tgt=None,
+             kl=A16 + 8192, ra=None, ca=None, lpr=None, lpc=None, st=None)
+    a.update(kw)
+    return lib.kld_full_vocab(a["ref"], a["cand"], a["dtype"], a["n"], a["V"], a["ldr"], a["ldc"],
+                              a["tgt"], a["kl"], a["ra"], a["ca"], a["lpr"], a["lpc"], a["st"], None)
+
+
+def test_full_vocab_validation(lib):
+    assert fv(lib, dtype=7) == _lib.KLD_ERR_UNSUPPORTED
+    assert fv(lib, n=-1) == _lib.KLD_ERR_INVALID_ARG
+    assert fv(lib, V=0) == _lib.KLD_ERR_INVALID_ARG
+    assert fv(lib, ldr=32) == _lib.KLD_ERR_INVALID_ARG
+    assert fv(lib, ref=None) == _lib.KLD_ERR_INVALID_ARG
+    assert fv(lib, kl=None) == _lib.KLD_ERR_INVALID_ARG
+    assert fv(lib, lpr=A16) == _lib.KLD_ERR_INVALID_ARG          # target lp without target ids
+    assert fv(lib, ref=MIS) == _lib.KLD_ERR_ALIGNMENT
+    assert fv(lib, ldr=68, V=64) == _lib.KLD_ERR_ALIGNMENT        # 136 B rows
+    assert fv(lib, dtype=_lib.KLD_F32, ldr=66) == _lib.KLD_ERR_ALIGNMENT
+    assert fv(lib, kl=A16 + 2) == _lib.KLD_ERR_ALIGNMENT
+    assert fv(lib, n=0) == _lib.KLD_OK                            # nothing to launch
+    assert fv(lib, n=0, ref=None, cand=None, kl=None) == _lib.KLD_OK
+    st = lib.kld_full_vocab_cluster(A16, A16, _lib.KLD_BF16, 4, 64, 64, 64, None, A16, None, None,
+                                    None, None, None, None, 9)
+    assert st == _lib.KLD_ERR_INVALID_ARG
+
+
+def tk(lib, **kw):
+    a = dict(ri=A16, rl=A16 + 4096, ci=A16 + 8192, cl=A16 + 12288, n=3, k=64, V=1000, kl=A16 + 16384,
+             t1=None, nm=None, st=None)
+    a.update(kw)
+    return lib.kld_topk_tail(a["ri"], a["rl"], a["ci"], a["cl"], a["n"], a["k"], a["V"], a["kl"],
+                             a["t1"], a["nm"], a["st"], None)
+
+
+def test_topk_validation(lib):
+    assert tk(lib, k=0) == _lib.KLD_ERR_INVALID_ARG
+    assert tk(lib, k=65) == _lib.KLD_ERR_INVALID_ARG
+    assert tk(lib, V=64) == _lib.KLD_ERR_INVALID_ARG              # vocab must exceed k
+    assert tk(lib, V=1 << 25) == _lib.KLD_ERR_INVALID_ARG
+    assert tk(lib, n=-3) == _lib.KLD_ERR_INVALID_ARG
+    assert tk(lib, ci=None) == _lib.KLD_ERR_INVALID_ARG
+    assert tk(lib, ri=A16 + 2) == _lib.KLD_ERR_ALIGNMENT
+    assert tk(lib, rl=A16 + 1) == _lib.KLD_ERR_ALIGNMENT
+    assert tk(lib, n=0) == _lib.KLD_OK
+
+
+def rd(lib, **kw):
+    a = dict(kl=A16, ra=None, ca=None, t1=None, lr=None, lc=None, m=None, n=100, q=(0.5,), t=(),
+             out=A16 + 4096, ws=A16 + 65536, wsb=None, st=None)
+    a.update(kw)
+    qs = (ctypes.c_double * max(8, len(a["q"])))(*a["q"])
+    ts = (ctypes.c_float * 8)(*a["t"])
+    wsb = lib.kld_reduce_workspace_size(a["n"]) if a["wsb"] is None else a["wsb"]
+    return lib.kld_reduce_stats(a["kl"], a["ra"], a["ca"], a["t1"], a["lr"], a["lc"], a["m"], a["n"],
+                                ctypes.cast(qs, ctypes.c_void_p), len(a["q"]),
+                                ctypes.cast(ts, ctypes.c_void_p), len(a["t"]), a["out"], a["ws"], wsb,
+                                a["st"], None)
+
+
+def test_reduce_validation(lib):
+    assert rd(lib, q=(1.5,)) == _lib.KLD_ERR_INVALID_ARG
+    assert rd(lib, q=(-0.1,)) == _lib.KLD_ERR_INVALID_ARG
+    assert rd(lib, q=tuple([0.5] * 9)) == _lib.KLD_ERR_INVALID_ARG
+    assert rd(lib, ra=A16) == _lib.KLD_ERR_INVALID_ARG            # argmax pair incomplete
+    assert rd(lib, out=None) == _lib.KLD_ERR_INVALID_ARG
+    assert rd(lib, n=-1) == _lib.KLD_ERR_INVALID_ARG
+    assert rd(lib, ws=None) == _lib.KLD_ERR_WORKSPACE
+    assert rd(lib, wsb=16) == _lib.KLD_ERR_WORKSPACE
+    assert rd(lib, ws=A16 + 128) == _lib.KLD_ERR_ALIGNMENT
+    assert rd(lib, out=A16 + 4) == _lib.KLD_ERR_ALIGNMENT

@@ -1,0 +1,191 @@
+"""Full-vocabulary scoring on the GPU against the f64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import quantization_fidelity_scoring_b200 as kq
+from oracle import kld_oracle as O
+from synth import workloads as W
+from tests.helpers import assert_kl_close, assert_lp_close, check_full_vocab, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def run(ref, cand, targets=None, **kw):
+    st = torch.zeros(1, dtype=torch.int32, device=ref.device)
+    res = kq.kld_full_vocab(ref, cand, targets, dev_status=st, **kw)
+    torch.cuda.synchronize()
+    res["status"] = int(st.item())
+    return res
+
+
+def ragged(seed, device, n_rows, vocab, dtype, sigma=0.05):
+    """Rows of `vocab` logits in storage padded to a 16-byte row stride."""
+    per16 = 8 if dtype == torch.bfloat16 else 4
+    ld = -(-vocab // per16) * per16
+    d = W.window_full_vocab(seed=seed, device=device, n_rows=n_rows, vocab=ld, dtype=dtype, sigma=sigma)
+    tg = torch.remainder(d["targets"], vocab).to(torch.int32)
+    return d["ref"][:, :vocab], d["cand"][:, :vocab], tg
+
+
+def test_tiny_planted_peak(cuda_device):
+    d = W.top1_planted_tiny(device=cuda_device)
+    res = run(d["ref"], d["cand"], d["targets"])
+    assert res["status"] == 0
+    check_full_vocab(res, to_f64(d["ref"]), to_f64(d["cand"]), d["targets"].cpu().numpy())
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("vocab", [1, 3, 7, 8, 9, 4096 + 8, 4099, 40_003, 262_147])
+def test_ragged_vocab(cuda_device, dtype, vocab):
+    ref, cand, tg = ragged(W.SEED_BASE + 100 + vocab, cuda_device, 37, vocab, dtype)
+    res = run(ref, cand, tg)
+    check_full_vocab(res, to_f64(ref), to_f64(cand), tg.cpu().numpy())
+
+
+@pytest.mark.parametrize("ctas", [1, 2, 3, 5, 8])
+def test_cta_split_and_padded_rows(cuda_device, ctas):
+    V, ld = 30_011, 30_016
+    d = W.window_full_vocab(seed=W.SEED_BASE + 200, device=cuda_device, n_rows=21, vocab=ld,
+                            dtype=torch.bfloat16, sigma=0.03)
+    ref, cand = d["ref"][:, :V], d["cand"][:, :V]
+    tg = torch.remainder(d["targets"], V).to(torch.int32)
+    res = run(ref, cand, tg, ctas_per_row=ctas)
+    check_full_vocab(res, to_f64(ref), to_f64(cand), tg.cpu().numpy())
+
+
+def test_one_window_bf16_full_size(cuda_device):
+    """One scored window (2047 x 248,320, bf16): every row against the oracle."""
+    d = W.window_full_vocab(device=cuda_device)
+    res = run(d["ref"], d["cand"], d["targets"])
+    assert res["status"] == 0
+    X, Y = to_f64(d["ref"]), to_f64(d["cand"])
+    check_full_vocab(res, X, Y, d["targets"].cpu().numpy())
+
+
+def test_batched_f32_full_size_sampled(cuda_device):
+    """16 windows x 2047 rows of f32 logits (65 GB): 192 seeded rows plus every
+    row whose candidate argmax was forced to differ, against the oracle."""
+    d = W.batched_full_vocab(device=cuda_device)
+    res = run(d["ref"], d["cand"], d["targets"])
+    assert res["status"] == 0
+    n = d["ref"].shape[0]
+    g = torch.Generator().manual_seed(7)
+    rows = torch.randperm(n, generator=g)[:192]
+    rows = torch.unique(torch.cat([rows, d["forced_rows"].cpu(), torch.tensor([0, n - 1])])).numpy()
+    X = to_f64(d["ref"][torch.as_tensor(rows, device=cuda_device)])
+    Y = to_f64(d["cand"][torch.as_tensor(rows, device=cuda_device)])
+    T = d["targets"].cpu().numpy()[rows]
+    check_full_vocab(res, X, Y, T, rows=rows)
+    forced = d["forced_rows"].cpu().numpy()
+    ra = res["ref_argmax"].cpu().numpy()
+    ca = res["cand_argmax"].cpu().numpy()
+    assert np.all(ra[forced] != ca[forced])
+    # every KL is finite and non-negative up to the tolerance, at full size
+    kl = res["kl"].cpu().numpy()
+    assert np.all(np.isfinite(kl)) and kl.min() >= -1e-5
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_identical_inputs_give_exact_zero(cuda_device, dtype):
+    ref, _, tg = ragged(W.SEED_BASE + 300, cuda_device, 64, 100_003, dtype)
+    for ctas in (0, 1, 3, 8):
+        res = run(ref, ref.clone(), tg, ctas_per_row=ctas)
+        assert torch.all(res["kl"] == 0.0)
+        assert torch.equal(res["ref_argmax"], res["cand_argmax"])
+        assert torch.equal(res["ref_target_lp"], res["cand_target_lp"])
+
+
+def test_deterministic(cuda_device):
+    d = W.window_full_vocab(seed=W.SEED_BASE + 400, device=cuda_device, n_rows=300, vocab=W.VOCAB)
+    outs = [run(d["ref"], d["cand"], d["targets"]) for _ in range(3)]
+    for o in outs[1:]:
+        for k in ("kl", "ref_argmax", "cand_argmax", "ref_target_lp", "cand_target_lp"):
+            assert torch.equal(o[k], outs[0][k]), k
+
+
+def test_closed_forms_on_gpu(cuda_device):
+    V = 248_320
+    # one-hot vs uniform: KL = ln V
+    x = torch.full((2, V), -math.inf, device=cuda_device)
+    x[0, 12345] = 0.0
+    x[1, V - 1] = 3.0
+    y = torch.zeros((2, V), device=cuda_device)
+    t = torch.tensor([12345, 5], dtype=torch.int32, device=cuda_device)
+    res = run(x, y, t)
+    assert abs(res["kl"][0].item() - math.log(V)) <= 1e-5 + 1e-3 * math.log(V)
+    assert res["ref_argmax"].tolist() == [12345, V - 1]
+    assert res["cand_argmax"].tolist() == [0, 0]
+    assert res["ref_target_lp"][0].item() == 0.0
+    assert math.isinf(res["ref_target_lp"][1].item())      # p_t = 0 exactly
+    assert abs(res["cand_target_lp"][0].item() + math.log(V)) <= 1e-5 * math.log(V)
+    # ties: lowest index wins
+    x = torch.zeros((1, 1000), device=cuda_device)
+    x[0, [17, 400, 999]] = 5.0
+    res = run(x, x.flip(1).contiguous())
+    assert res["ref_argmax"].item() == 17 and res["cand_argmax"].item() == 0
+
+
+def test_non_finite_rows(cuda_device):
+    V = 5000
+    rng = np.random.default_rng(3)
+    X = rng.normal(0, 2, (8, V)).astype(np.float32)
+    Y = (X + rng.normal(0, 0.1, (8, V))).astype(np.float32)
+    X[0, 17] = np.nan                       # NaN in the reference
+    Y[1, 4000] = np.nan                     # NaN in the candidate
+    X[2, 5] = np.inf                        # +inf
+    X[3, :] = -np.inf                       # no finite reference logit
+    X[4, :2500] = -np.inf                   # masked reference ids
+    Y[4, :100] = -np.inf                    # ... also masked in the candidate
+    Y[5, int(np.argmax(X[5]))] = -np.inf    # candidate gives zero mass to the top id
+    X[6, :4990] = -np.inf                   # leading -inf run in every thread's first chunk
+    Y[6, :4990] = -np.inf
+    ref = torch.tensor(X, device=cuda_device)
+    cand = torch.tensor(Y, device=cuda_device)
+    tg = torch.tensor([0, 1, 2, 3, 4000, 6, 4995, -1], dtype=torch.int32, device=cuda_device)
+    res = run(ref, cand, tg)
+    assert res["status"] & 0x1                              # target -1 reported
+    want = O.full_vocab(X.astype(np.float64), Y.astype(np.float64), None)
+    assert_kl_close(res["kl"].cpu().numpy(), want["kl"])
+    assert np.array_equal(res["ref_argmax"].cpu().numpy(), want["ref_argmax"])
+    assert np.array_equal(res["cand_argmax"].cpu().numpy(), want["cand_argmax"])
+    assert math.isnan(res["ref_target_lp"][7].item())
+    for r in (0, 1, 2, 3):
+        assert res["ref_argmax"][r].item() == -1 and math.isnan(res["kl"][r].item())
+    assert res["kl"][5].item() == math.inf
+
+
+def test_bad_target_reported(cuda_device):
+    d = W.window_full_vocab(seed=W.SEED_BASE + 500, device=cuda_device, n_rows=4, vocab=1000)
+    tg = torch.tensor([0, 999, 1000, -5], dtype=torch.int32, device=cuda_device)
+    res = run(d["ref"], d["cand"], tg)
+    assert res["status"] == 0x1
+    lp = res["ref_target_lp"].cpu().numpy()
+    assert np.isfinite(lp[:2]).all() and np.isnan(lp[2:]).all()
+    assert torch.isfinite(res["kl"]).all()
+
+
+def test_near_certain_target_relative_error(cuda_device):
+    """A near-certain token: log p_t ~ -1e-6 must still be within 1e-5 relative."""
+    V = 248_320
+    rng = np.random.default_rng(5)
+    X = rng.normal(-30, 1, (4, V)).astype(np.float32)
+    X[:, 99] = 0.0
+    Y = (X + rng.normal(0, 0.01, (4, V))).astype(np.float32)
+    ref = torch.tensor(X, device=cuda_device)
+    cand = torch.tensor(Y, device=cuda_device)
+    tg = torch.full((4,), 99, dtype=torch.int32, device=cuda_device)
+    res = run(ref, cand, tg)
+    want = O.full_vocab(X.astype(np.float64), Y.astype(np.float64), np.full(4, 99))
+    assert np.all(np.abs(want["ref_target_lp"]) < 1e-4)
+    assert_lp_close(res["ref_target_lp"].cpu().numpy(), want["ref_target_lp"])
+    assert_lp_close(res["cand_target_lp"].cpu().numpy(), want["cand_target_lp"])
+    assert_kl_close(res["kl"].cpu().numpy(), want["kl"])
+
+
+def test_empty_batch(cuda_device):
+    ref = torch.empty((0, 100), device=cuda_device)
+    res = kq.kld_full_vocab(ref, ref.clone())
+    assert res["kl"].numel() == 0
