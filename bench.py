@@ -205,10 +205,12 @@ def run_reference(args) -> int:
     return 0
 
 
-def config_dict() -> dict:
-    return {"workload": WORKLOAD, "n_rows": N_ROWS, "vocab": VOCAB, "input_dtype": "bf16",
+def config_dict(rows: int = N_ROWS) -> dict:
+    workload = WORKLOAD if rows == N_ROWS else WORKLOAD.replace("2047 positions", f"{rows} positions") + \
+        " (reduced profiling case)"
+    return {"workload": workload, "n_rows": rows, "vocab": VOCAB, "input_dtype": "bf16",
             "step": "kld_full_vocab + kld_reduce_stats (mean, p50, p99, p99.9, top-1, ppl)",
-            "l2": "inputs larger than L2: 2.03 GB of logits per step",
+            "l2": f"inputs larger than L2: {2 * rows * VOCAB * 2 / 1e9:.2f} GB of logits per step",
             "parallelism": "dp (each rank scores its own window)"}
 
 
@@ -229,7 +231,7 @@ def run_ours(args) -> int:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     kq.load_library()
 
-    d = W.window_full_vocab(seed=W.seed_for(2) + 1000 * rank, device=dev)
+    d = W.window_full_vocab(seed=W.seed_for(2) + 1000 * rank, device=dev, n_rows=args.rows)
     ref, cand, targets = d["ref"], d["cand"], d["targets"]
     n = ref.shape[0]
     stream = torch.cuda.current_stream()
@@ -311,7 +313,7 @@ def run_ours(args) -> int:
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded Zipf/Gumbel logits; no corpus or model)",
-            "config": config_dict(), "roofline": roofline,
+            "config": config_dict(args.rows), "roofline": roofline,
             "clocks": sampler.summary(t0, t1), "gpu_launches": 2 * args.steps, "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -402,6 +404,8 @@ def main(argv=None) -> int:
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rows", type=int, default=N_ROWS,
+                    help="positions per window (default 2047; smaller only for profiling runs)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

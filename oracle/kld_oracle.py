@@ -307,6 +307,17 @@ def topk_tail(ref_ids, ref_lp, cand_ids, cand_lp, vocab: int, chunk: int = 8192)
 # reductions
 # ---------------------------------------------------------------------------
 
+def exact_mean(vals: np.ndarray) -> float:
+    """Correctly rounded mean (math.fsum), with IEEE results for infinite
+    members: +inf and -inf together give NaN, one kind alone gives itself."""
+    if vals.shape[0] == 0:
+        return math.nan
+    try:
+        return math.fsum(vals.tolist()) / vals.shape[0]
+    except ValueError:      # both +inf and -inf present
+        return math.nan
+
+
 def quantile_linear(sorted_vals: np.ndarray, q: float) -> tuple[float, float, float]:
     """Linear-interpolation percentile of an ascending array.
 
@@ -350,7 +361,7 @@ def reduce_stats(kl, ref_argmax=None, cand_argmax=None, top1=None,
     vals = kl[valid].astype(np.float64)
     n = int(vals.shape[0])
     out = dict(n=n, n_nan=int(np.sum(sel & isnan)))
-    out["mean_kl"] = math.fsum(vals.tolist()) / n if n else math.nan
+    out["mean_kl"] = exact_mean(vals)
     s = np.sort(kl[valid])
     qv, qlo, qhi = [], [], []
     for q in quantiles:
@@ -375,7 +386,7 @@ def reduce_stats(kl, ref_argmax=None, cand_argmax=None, top1=None,
         if arr is None:
             continue
         nll = -np.asarray(arr, dtype=np.float32)[valid].astype(np.float64)
-        out[f"{name}_mean_nll"] = math.fsum(nll.tolist()) / n if n else math.nan
+        out[f"{name}_mean_nll"] = exact_mean(nll)
         out[f"{name}_ppl"] = math.exp(out[f"{name}_mean_nll"]) if n else math.nan
     if "ref_ppl" in out and "cand_ppl" in out:
         out["ppl_ratio"] = out["cand_ppl"] / out["ref_ppl"]

@@ -83,7 +83,7 @@ __device__ __forceinline__ bool scored(const ReduceParams& p, long long i, float
 }
 
 // Targets from the scored count: for every quantile, the lower and upper
-// order statistic ranks of linear interpolation at h = (n - 1) q.
+// order statistic ranks of linear interpolation at h = (n - 1) q.  Thread 0.
 __device__ void select_init(Select& s, const ReduceParams& p, long long n) {
   s.n = n;
   s.nt = (n > 0) ? 2 * p.nq : 0;
@@ -99,31 +99,63 @@ __device__ void select_init(Select& s, const ReduceParams& p, long long n) {
   for (int t = 0; t < s.nt; ++t) s.prefix[t] = 0u;
 }
 
+// Group targets by prefix (warp 0): uslot[t] indexes uprefix[] of unique
+// prefixes, numbered in order of their first target.  Call from every thread.
 __device__ void select_unique(Select& s) {
-  s.nu = 0;
-  for (int t = 0; t < s.nt; ++t) {
-    int u = 0;
-    while (u < s.nu && s.uprefix[u] != s.prefix[t]) ++u;
-    if (u == s.nu) s.uprefix[s.nu++] = s.prefix[t];
-    s.uslot[t] = u;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const unsigned act = __ballot_sync(0xffffffffu, lane < s.nt);
+    unsigned leaders = 0;
+    if (lane < s.nt) {
+      const unsigned same = __match_any_sync(act, s.prefix[lane]);
+      const int leader = __ffs(same) - 1;
+      leaders = __ballot_sync(act, lane == leader);
+      const int my_u = __popc(leaders & ((1u << leader) - 1u));
+      s.uslot[lane] = my_u;
+      if (lane == leader) s.uprefix[my_u] = s.prefix[lane];
+    }
+    if (lane == 0) s.nu = __popc(leaders);  // lane 0 is active whenever nt > 0
   }
+  __syncthreads();
 }
 
-// Advance every target by one 8-bit digit using histogram h[u][bin].
+// Advance every target by one 8-bit digit using histogram h[u][bin]: warp w
+// takes targets w, w + warps, ...  Lane l holds bins 8l .. 8l+7; a warp scan
+// of the lane totals finds the bin holding the target rank.  Call from every
+// thread; regroups the prefixes afterwards.
 __device__ void select_step(Select& s, const unsigned* h) {
-  for (int t = 0; t < s.nt; ++t) {
-    const unsigned* row = h + s.uslot[t] * kBins;
-    long long acc = 0;
-    int d = 0;
-    for (; d < kBins; ++d) {
-      const long long c = row[d];
-      if (s.rem[t] < acc + c) break;
-      acc += c;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int t = w; t < s.nt; t += nw) {
+    const unsigned* row = h + s.uslot[t] * kBins + lane * 8;
+    unsigned c[8];
+    unsigned run = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      run += row[k];
+      c[k] = run;  // inclusive prefix within the lane
     }
-    if (d == kBins) d = kBins - 1;  // unreachable for consistent histograms
-    s.rem[t] -= acc;
-    s.prefix[t] = (s.prefix[t] << 8) | (uint32_t)d;
+    unsigned base = run;  // inclusive warp scan of lane totals
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned o = __shfl_up_sync(0xffffffffu, base, off);
+      if (lane >= off) base += o;
+    }
+    base -= run;  // exclusive
+    const unsigned long long rem = (unsigned long long)s.rem[t];
+    const unsigned hit = __ballot_sync(0xffffffffu, (unsigned long long)base + run > rem);
+    const int L = hit ? __ffs(hit) - 1 : 31;
+    if (lane == L) {
+      int k = 7;
+      for (int j = 7; j >= 0; --j)
+        if ((unsigned long long)base + c[j] > rem) k = j;
+      const unsigned before = base + (k ? c[k - 1] : 0u);
+      s.rem[t] = (long long)(rem - before);
+      s.prefix[t] = (s.prefix[t] << 8) | (uint32_t)(8 * L + k);
+    }
+    __syncwarp();
   }
+  __syncthreads();
+  select_unique(s);
 }
 
 // One histogram pass over [begin, end) with stride `stride`, adding into the
@@ -254,28 +286,21 @@ __global__ void __launch_bounds__(kSmallThreads) reduce_small_kernel(const Reduc
   __shared__ unsigned sh[kMaxTargets * kBins];
   __shared__ Partial sh_warp[kSmallThreads / 32];
   __shared__ Select sel;
-  __shared__ long long n_scored;
 
   Partial acc;
   thread_sums(p, threadIdx.x, blockDim.x, acc);
   block_sum(acc, sh_warp);
-  if (threadIdx.x == 0) n_scored = acc.n;
-  __syncthreads();
   if (threadIdx.x == 0) {
-    select_init(sel, p, n_scored);
-    select_unique(sel);
+    select_init(sel, p, acc.n);
   }
   __syncthreads();
+  select_unique(sel);
   for (int pass = 0; pass < kPasses; ++pass) {
     for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
     if (sel.nt > 0) hist_pass(p, sel, pass, threadIdx.x, blockDim.x, sh);
     __syncthreads();
-    if (threadIdx.x == 0) {
-      select_step(sel, sh);
-      select_unique(sel);
-    }
-    __syncthreads();
+    select_step(sel, sh);
   }
   if (threadIdx.x == 0) write_stats(p, acc, sel);
 }
@@ -286,16 +311,17 @@ __global__ void reduce_zero_kernel(unsigned* hist) {
   for (int i = threadIdx.x; i < kPasses * kMaxTargets * kBins; i += blockDim.x) hist[i] = 0u;
 }
 
-// Rebuild the select state from the histograms of passes < pass.
+// Rebuild the select state from the histograms of passes < pass.  Call
+// from every thread of the block.
 __device__ void select_replay(Select& s, const ReduceParams& p, int pass) {
-  long long n = 0;
-  for (int d = 0; d < kBins; ++d) n += p.hist[d];
-  select_init(s, p, n);
-  select_unique(s);
-  for (int q = 0; q < pass; ++q) {
-    select_step(s, p.hist + q * kMaxTargets * kBins);
-    select_unique(s);
+  if (threadIdx.x == 0) {
+    long long n = 0;
+    for (int d = 0; d < kBins; ++d) n += p.hist[d];
+    select_init(s, p, n);
   }
+  __syncthreads();
+  select_unique(s);
+  for (int q = 0; q < pass; ++q) select_step(s, p.hist + q * kMaxTargets * kBins);
 }
 
 __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReduceParams p, int pass) {
@@ -303,15 +329,15 @@ __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReducePa
   __shared__ Select sel;
   __shared__ Partial sh_warp[kBigThreads / 32];
   for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) sh[i] = 0u;
-  if (threadIdx.x == 0) {
-    if (pass == 0) {
+  if (pass == 0) {
+    if (threadIdx.x == 0) {
       sel.nt = 1;  // histogram every scored element
       sel.nu = 0;
-    } else {
-      select_replay(sel, p, pass);
     }
+    __syncthreads();
+  } else {
+    select_replay(sel, p, pass);
   }
-  __syncthreads();
   const long long begin = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long stride = (long long)gridDim.x * blockDim.x;
   if (sel.nt > 0) hist_pass(p, sel, pass, begin, stride, sh);
@@ -328,12 +354,12 @@ __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReducePa
     if (sh[i]) atomicAdd(&g[i], sh[i]);
 }
 
-__global__ void reduce_final_kernel(const ReduceParams p, int n_partials) {
+__global__ void __launch_bounds__(kBigThreads) reduce_final_kernel(const ReduceParams p, int n_partials) {
+  __shared__ Select sel;
+  select_replay(sel, p, kPasses);
   if (threadIdx.x != 0) return;
   Partial tot = p.partials[0];
   for (int b = 1; b < n_partials; ++b) partial_add(tot, p.partials[b]);
-  Select sel;
-  select_replay(sel, p, kPasses);
   write_stats(p, tot, sel);
 }
 
@@ -379,7 +405,7 @@ cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
   const int grid = big_grid(a.n);
   reduce_zero_kernel<<<1, 1024, 0, stream>>>(p.hist);
   for (int pass = 0; pass < kPasses; ++pass) reduce_pass_kernel<<<grid, kBigThreads, 0, stream>>>(p, pass);
-  reduce_final_kernel<<<1, 32, 0, stream>>>(p, grid);
+  reduce_final_kernel<<<1, kBigThreads, 0, stream>>>(p, grid);
   return cudaGetLastError();
 }
 

@@ -77,8 +77,10 @@ def test_special_values(cuda_device):
     st = kq.kld_reduce_stats(T(kl), quantiles=QS)
     want = O.reduce_stats(kl, quantiles=QS)
     assert st["n"] == 7 and st["n_nan"] == 1 and st["top1_agree"] == -1
-    for g, w in zip(st["q_lo"], want["q_lo"]):
-        assert g == w
+    assert math.isnan(st["mean_kl"]) and math.isnan(want["mean_kl"])   # +inf and -inf together
+    for key in ("q_lo", "q_hi", "q_value"):
+        for g, w in zip(st[key], want[key]):
+            assert (g == w) or (math.isnan(g) and math.isnan(w)), key
 
 
 def test_empty_and_all_nan(cuda_device):

@@ -314,6 +314,12 @@ def pin_mean_and_counts(O):
     assert _close(st["ref_ppl"], math.exp(nll_r), rtol=1e-15)
 
 
+def pin_mean_infinities(O):
+    assert math.isnan(O.reduce_stats(np.array([np.inf, -np.inf, 1.0], np.float32))["mean_kl"])
+    assert O.reduce_stats(np.array([np.inf, 2.0], np.float32))["mean_kl"] == math.inf
+    assert O.reduce_stats(np.array([-np.inf, 2.0], np.float32))["mean_kl"] == -math.inf
+
+
 def pin_uniform_perplexity(O):
     # A uniform reference over V ids has perplexity V.
     V = 4096
@@ -394,8 +400,8 @@ MUTANTS = [
      "            q[j] = leftover\n            logq[j] = math.log(max(leftover, Q_FLOOR))"),
     ("q_tail from the reference side", "q_tail = 1.0 - float(np.sum(q))", "q_tail = 1.0 - float(np.sum(p))"),
     ("percentile index n q", "h = (n - 1) * float(q)", "h = n * float(q) - 0.5"),
-    ("mean over all positions", "out[\"mean_kl\"] = math.fsum(vals.tolist()) / n if n else math.nan",
-     "out[\"mean_kl\"] = math.fsum(vals.tolist()) / max(n_all, 1)"),
+    ("mean over all positions", "out[\"mean_kl\"] = exact_mean(vals)",
+     "out[\"mean_kl\"] = exact_mean(kl.astype(np.float64))"),
     ("transposed head", "return np.asarray(H, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T",
      "return (np.asarray(W, dtype=np.float64) @ np.asarray(H, dtype=np.float64).T).T[:, ::-1]"),
 ]
