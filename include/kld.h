@@ -92,7 +92,10 @@ const char* kld_status_string(kld_status s);
  *    ref_argmax[r]     = lowest i with x_i = max x   (cand_argmax: same on y)
  *    ref_target_lp[r]  = log p_t,  cand_target_lp[r] = log q_t,  t = target_ids[r]
  *
- * Each logit is read from HBM exactly once (single streaming pass).
+ * Each logit is read from HBM exactly once (single streaming pass).  The
+ * work is split over a fixed set of warps that write per-row partial states
+ * to `workspace`; a second kernel merges them in index order, so results
+ * are bitwise reproducible and do not depend on the device.
  *
  * Arguments:
  *   ref_logits, cand_logits  [n_rows, ld_*] row-major, element type `dtype`.
@@ -105,6 +108,9 @@ const char* kld_status_string(kld_status s);
  *   kl                       f32 [n_rows], required.
  *   ref_argmax, cand_argmax  int32 [n_rows], each may be NULL.
  *   ref_target_lp, cand_target_lp  f32 [n_rows], each may be NULL.
+ *   workspace                device scratch of at least
+ *                            kld_full_vocab_workspace_size(n_rows) bytes,
+ *                            256-byte aligned; no initial contents needed.
  *   dev_status               int32 device word, may be NULL.
  *
  * Non-finite input: -inf logits are allowed (an id with p_i = 0 contributes
@@ -117,7 +123,11 @@ kld_status kld_full_vocab(const void* ref_logits, const void* cand_logits, kld_d
                           int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
                           const int32_t* target_ids, float* kl, int32_t* ref_argmax,
                           int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
-                          int32_t* dev_status, void* stream);
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                          void* stream);
+
+/* Workspace bytes kld_full_vocab needs for n_rows rows (any vocab, dtype). */
+size_t kld_full_vocab_workspace_size(int64_t n_rows);
 
 /*
  * kld_topk_tail - KL over the reference's top-k ids plus one tail bucket.

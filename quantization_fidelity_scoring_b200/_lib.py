@@ -62,7 +62,8 @@ PROTOTYPES = {
     "kld_version": (ctypes.c_int, []),
     "kld_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kld_full_vocab": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P, _P,
-                                      _P, _P, _P, _P]),
+                                      _P, _P, _P, _SZ, _P, _P]),
+    "kld_full_vocab_workspace_size": (_SZ, [_I64]),
     "kld_topk_tail": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I64, _P, _P, _P, _P, _P]),
     "kld_reduce_workspace_size": (_SZ, [_I64]),
     "kld_reduce_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _I32, _P, _P,
@@ -71,8 +72,8 @@ PROTOTYPES = {
 
 # exported for tests only (not part of the public header)
 TEST_PROTOTYPES = {
-    "kld_full_vocab_cluster": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
-                                              _P, _P, _P, _P, _P, _I32]),
+    "kld_full_vocab_split": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
+                                            _P, _P, _P, _P, _SZ, _P, _P, _I32]),
 }
 
 _lib = None

@@ -55,11 +55,12 @@ _DTYPES = {torch.float32: _lib.KLD_F32, torch.bfloat16: _lib.KLD_BF16}
 
 def kld_full_vocab(ref: torch.Tensor, cand: torch.Tensor, targets: torch.Tensor | None = None, *,
                    argmax: bool = True, kl=None, ref_argmax=None, cand_argmax=None,
-                   ref_target_lp=None, cand_target_lp=None, dev_status=None, stream=None,
-                   ctas_per_row: int = 0) -> dict:
+                   ref_target_lp=None, cand_target_lp=None, workspace=None, dev_status=None,
+                   stream=None, warps: int = 0) -> dict:
     """Full-vocabulary KL / argmax / target log-probs of [n, V] logit rows
-    (f32 or bf16, unit stride along V).  Outputs are allocated when not
-    given.  ctas_per_row forces the split of a row across CTAs (tests)."""
+    (f32 or bf16, unit stride along V).  Outputs and the workspace are
+    allocated when not given.  `warps` forces the number of streaming warps
+    (tests of the piece merge)."""
     _need_cuda("ref", ref, ndim=2)
     _need_cuda("cand", cand, ndim=2)
     if ref.dtype != cand.dtype or ref.dtype not in _DTYPES:
@@ -80,11 +81,14 @@ def kld_full_vocab(ref: torch.Tensor, cand: torch.Tensor, targets: torch.Tensor 
         ref_target_lp = _out(ref_target_lp, n, torch.float32, dev)
         cand_target_lp = _out(cand_target_lp, n, torch.float32, dev)
     lib = _lib.load()
+    if workspace is None:
+        workspace = torch.empty(lib.kld_full_vocab_workspace_size(n), dtype=torch.uint8, device=dev)
     args = (_ptr(ref), _ptr(cand), _DTYPES[ref.dtype], n, V, ref.stride(0), cand.stride(0),
             _ptr(targets), _ptr(kl), _ptr(ref_argmax), _ptr(cand_argmax), _ptr(ref_target_lp),
-            _ptr(cand_target_lp), _ptr(dev_status), _stream_handle(stream))
-    if ctas_per_row:
-        st = lib.kld_full_vocab_cluster(*args, ctas_per_row)
+            _ptr(cand_target_lp), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+            _stream_handle(stream))
+    if warps:
+        st = lib.kld_full_vocab_split(*args, warps)
     else:
         st = lib.kld_full_vocab(*args)
     _check(st, "kld_full_vocab")
@@ -116,6 +120,10 @@ def kld_topk_tail(ref_ids, ref_lp, cand_ids, cand_lp, vocab: int, *, kl=None, to
                            _stream_handle(stream))
     _check(st, "kld_topk_tail")
     return dict(kl=kl, top1=top1, n_matched=n_matched)
+
+
+def kld_full_vocab_workspace_size(n_rows: int) -> int:
+    return int(_lib.load().kld_full_vocab_workspace_size(n_rows))
 
 
 def kld_reduce_workspace_size(n: int) -> int:

@@ -1,42 +1,66 @@
 // Full-vocabulary scoring: one streaming pass over both logit rows.
 //
-// Per row the reference logits x and candidate logits y are read once from
-// HBM with 128-bit non-allocating loads; a cluster of CTAs splits the row.
-// Each warp walks 32 consecutive 16-byte vectors (two per lane) per step and
-// keeps an online log-sum-exp state (kld_common.cuh) whose running maximum
-// and argmax are warp-uniform: one redux.sync finds the step's maximum, and
-// only a step that raises it (a handful per warp per row) takes the branch
-// that rescales, locates the new argmax and leaves it out of the sum.  Every
-// other step is two ex2 per element pair on paired f32x2 arithmetic.  Warp
-// states merge across the CTA's warps and then across the cluster's CTAs
-// through distributed shared memory, in fixed orders.
+// The rows' 16-byte vectors, flattened in (row, vector) order, are split
+// evenly over a fixed set of persistent warps.  Each warp streams its range
+// with 128-bit non-allocating loads, two vectors per lane per step, and
+// keeps an online log-sum-exp state (kld_common.cuh) whose running maximum and argmax are
+// warp-uniform: one redux.sync finds a step's maximum, and only a step that
+// raises it (a handful per row piece) takes the branch that rescales,
+// locates the new argmax and leaves it out of the sum.  Every other step is
+// two ex2 per element pair on paired f32x2 arithmetic.  A warp writes one
+// partial state per row it touches to the workspace; a second kernel merges
+// each row's pieces in index order (one warp per row), adds the ragged tail
+// and forms the outputs.  No barrier is shared between warps of the
+// streaming kernel, and every merge order is fixed, so results are bitwise
+// reproducible.
 //
 // Sources: "Qwen3.8-27B Quantization Challenge", sections "How the
 // references were made" (full 248,320-token distribution in f32) and "The
 // score" (KL over cells); "Qwopus3.8-27B-Coder-Flash: quality-eval
 // reference", "Method" (exact argmax top-1, perplexity from the true-token
 // log-prob).
-#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cfloat>
 
 #include "kld_common.cuh"
 #include "launch.h"
 
-namespace cg = cooperative_groups;
-
 namespace kld {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kWarpsPerCta = kThreads / 32;
+constexpr int kStepVecs = 64;                    // vectors a warp covers per step
+constexpr int kMinVecsPerWarp = 8 * kStepVecs;   // below this, use fewer warps
+constexpr int kMaxStreamWarps = kFullVocabMaxWarps;
 
-struct FullVocabParams {
+// Partial state of one warp over one row piece (32 bytes).
+struct Piece {
+  float mx, rx;
+  int ax;
+  float my, ry;
+  int ay;
+  float A;
+  int pad;
+};
+
+struct StreamParams {
   const void* x;
   const void* y;
   int64_t ld_x, ld_y;  // elements
-  int vocab;
-  int cl;              // CTAs per row (cluster size)
+  int nvec;            // full 16-byte vectors per row
+  int nwarps;
+  int64_t total;       // n_rows * nvec
+  Piece* pieces;       // slot row + warp
+};
+
+struct MergeParams {
+  const void* x;
+  const void* y;
+  int64_t ld_x, ld_y;
+  int vocab, nvec, n_rows, nwarps;
+  int64_t total;
+  const Piece* pieces;
   const int32_t* targets;
   float* kl;
   int32_t* ax;
@@ -45,6 +69,10 @@ struct FullVocabParams {
   float* lpy;
   int32_t* dev_status;
 };
+
+__host__ __device__ __forceinline__ int64_t warp_begin(int64_t w, int64_t total, int nwarps) {
+  return (total * w) / nwarps;
+}
 
 __device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 v;
@@ -102,9 +130,10 @@ struct StepRaw {
 };
 
 // Order-preserving map between floats and signed ints, so that a warp-wide
-// float maximum is one redux.sync.max.s32 (NaN is mapped to -inf first).
+// float maximum is one redux.sync.max.s32.  A lane maximum is NaN only when
+// all its elements are NaN; that row is invalid whatever maximum wins.
 __device__ __forceinline__ int ordered_key(float f) {
-  const int i = __float_as_int(f != f ? -CUDART_INF_F : f);
+  const int i = __float_as_int(f);
   return i ^ ((i >> 31) & 0x7fffffff);
 }
 __device__ __forceinline__ float key_value(int k) { return __int_as_float(k ^ ((k >> 31) & 0x7fffffff)); }
@@ -218,85 +247,79 @@ __device__ __forceinline__ float slot_diff(const StepRaw& raw, int j) {
   return fmaxf(d, -FLT_MAX);
 }
 
+
+// Stream vectors [a, b) of one row; returns the warp's partial state
+// (identical in every lane).
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads) full_vocab_kernel(const FullVocabParams p) {
+__device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow, int a, int b, int lane) {
   using El = Elems<kBF16>;
-  constexpr int E = El::E;  // elements per 16-byte vector
-  constexpr int kElemBytes = kBF16 ? 2 : 4;
+  constexpr int E = El::E;
   constexpr uint32_t kNegInfWord = kBF16 ? 0xff80ff80u : 0xff800000u;
-
-  const int cl = p.cl;
-  const int row = blockIdx.x / cl;
-  const int rank = blockIdx.x % cl;
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-
-  const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld_x * kElemBytes;
-  const char* yrow = reinterpret_cast<const char*>(p.y) + (int64_t)row * p.ld_y * kElemBytes;
-
-  const int nvec = p.vocab / E;
-  const int seg_begin = (int)(((int64_t)nvec * rank) / cl);
-  const int seg_end = (int)(((int64_t)nvec * (rank + 1)) / cl);
-  const int steps = (seg_end - seg_begin + 2 * kThreads - 1) / (2 * kThreads);
-  const int lane_base = seg_begin + warp * 32 + lane;
   const uint4 neg_inf = make_uint4(kNegInfWord, kNegInfWord, kNegInfWord, kNegInfWord);
-
-  auto load_step = [&](int st, StepRaw& r) {
-    const int v0 = lane_base + st * 2 * kThreads;
-    const int v1 = v0 + kThreads;
-    r.x0 = v0 < seg_end ? ld_stream(xrow + (int64_t)v0 * 16) : neg_inf;
-    r.y0 = v0 < seg_end ? ld_stream(yrow + (int64_t)v0 * 16) : neg_inf;
-    r.x1 = v1 < seg_end ? ld_stream(xrow + (int64_t)v1 * 16) : neg_inf;
-    r.y1 = v1 < seg_end ? ld_stream(yrow + (int64_t)v1 * 16) : neg_inf;
-  };
 
   WarpSide sx{-CUDART_INF_F, -1, 0.f}, sy{-CUDART_INF_F, -1, 0.f};
   float2 rx2 = make_float2(0.f, 0.f), ry2 = rx2, a2 = rx2;
 
-  StepRaw cur;
-  if (steps > 0) load_step(0, cur);
-  for (int st = 0; st < steps; ++st) {
-    // the next step's loads are in flight while this step computes
-    StepRaw nxt;
-    if (st + 1 < steps) load_step(st + 1, nxt);
+  const int n = b - a;
+  const int nfull = n / kStepVecs;
+  const char* xl = xrow + (int64_t)(a + lane) * 16;
+  const char* yl = yrow + (int64_t)(a + lane) * 16;
 
+  auto load_full = [&](StepRaw& r, int st) {
+    const int64_t o = (int64_t)st * kStepVecs * 16;
+    r.x0 = ld_stream(xl + o);
+    r.y0 = ld_stream(yl + o);
+    r.x1 = ld_stream(xl + o + 32 * 16);
+    r.y1 = ld_stream(yl + o + 32 * 16);
+  };
+  auto step = [&](const StepRaw& cur, int st) {
     const float cx0 = El::vmax(cur.x0), cx1 = El::vmax(cur.x1);
     const float cy0 = El::vmax(cur.y0), cy1 = El::vmax(cur.y1);
     const float CMX = warp_max(fmaxf(cx0, cx1));
     const float CMY = warp_max(fmaxf(cy0, cy1));
-
     if (!((CMX > sx.m) || (CMY > sy.m) || (sx.a < 0) || (sy.a < 0))) {  // warp-uniform
       accumulate<kBF16, false>(cur, sx.m, sy.m, -1, -1, rx2, ry2, a2);
-    } else {
-      // a new maximum on either side, or a side still without a finite
-      // value: fold the paired sums, move to the new maxima, weigh with the
-      // new argmaxes masked out of r
-      sx.r += rx2.x + rx2.y;
-      sy.r += ry2.x + ry2.y;
-      float A = a2.x + a2.y;
-      const int i0 = (lane_base + st * 2 * kThreads) * E;
-      const int i1 = i0 + kThreads * E;
-      int ex_x, ex_y;
-      const float scx = side_new_max<kBF16>(sx, CMX, cur.x0, cur.x1, cx0, cx1, i0, i1, lane, ex_x);
-      side_new_max<kBF16>(sy, CMY, cur.y0, cur.y1, cy0, cy1, i0, i1, lane, ex_y);
-      A *= scx;
-      if (ex_x >= 0) A += slot_diff<kBF16>(cur, ex_x);
-      rx2 = ry2 = make_float2(0.f, 0.f);
-      a2 = make_float2(A, 0.f);
-      // a side with no finite value yet has only -inf (weight 0) or NaN
-      // (poisons r, marking the row invalid); any finite offset serves
-      accumulate<kBF16, true>(cur, sx.a < 0 ? 0.f : sx.m, sy.a < 0 ? 0.f : sy.m, ex_x, ex_y, rx2, ry2, a2);
+      return;
     }
-    if (st + 1 < steps) cur = nxt;
+    // a new maximum on either side, or a side still without a finite value:
+    // fold the paired sums, move to the new maxima, weigh with the new
+    // argmaxes masked out of r
+    sx.r += rx2.x + rx2.y;
+    sy.r += ry2.x + ry2.y;
+    float A = a2.x + a2.y;
+    const int i0 = (a + st * kStepVecs + lane) * E;
+    const int i1 = i0 + 32 * E;
+    int ex_x, ex_y;
+    const float scx = side_new_max<kBF16>(sx, CMX, cur.x0, cur.x1, cx0, cx1, i0, i1, lane, ex_x);
+    side_new_max<kBF16>(sy, CMY, cur.y0, cur.y1, cy0, cy1, i0, i1, lane, ex_y);
+    A *= scx;
+    if (ex_x >= 0) A += slot_diff<kBF16>(cur, ex_x);
+    rx2 = ry2 = make_float2(0.f, 0.f);
+    a2 = make_float2(A, 0.f);
+    // a side with no finite value yet has only -inf (weight 0) or NaN
+    // (poisons r, marking the row invalid); any finite offset serves
+    accumulate<kBF16, true>(cur, sx.a < 0 ? 0.f : sx.m, sy.a < 0 ? 0.f : sy.m, ex_x, ex_y, rx2, ry2, a2);
+  };
+
+  // full steps: the warp's four 16-byte loads per lane are issued together
+  // at the top of each step; other warps cover the latency
+  StepRaw A;
+  int st = 0;
+  for (; st < nfull; ++st) {
+    load_full(A, st);
+    step(A, st);
+  }
+  // ragged last step: lanes past b read -inf
+  if (st * kStepVecs < n) {
+    const int v0 = st * kStepVecs + lane, v1 = v0 + 32;
+    const int64_t o = (int64_t)st * kStepVecs * 16;
+    A.x0 = v0 < n ? ld_stream(xl + o) : neg_inf;
+    A.y0 = v0 < n ? ld_stream(yl + o) : neg_inf;
+    A.x1 = v1 < n ? ld_stream(xl + o + 32 * 16) : neg_inf;
+    A.y1 = v1 < n ? ld_stream(yl + o + 32 * 16) : neg_inf;
+    step(A, st);
   }
 
-  // warp state: uniform maxima, lane shares summed in a fixed butterfly
-  RowState s;
-  s.x.m = sx.m;
-  s.x.a = sx.a;
-  s.y.m = sy.m;
-  s.y.a = sy.a;
   float rxs = sx.r + (rx2.x + rx2.y);
   float rys = sy.r + (ry2.x + ry2.y);
   float as = a2.x + a2.y;
@@ -306,48 +329,79 @@ __global__ void __launch_bounds__(kThreads) full_vocab_kernel(const FullVocabPar
     rys += __shfl_xor_sync(0xffffffffu, rys, off);
     as += __shfl_xor_sync(0xffffffffu, as, off);
   }
-  s.x.r = rxs;
-  s.y.r = rys;
-  s.A = as;
+  return Piece{sx.m, rxs, sx.a, sy.m, rys, sy.a, as, 0};
+}
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads) stream_kernel(const StreamParams p) {
+  constexpr int kElemBytes = kBF16 ? 2 : 4;
+  const int lane = threadIdx.x & 31;
+  const int w = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (w >= p.nwarps) return;  // the whole warp leaves together
+  int64_t pos = warp_begin(w, p.total, p.nwarps);
+  const int64_t end = warp_begin(w + 1, p.total, p.nwarps);
+  while (pos < end) {
+    const int row = (int)(pos / p.nvec);
+    const int64_t row0 = (int64_t)row * p.nvec;
+    const int a = (int)(pos - row0);
+    const int b = (int)min((int64_t)p.nvec, end - row0);
+    const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld_x * kElemBytes;
+    const char* yrow = reinterpret_cast<const char*>(p.y) + (int64_t)row * p.ld_y * kElemBytes;
+    const Piece pc = stream_piece<kBF16>(xrow, yrow, a, b, lane);
+    if (lane == 0) p.pieces[row + w] = pc;
+    pos = row0 + b;
+  }
+}
+
+__device__ __forceinline__ int warp_of(int64_t g, int64_t total, int nwarps) {
+  int w = (int)((g * nwarps) / total);
+  while (w + 1 < nwarps && warp_begin(w + 1, total, nwarps) <= g) ++w;
+  while (w > 0 && warp_begin(w, total, nwarps) > g) --w;
+  return w;
+}
+
+__device__ __forceinline__ RowState piece_state(const Piece& pc) {
+  RowState s;
+  s.x = Side{pc.mx, pc.rx, pc.ax};
+  s.y = Side{pc.my, pc.ry, pc.ay};
+  s.A = pc.A;
   s.bad = 0;
+  return s;
+}
 
-  __shared__ RowState warp_states[kWarps];
-  __shared__ RowState cta_state;
-  if (lane == 0) warp_states[warp] = s;
-  __syncthreads();
-  if (tid == 0) {
-    RowState c = warp_states[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) c = row_merge(c, warp_states[w]);
-    // ragged tail (vocab not a multiple of E): the row's last ids, pushed
-    // one by one in index order into the last CTA's state
-    if (rank == cl - 1) {
-      for (int i = nvec * E; i < p.vocab; ++i) {
-        const float xv = El::load1(xrow, i), yv = El::load1(yrow, i);
-        float wx, scx, wy, scy;
-        side_push(c.x, xv, i, wx, scx, c.bad);
-        side_push(c.y, yv, i, wy, scy, c.bad);
-        c.A = c.A * scx + wx * fmaxf(xv - yv, -FLT_MAX);
-      }
+// One warp per row: merge the row's pieces in warp (= index) order, push the
+// ragged tail ids, gather the target logits and write the outputs.
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads) merge_kernel(const MergeParams p) {
+  using El = Elems<kBF16>;
+  constexpr int E = El::E;
+  constexpr int kElemBytes = kBF16 ? 2 : 4;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (row >= p.n_rows) return;
+  const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld_x * kElemBytes;
+  const char* yrow = reinterpret_cast<const char*>(p.y) + (int64_t)row * p.ld_y * kElemBytes;
+
+  RowState acc = row_empty();
+  if (p.nvec > 0) {
+    const int64_t f = (int64_t)row * p.nvec;
+    const int w0 = warp_of(f, p.total, p.nwarps);
+    const int w1 = warp_of(f + p.nvec - 1, p.total, p.nwarps);
+    for (int c = w0; c <= w1; c += 32) {
+      const int w = c + lane;
+      RowState s = (w <= w1) ? piece_state(p.pieces[row + w]) : row_empty();
+      s = warp_merge_row(s);
+      acc = (c == w0) ? s : row_merge(acc, s);
     }
-    cta_state = c;
   }
-
-  if (cl > 1) {
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    if (rank == 0 && tid == 0) {
-      RowState c = *cluster.map_shared_rank(&cta_state, 0);
-      for (int r = 1; r < cl; ++r) c = row_merge(c, *cluster.map_shared_rank(&cta_state, r));
-      cta_state = c;
-    }
-    cluster.sync();  // keep every CTA's shared memory alive until rank 0 has read it
-  } else {
-    __syncthreads();
+  if (lane != 0) return;
+  for (int i = p.nvec * E; i < p.vocab; ++i) {
+    const float xv = El::load1(xrow, i), yv = El::load1(yrow, i);
+    float wx, scx, wy, scy;
+    side_push(acc.x, xv, i, wx, scx, acc.bad);
+    side_push(acc.y, yv, i, wy, scy, acc.bad);
+    acc.A = acc.A * scx + wx * fmaxf(xv - yv, -FLT_MAX);
   }
-  if (rank != 0 || tid != 0) return;
-
-  const RowState fin = cta_state;
   bool have_t = false;
   float xt = 0.f, yt = 0.f;
   if (p.targets) {
@@ -360,7 +414,7 @@ __global__ void __launch_bounds__(kThreads) full_vocab_kernel(const FullVocabPar
       set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
     }
   }
-  const RowOut o = row_finish(fin, have_t, xt, yt);
+  const RowOut o = row_finish(acc, have_t, xt, yt);
   p.kl[row] = o.kl;
   if (p.ax) p.ax[row] = o.ax;
   if (p.ay) p.ay[row] = o.ay;
@@ -368,48 +422,43 @@ __global__ void __launch_bounds__(kThreads) full_vocab_kernel(const FullVocabPar
   if (p.lpy) p.lpy[row] = o.lp_y;
 }
 
-int choose_cluster(int nvec) {
-  // about 32 vectors per thread per CTA, at most 8 CTAs (portable cluster)
-  const int per_cta = kThreads * 32;
-  int cl = (nvec + per_cta - 1) / per_cta;
-  if (cl < 1) cl = 1;
-  if (cl > 8) cl = 8;
-  return cl;
+int stream_warps(int64_t total, int override_warps) {
+  if (override_warps > 0) {
+    int64_t w = override_warps < kMaxStreamWarps ? override_warps : kMaxStreamWarps;
+    return (int)(w < total ? w : (total > 0 ? total : 1));
+  }
+  int64_t w = total / kMinVecsPerWarp;
+  if (w < 1) w = 1;
+  if (w > kMaxStreamWarps) w = kMaxStreamWarps;
+  return (int)w;
 }
 
 }  // namespace
 
-cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream) {
-  FullVocabParams p;
-  p.x = a.x;
-  p.y = a.y;
-  p.ld_x = a.ld_x;
-  p.ld_y = a.ld_y;
-  p.vocab = (int)a.vocab;
-  p.targets = a.targets;
-  p.kl = a.kl;
-  p.ax = a.ax;
-  p.ay = a.ay;
-  p.lpx = a.lpx;
-  p.lpy = a.lpy;
-  p.dev_status = a.dev_status;
-  const int E = a.bf16 ? 8 : 4;
-  p.cl = a.cluster_override > 0 ? a.cluster_override : choose_cluster((int)(a.vocab / E));
+size_t full_vocab_workspace_bytes(int64_t n_rows) {
+  return sizeof(Piece) * (size_t)(n_rows + kMaxStreamWarps);
+}
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(a.n_rows * p.cl), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.cl;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (a.bf16) return cudaLaunchKernelEx(&cfg, full_vocab_kernel<true>, p);
-  return cudaLaunchKernelEx(&cfg, full_vocab_kernel<false>, p);
+cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream) {
+  const int E = a.bf16 ? 8 : 4;
+  const int nvec = (int)(a.vocab / E);
+  const int64_t total = a.n_rows * (int64_t)nvec;
+  const int nwarps = stream_warps(total, a.warps_override);
+  Piece* pieces = reinterpret_cast<Piece*>(a.workspace);
+  if (total > 0) {
+    StreamParams sp{a.x, a.y, a.ld_x, a.ld_y, nvec, nwarps, total, pieces};
+    const unsigned grid = (unsigned)((nwarps + kWarpsPerCta - 1) / kWarpsPerCta);
+    if (a.bf16) stream_kernel<true><<<grid, kThreads, 0, stream>>>(sp);
+    else stream_kernel<false><<<grid, kThreads, 0, stream>>>(sp);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  MergeParams mp{a.x, a.y, a.ld_x, a.ld_y, (int)a.vocab, nvec, (int)a.n_rows, nwarps, total, pieces,
+                 a.targets, a.kl, a.ax, a.ay, a.lpx, a.lpy, a.dev_status};
+  const unsigned mgrid = (unsigned)((a.n_rows + kWarpsPerCta - 1) / kWarpsPerCta);
+  if (a.bf16) merge_kernel<true><<<mgrid, kThreads, 0, stream>>>(mp);
+  else merge_kernel<false><<<mgrid, kThreads, 0, stream>>>(mp);
+  return cudaGetLastError();
 }
 
 }  // namespace kld

@@ -38,16 +38,18 @@ static kld_status full_vocab_impl(const void* ref_logits, const void* cand_logit
                                   int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
                                   const int32_t* target_ids, float* kl, int32_t* ref_argmax,
                                   int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
-                                  int32_t* dev_status, void* stream, int ctas_per_row) {
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                  void* stream, int warps) {
   if (dtype != KLD_F32 && dtype != KLD_BF16) return KLD_ERR_UNSUPPORTED;
   if (n_rows < 0 || vocab < 1 || vocab > INT32_MAX) return KLD_ERR_INVALID_ARG;
   if (ld_ref < vocab || ld_cand < vocab) return KLD_ERR_INVALID_ARG;
   if (!target_ids && (ref_target_lp || cand_target_lp)) return KLD_ERR_INVALID_ARG;
-  if (ctas_per_row < 0 || ctas_per_row > 8) return KLD_ERR_INVALID_ARG;
+  if (warps < 0) return KLD_ERR_INVALID_ARG;
   if (n_rows == 0) return KLD_OK;
   if (!ref_logits || !cand_logits || !kl) return KLD_ERR_INVALID_ARG;
-  // one cluster of up to 8 CTAs per row in a 1-D grid
-  if (n_rows > (int64_t)(INT32_MAX / 8)) return KLD_ERR_UNSUPPORTED;
+  if (n_rows > (int64_t)INT32_MAX - kld::kFullVocabMaxWarps) return KLD_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < kld::full_vocab_workspace_bytes(n_rows)) return KLD_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return KLD_ERR_ALIGNMENT;
   const int64_t esize = dtype == KLD_BF16 ? 2 : 4;
   if (!aligned(ref_logits, 16) || !aligned(cand_logits, 16)) return KLD_ERR_ALIGNMENT;
   if ((ld_ref * esize) % 16 != 0 || (ld_cand * esize) % 16 != 0) return KLD_ERR_ALIGNMENT;
@@ -71,29 +73,36 @@ static kld_status full_vocab_impl(const void* ref_logits, const void* cand_logit
   a.lpx = ref_target_lp;
   a.lpy = cand_target_lp;
   a.dev_status = dev_status;
-  a.cluster_override = ctas_per_row;
+  a.workspace = workspace;
+  a.warps_override = warps;
   return cuda_status(kld::launch_full_vocab(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kld_full_vocab_workspace_size(int64_t n_rows) {
+  return n_rows < 0 ? 0 : kld::full_vocab_workspace_bytes(n_rows);
 }
 
 kld_status kld_full_vocab(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
                           int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
                           const int32_t* target_ids, float* kl, int32_t* ref_argmax,
                           int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
-                          int32_t* dev_status, void* stream) {
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
   return full_vocab_impl(ref_logits, cand_logits, dtype, n_rows, vocab, ld_ref, ld_cand, target_ids, kl,
-                         ref_argmax, cand_argmax, ref_target_lp, cand_target_lp, dev_status, stream, 0);
+                         ref_argmax, cand_argmax, ref_target_lp, cand_target_lp, workspace, workspace_bytes,
+                         dev_status, stream, 0);
 }
 
-// kld_full_vocab with the number of CTAs per row forced to 1..8 (0 = automatic).
-// Exported for tests of the cross-CTA merge; not declared in kld.h.
-kld_status kld_full_vocab_cluster(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
-                                  int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
-                                  const int32_t* target_ids, float* kl, int32_t* ref_argmax,
-                                  int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
-                                  int32_t* dev_status, void* stream, int32_t ctas_per_row) {
+// kld_full_vocab with the number of streaming warps forced (0 = automatic),
+// to test how pieces of rows merge.  Exported for tests; not in kld.h.
+kld_status kld_full_vocab_split(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
+                                int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
+                                const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                                int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream,
+                                int32_t warps) {
   return full_vocab_impl(ref_logits, cand_logits, dtype, n_rows, vocab, ld_ref, ld_cand, target_ids, kl,
-                         ref_argmax, cand_argmax, ref_target_lp, cand_target_lp, dev_status, stream,
-                         ctas_per_row);
+                         ref_argmax, cand_argmax, ref_target_lp, cand_target_lp, workspace, workspace_bytes,
+                         dev_status, stream, warps);
 }
 
 kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp, const int32_t* cand_ids,

@@ -22,8 +22,12 @@ struct FullVocabArgs {
   float* lpx;
   float* lpy;
   int32_t* dev_status;
-  int cluster_override;  // 0: choose from the vocabulary size
+  void* workspace;       // >= full_vocab_workspace_bytes(n_rows)
+  int warps_override;    // 0: choose from the problem size
 };
+// Upper bound on the streaming warps (fixed, so results do not depend on the device).
+constexpr int kFullVocabMaxWarps = 148 * 32;
+size_t full_vocab_workspace_bytes(int64_t n_rows);
 cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream);
 
 struct TopkTailArgs {

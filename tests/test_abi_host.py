@@ -51,10 +51,12 @@ MIS = A16 + 4          # 4-byte aligned only
 
 def fv(lib, **kw):
     a = dict(ref=A16, cand=A16 + 4096, dtype=_lib.KLD_BF16, n=4, V=64, ldr=64, ldc=64, tgt=None,
-             kl=A16 + 8192, ra=None, ca=None, lpr=None, lpc=None, st=None)
+             kl=A16 + 8192, ra=None, ca=None, lpr=None, lpc=None, ws=A16 + 65536, wsb=None, st=None)
     a.update(kw)
+    wsb = lib.kld_full_vocab_workspace_size(max(a["n"], 0)) if a["wsb"] is None else a["wsb"]
     return lib.kld_full_vocab(a["ref"], a["cand"], a["dtype"], a["n"], a["V"], a["ldr"], a["ldc"],
-                              a["tgt"], a["kl"], a["ra"], a["ca"], a["lpr"], a["lpc"], a["st"], None)
+                              a["tgt"], a["kl"], a["ra"], a["ca"], a["lpr"], a["lpc"], a["ws"], wsb,
+                              a["st"], None)
 
 
 def test_full_vocab_validation(lib):
@@ -69,11 +71,16 @@ def test_full_vocab_validation(lib):
     assert fv(lib, ldr=68, V=64) == _lib.KLD_ERR_ALIGNMENT        # 136 B rows
     assert fv(lib, dtype=_lib.KLD_F32, ldr=66) == _lib.KLD_ERR_ALIGNMENT
     assert fv(lib, kl=A16 + 2) == _lib.KLD_ERR_ALIGNMENT
+    assert fv(lib, ws=None) == _lib.KLD_ERR_WORKSPACE
+    assert fv(lib, wsb=64) == _lib.KLD_ERR_WORKSPACE
+    assert fv(lib, ws=A16 + 16) == _lib.KLD_ERR_ALIGNMENT
     assert fv(lib, n=0) == _lib.KLD_OK                            # nothing to launch
-    assert fv(lib, n=0, ref=None, cand=None, kl=None) == _lib.KLD_OK
-    st = lib.kld_full_vocab_cluster(A16, A16, _lib.KLD_BF16, 4, 64, 64, 64, None, A16, None, None,
-                                    None, None, None, None, 9)
+    assert fv(lib, n=0, ref=None, cand=None, kl=None, ws=None) == _lib.KLD_OK
+    st = lib.kld_full_vocab_split(A16, A16, _lib.KLD_BF16, 4, 64, 64, 64, None, A16, None, None,
+                                  None, None, A16, 1 << 20, None, None, -1)
     assert st == _lib.KLD_ERR_INVALID_ARG
+    assert lib.kld_full_vocab_workspace_size(0) > 0
+    assert lib.kld_full_vocab_workspace_size(1000) > lib.kld_full_vocab_workspace_size(10)
 
 
 def tk(lib, **kw):

@@ -52,14 +52,15 @@ def test_ragged_vocab(cuda_device, dtype, vocab):
     check_full_vocab(res, to_f64(ref), to_f64(cand), tg.cpu().numpy())
 
 
-@pytest.mark.parametrize("ctas", [1, 2, 3, 5, 8])
-def test_cta_split_and_padded_rows(cuda_device, ctas):
+@pytest.mark.parametrize("warps", [1, 2, 3, 7, 20, 64, 500, 4736])
+def test_warp_split_and_padded_rows(cuda_device, warps):
+    """Rows cut into pieces at every position a warp range can end, merged back."""
     V, ld = 30_011, 30_016
     d = W.window_full_vocab(seed=W.SEED_BASE + 200, device=cuda_device, n_rows=21, vocab=ld,
                             dtype=torch.bfloat16, sigma=0.03)
     ref, cand = d["ref"][:, :V], d["cand"][:, :V]
     tg = torch.remainder(d["targets"], V).to(torch.int32)
-    res = run(ref, cand, tg, ctas_per_row=ctas)
+    res = run(ref, cand, tg, warps=warps)
     check_full_vocab(res, to_f64(ref), to_f64(cand), tg.cpu().numpy())
 
 
@@ -98,8 +99,8 @@ def test_batched_f32_full_size_sampled(cuda_device):
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_identical_inputs_give_exact_zero(cuda_device, dtype):
     ref, _, tg = ragged(W.SEED_BASE + 300, cuda_device, 64, 100_003, dtype)
-    for ctas in (0, 1, 3, 8):
-        res = run(ref, same_layout_copy(ref), tg, ctas_per_row=ctas)
+    for warps in (0, 1, 3, 64, 1000):
+        res = run(ref, same_layout_copy(ref), tg, warps=warps)
         assert torch.all(res["kl"] == 0.0)
         assert torch.equal(res["ref_argmax"], res["cand_argmax"])
         assert torch.equal(res["ref_target_lp"], res["cand_target_lp"])
@@ -111,6 +112,17 @@ def test_deterministic(cuda_device):
     for o in outs[1:]:
         for k in ("kl", "ref_argmax", "cand_argmax", "ref_target_lp", "cand_target_lp"):
             assert torch.equal(o[k], outs[0][k]), k
+    # other splits give the same argmaxes and KLs within the contract
+    other = run(d["ref"], d["cand"], d["targets"], warps=333)
+    assert torch.equal(other["ref_argmax"], outs[0]["ref_argmax"])
+    assert torch.allclose(other["kl"], outs[0]["kl"], rtol=1e-4, atol=1e-6)
+
+
+def test_many_pieces_per_row(cuda_device):
+    """Few rows, many warps: a row spans more than 32 pieces (chunked merge)."""
+    d = W.window_full_vocab(seed=W.SEED_BASE + 450, device=cuda_device, n_rows=3, vocab=W.VOCAB)
+    res = run(d["ref"], d["cand"], d["targets"], warps=150)
+    check_full_vocab(res, to_f64(d["ref"]), to_f64(d["cand"]), d["targets"].cpu().numpy())
 
 
 def test_closed_forms_on_gpu(cuda_device):
