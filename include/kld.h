@@ -130,6 +130,40 @@ kld_status kld_full_vocab(const void* ref_logits, const void* cand_logits, kld_d
 size_t kld_full_vocab_workspace_size(int64_t n_rows);
 
 /*
+ * kld_full_vocab_noalloc - kld_full_vocab for callers that cannot allocate
+ * device memory.
+ *
+ * No counterpart on the pages: this entry exists for the library's users,
+ * not for the method.  Some callers cannot call cudaMalloc, or hand this
+ * library a workspace, at the point where they score: code running inside
+ * another framework that owns every byte of device memory through its own
+ * pool and forbids side allocations, a process already at its memory limit,
+ * or a latency-sensitive loop where an allocation (which may synchronise the
+ * device) is not acceptable.  They pass inputs and outputs only; the scratch
+ * lives in a fixed device array inside the library.
+ *
+ * Same arguments and results as kld_full_vocab without the workspace.
+ * Limits and behaviour:
+ *   - n_rows <= KLD_NOALLOC_MAX_ROWS; larger n_rows returns
+ *     KLD_ERR_UNSUPPORTED and launches nothing (split the batch instead).
+ *   - The array takes about 1.2 MB on every GPU that loads the library and
+ *     stays allocated until the process exits.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array.  Calls that may overlap
+ *     on the GPU (different streams, or several host threads) race and can
+ *     corrupt each other's results: serialise them.  The array keeps the last
+ *     call's contents; nothing in it needs to start at zero.
+ */
+#define KLD_NOALLOC_MAX_ROWS 32768
+kld_status kld_full_vocab_noalloc(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
+                                  int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
+                                  const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                                  int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
+                                  int32_t* dev_status, void* stream);
+
+/*
  * kld_topk_tail - KL over the reference's top-k ids plus one tail bucket.
  *
  * Defines ("Qwopus3.8-27B-Coder-Flash: quality-eval reference", "Method";

@@ -24,6 +24,8 @@ KLD_DEV_TIMEOUT = 0x4
 KLD_F32 = 0
 KLD_BF16 = 1
 
+KLD_NOALLOC_MAX_ROWS = 32768
+
 KLD_MAX_QUANTILES = 8
 KLD_MAX_THRESHOLDS = 8
 
@@ -64,6 +66,8 @@ PROTOTYPES = {
     "kld_full_vocab": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P, _P,
                                       _P, _P, _P, _SZ, _P, _P]),
     "kld_full_vocab_workspace_size": (_SZ, [_I64]),
+    "kld_full_vocab_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
+                                              _P, _P, _P, _P, _P]),
     "kld_topk_tail": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I64, _P, _P, _P, _P, _P]),
     "kld_reduce_workspace_size": (_SZ, [_I64]),
     "kld_reduce_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _I32, _P, _P,

@@ -21,6 +21,7 @@
 // log-prob).
 #include <cuda_bf16.h>
 #include <cfloat>
+#include <mutex>
 
 #include "kld_common.cuh"
 #include "launch.h"
@@ -433,7 +434,35 @@ int stream_warps(int64_t total, int override_warps) {
   return (int)w;
 }
 
+// Library-owned scratch for kld_full_vocab_noalloc: room for the row pieces
+// of up to kNoAllocMaxRows rows.  Every device that loads this module holds
+// it until the process exits; all calls on a device share it.
+constexpr int64_t kNoAllocRows = kNoAllocMaxRows;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(Piece) * (kNoAllocRows + kMaxStreamWarps)];
+
 }  // namespace
+
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
+  // Host code cannot use g_noalloc_scratch's name as a device address: look
+  // the address up once per device, with that device current, and cache it.
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* cached[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cached[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    cached[dev] = p;
+  }
+  *ptr = cached[dev];
+  *bytes = sizeof(g_noalloc_scratch);
+  return cudaSuccess;
+}
 
 size_t full_vocab_workspace_bytes(int64_t n_rows) {
   return sizeof(Piece) * (size_t)(n_rows + kMaxStreamWarps);

@@ -92,6 +92,23 @@ kld_status kld_full_vocab(const void* ref_logits, const void* cand_logits, kld_d
                          dev_status, stream, 0);
 }
 
+// kld_full_vocab for callers that cannot allocate: the scratch is the
+// library's own device array (see kld.h).  Too many rows is refused before
+// any CUDA call; every other argument is checked by kld_full_vocab.
+kld_status kld_full_vocab_noalloc(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
+                                  int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
+                                  const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                                  int32_t* cand_argmax, float* ref_target_lp, float* cand_target_lp,
+                                  int32_t* dev_status, void* stream) {
+  if (n_rows > kld::kNoAllocMaxRows) return KLD_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  if (n_rows > 0 && kld::noalloc_scratch(&scratch, &scratch_bytes) != cudaSuccess) return KLD_ERR_CUDA;
+  return kld_full_vocab(ref_logits, cand_logits, dtype, n_rows, vocab, ld_ref, ld_cand, target_ids, kl,
+                        ref_argmax, cand_argmax, ref_target_lp, cand_target_lp, scratch, scratch_bytes,
+                        dev_status, stream);
+}
+
 // kld_full_vocab with the number of streaming warps forced (0 = automatic),
 // to test how pieces of rows merge.  Exported for tests; not in kld.h.
 kld_status kld_full_vocab_split(const void* ref_logits, const void* cand_logits, kld_dtype dtype,

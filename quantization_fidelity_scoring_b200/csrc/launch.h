@@ -29,6 +29,11 @@ struct FullVocabArgs {
 constexpr int kFullVocabMaxWarps = 148 * 32;
 size_t full_vocab_workspace_bytes(int64_t n_rows);
 cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream);
+// Rows the library-owned scratch of kld_full_vocab_noalloc can hold.
+constexpr int64_t kNoAllocMaxRows = KLD_NOALLOC_MAX_ROWS;
+// Device address and size of that scratch on the current device (looked up
+// on the first call per device).
+cudaError_t noalloc_scratch(void** ptr, size_t* bytes);
 
 struct TopkTailArgs {
   const int32_t* ref_ids;
