@@ -317,8 +317,12 @@ def run_ours(args) -> int:
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded Zipf/Gumbel logits; no corpus or model)",
             "config": config_dict(args.rows), "roofline": roofline,
-            "clocks": sampler.summary(t0, t1), "gpu_launches": 2 * args.steps, "e2e": e2e,
+            "clocks": sampler.summary(t0, t1), "gpu_launches": launches_per_step(n) * args.steps,
+            "e2e": e2e,
         }
+        if not args.no_extra:
+            line["extra_paths"] = {"topk_tail": measure_topk(args, kq, dev),
+                                   "shared_head": measure_shared_head(args, kq, dev)}
         if world == 1 and not args.no_cpu_baseline:
             rows = list(range(0, n, max(1, n // args.cpu_rows)))[:args.cpu_rows]
             dt = oracle_rows(ref, cand, targets, rows)
@@ -329,6 +333,125 @@ def run_ours(args) -> int:
     if line is not None:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def launches_per_step(n: int) -> int:
+    """Library kernels per step: streaming pass + piece merge + reduction
+    (one CTA up to 65,536 positions, else zero + 4 passes + final)."""
+    return 2 + (1 if n <= 65536 else 6)
+
+
+def measure_topk(args, kq, dev) -> dict:
+    """Top-64 + tail bucket on its full workload (512 windows x 2047
+    positions): kld_topk_tail + kld_reduce_stats (mean/p50/p99/p99.9, top-1,
+    both perplexities), inputs resident, larger than L2."""
+    import torch
+    from synth import workloads as W
+    d = W.topk_tail_windows(seed=W.seed_for(4), device=dev)
+    ri, rl = d["ref_ids"].reshape(-1, 64), d["ref_lp"].reshape(-1, 64)
+    ci, cl = d["cand_ids"].reshape(-1, 64), d["cand_lp"].reshape(-1, 64)
+    rt, ct = d["ref_target_lp"].reshape(-1), d["cand_target_lp"].reshape(-1)
+    n = ri.shape[0]
+    kl = torch.empty(n, dtype=torch.float32, device=dev)
+    top1 = torch.empty(n, dtype=torch.uint8, device=dev)
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    out = torch.empty(280, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kq.kld_topk_tail(ri, rl, ci, cl, d["vocab"], kl=kl, top1=top1, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kq.kld_reduce_stats(kl, None, None, top1, rt, ct, None, QUANTILES, (), out=out, workspace=ws,
+                            stream=stream, to_host=False)
+
+    steps = max(1, min(args.steps, 100))
+    for _ in range(max(3, args.warmup)):
+        step()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        step(kev[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(stop) / steps
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    alg = n * (2 * 64 * 4 + 2 * 64 * 2 + 4 + 1)   # both lists in, kl and top-1 out
+    peak, _ = measured_peaks()
+    return {"workload": "top-64 + tail bucket: 512 windows x 2047 positions, V=248,320",
+            "value": n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "step": "kld_topk_tail + kld_reduce_stats", "gpu_launches_per_step": 1 + launches_per_step(n) - 2,
+            "roofline": {"bound": "hbm", "achieved": alg / (k_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": alg / (k_ms / 1e3) / 1e9 / peak, "kernel": "kld::topk_tail_kernel",
+                         "kernel_ms": k_ms}}
+
+
+def measured_tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), float(d["bf16_tflops"]), "measured"
+    return 1400.0, 1590.0, "fallback"
+
+
+def measure_shared_head(args, kq, dev, n_rows=8192, hidden=5120, vocab=VOCAB, steps=None) -> dict:
+    """Fused shared head (hidden states through one bf16 head, logits in
+    tensor memory only): kld_from_hidden_shared_head + kld_reduce_stats."""
+    import torch
+    from synth import workloads as W
+    d = W.shared_head_states(seed=W.seed_for(5), device=dev, n_rows=n_rows, hidden=hidden, vocab=vocab)
+    n = n_rows
+    kl = torch.empty(n, dtype=torch.float32, device=dev)
+    ra = torch.empty(n, dtype=torch.int32, device=dev)
+    ca = torch.empty(n, dtype=torch.int32, device=dev)
+    lpr = torch.empty(n, dtype=torch.float32, device=dev)
+    lpc = torch.empty(n, dtype=torch.float32, device=dev)
+    hws = torch.empty(kq.kld_shared_head_workspace_size(n, hidden, vocab), dtype=torch.uint8, device=dev)
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    out = torch.empty(280, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kq.kld_from_hidden_shared_head(d["h_ref"], d["h_cand"], d["W"], d["targets"], kl=kl, ref_argmax=ra,
+                                       cand_argmax=ca, ref_target_lp=lpr, cand_target_lp=lpc, workspace=hws,
+                                       dev_status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=out, workspace=ws,
+                            stream=stream, to_host=False)
+
+    steps = steps or max(1, min(args.steps, 10))
+    for _ in range(3):
+        step()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        step(kev[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item()}"
+    ms = start.elapsed_time(stop) / steps
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    flop = 2.0 * 2.0 * n * vocab * hidden          # both sides' logits
+    sustained, burst, kind = measured_tensor_peak()
+    achieved = flop / (k_ms / 1e3) / 1e12
+    return {"workload": f"fused shared head: {n} positions, hidden {hidden}, head {vocab} x {hidden} bf16",
+            "value": n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "step": "kld_from_hidden_shared_head + kld_reduce_stats",
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                         "frac": achieved / sustained, "frac_of_burst_peak": achieved / burst,
+                         "kernel": "kld::head_kernel + kld::head_merge_kernel", "kernel_ms": k_ms,
+                         "peak_source": f"{kind} bf16_tflops_sustained (burst {burst})"}}
 
 
 def measure_e2e(args, kq, d, dev, world) -> dict:
@@ -408,6 +531,9 @@ def main(argv=None) -> int:
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the top-64 and shared-head lines")
+    ap.add_argument("--profile-head", nargs=2, type=int, metavar=("ROWS", "VOCAB"),
+                    help="only time the shared-head path at a reduced size (for profiling)")
     ap.add_argument("--rows", type=int, default=N_ROWS,
                     help="positions per window (default 2047; smaller only for profiling runs)")
     args = ap.parse_args(argv)
@@ -415,6 +541,14 @@ def main(argv=None) -> int:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_head:
+        import torch
+        import quantization_fidelity_scoring_b200 as kq
+        kq.load_library()
+        r = measure_shared_head(args, kq, torch.device("cuda:0"), n_rows=args.profile_head[0],
+                                vocab=args.profile_head[1], steps=args.steps)
+        print(json.dumps(r), flush=True)
+        return 0
     return run_ours(args)
 
 

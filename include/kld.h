@@ -197,6 +197,35 @@ kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp,
                          int32_t* dev_status, void* stream);
 
 /*
+ * kld_from_hidden_shared_head - full-vocabulary scoring from final hidden
+ * states pushed through one shared LM head.
+ *
+ * Defines ("Qwen3.8-27B fidelity suite v5", opening paragraph: KLD from final
+ * hidden states through one shared BF16 LM head, so no candidate is credited
+ * or penalised for its own head): with x = W h_ref[r] and y = W h_cand[r]
+ * (logits accumulated in f32 on the tensor cores, never rounded to bf16 and
+ * never written to memory), the outputs are those of kld_full_vocab on x, y.
+ *
+ * Arguments:
+ *   h_ref, h_cand   bf16 [n_rows, hidden] row-major, 16-byte aligned.
+ *   head_w          bf16 [vocab, hidden] row-major, 16-byte aligned.
+ *   hidden          8 .. 2^20, a multiple of 8.   vocab: 1 .. 2^31 - 1.
+ *   target_ids .. cand_target_lp, dev_status: as in kld_full_vocab.
+ *   workspace       >= kld_shared_head_workspace_size(n_rows, hidden, vocab)
+ *                   bytes, 256-byte aligned (per 256-id vocabulary tile and
+ *                   row, 32 bytes of partial state).
+ * A bounded wait inside the kernel that gives up (after about 2 s) sets
+ * KLD_DEV_TIMEOUT; the outputs are then invalid.
+ */
+size_t kld_shared_head_workspace_size(int64_t n_rows, int64_t hidden, int64_t vocab);
+kld_status kld_from_hidden_shared_head(const void* h_ref, const void* h_cand, const void* head_w,
+                                       int64_t n_rows, int64_t hidden, int64_t vocab,
+                                       const int32_t* target_ids, float* kl, int32_t* ref_argmax,
+                                       int32_t* cand_argmax, float* ref_target_lp,
+                                       float* cand_target_lp, void* workspace, size_t workspace_bytes,
+                                       int32_t* dev_status, void* stream);
+
+/*
  * Result of kld_reduce_stats, written to DEVICE memory.  Plain C layout:
  * 8-byte fields first, then 4-byte fields; sizeof = 360 on LP64.
  */

@@ -188,6 +188,14 @@ def shared_head(H_ref, H_cand, W, targets=None, v_chunk: int = 1 << 15) -> dict:
     return res
 
 
+def logit_error_bound(H_row: np.ndarray, W_row, unit_roundoff=2.0 ** -24) -> float:
+    """gamma_K * sum_k |h_k w_k|: the standard bound on the error of an
+    f32-accumulated dot product of length K (Higham, "Accuracy and Stability
+    of Numerical Algorithms", Sec. 3.1)."""
+    h = np.abs(np.asarray(H_row, dtype=np.float64))
+    return H_row.shape[0] * unit_roundoff * float(h @ np.abs(np.asarray(W_row, dtype=np.float64)))
+
+
 def argmax_ambiguous(logits_row: np.ndarray, H_row: np.ndarray, W, unit_roundoff=2.0 ** -24) -> bool:
     """True when the row's top-2 logits are closer than twice the standard
     f32 dot-product error bound gamma_K * sum_k |h_k w_vk| (gamma_K = K u,

@@ -69,6 +69,9 @@ PROTOTYPES = {
     "kld_full_vocab_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
                                               _P, _P, _P, _P, _P]),
     "kld_topk_tail": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I64, _P, _P, _P, _P, _P]),
+    "kld_shared_head_workspace_size": (_SZ, [_I64, _I64, _I64]),
+    "kld_from_hidden_shared_head": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
+                                                   _SZ, _P, _P]),
     "kld_reduce_workspace_size": (_SZ, [_I64]),
     "kld_reduce_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _I32, _P, _P,
                                         _SZ, _P, _P]),
@@ -76,6 +79,7 @@ PROTOTYPES = {
 
 # exported for tests only (not part of the public header)
 TEST_PROTOTYPES = {
+    "kld_from_hidden_shared_head_withhold": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P, _P]),
     "kld_full_vocab_split": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
                                             _P, _P, _P, _P, _SZ, _P, _P, _I32]),
 }

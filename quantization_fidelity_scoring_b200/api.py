@@ -122,6 +122,46 @@ def kld_topk_tail(ref_ids, ref_lp, cand_ids, cand_lp, vocab: int, *, kl=None, to
     return dict(kl=kl, top1=top1, n_matched=n_matched)
 
 
+def kld_from_hidden_shared_head(h_ref, h_cand, head_w, targets=None, *, argmax: bool = True, kl=None,
+                                ref_argmax=None, cand_argmax=None, ref_target_lp=None, cand_target_lp=None,
+                                workspace=None, dev_status=None, stream=None) -> dict:
+    """Full-vocabulary scores of hidden states [n, K] (bf16) through one
+    head W [V, K] (bf16), all contiguous.  Outputs and the workspace are
+    allocated when not given."""
+    for name, t in (("h_ref", h_ref), ("h_cand", h_cand), ("head_w", head_w)):
+        _need_cuda(name, t, torch.bfloat16, 2)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if h_ref.shape != h_cand.shape or head_w.shape[1] != h_ref.shape[1]:
+        raise ValueError("shape mismatch between hidden states and head")
+    n, K = h_ref.shape
+    V = head_w.shape[0]
+    dev = h_ref.device
+    if targets is not None:
+        _need_cuda("targets", targets, torch.int32, 1)
+    kl = _out(kl, n, torch.float32, dev)
+    if argmax:
+        ref_argmax = _out(ref_argmax, n, torch.int32, dev)
+        cand_argmax = _out(cand_argmax, n, torch.int32, dev)
+    if targets is not None:
+        ref_target_lp = _out(ref_target_lp, n, torch.float32, dev)
+        cand_target_lp = _out(cand_target_lp, n, torch.float32, dev)
+    lib = _lib.load()
+    if workspace is None:
+        workspace = torch.empty(lib.kld_shared_head_workspace_size(n, K, V), dtype=torch.uint8, device=dev)
+    st = lib.kld_from_hidden_shared_head(_ptr(h_ref), _ptr(h_cand), _ptr(head_w), n, K, V, _ptr(targets),
+                                         _ptr(kl), _ptr(ref_argmax), _ptr(cand_argmax), _ptr(ref_target_lp),
+                                         _ptr(cand_target_lp), _ptr(workspace), workspace.numel(),
+                                         _ptr(dev_status), _stream_handle(stream))
+    _check(st, "kld_from_hidden_shared_head")
+    return dict(kl=kl, ref_argmax=ref_argmax, cand_argmax=cand_argmax, ref_target_lp=ref_target_lp,
+                cand_target_lp=cand_target_lp)
+
+
+def kld_shared_head_workspace_size(n_rows: int, hidden: int, vocab: int) -> int:
+    return int(_lib.load().kld_shared_head_workspace_size(n_rows, hidden, vocab))
+
+
 def kld_full_vocab_workspace_size(n_rows: int) -> int:
     return int(_lib.load().kld_full_vocab_workspace_size(n_rows))
 

@@ -377,6 +377,7 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(const MergeParams p) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
   constexpr int kElemBytes = kBF16 ? 2 : 4;
+  wait_prior_grid();
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (row >= p.n_rows) return;
@@ -485,9 +486,8 @@ cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream) {
   MergeParams mp{a.x, a.y, a.ld_x, a.ld_y, (int)a.vocab, nvec, (int)a.n_rows, nwarps, total, pieces,
                  a.targets, a.kl, a.ax, a.ay, a.lpx, a.lpy, a.dev_status};
   const unsigned mgrid = (unsigned)((a.n_rows + kWarpsPerCta - 1) / kWarpsPerCta);
-  if (a.bf16) merge_kernel<true><<<mgrid, kThreads, 0, stream>>>(mp);
-  else merge_kernel<false><<<mgrid, kThreads, 0, stream>>>(mp);
-  return cudaGetLastError();
+  if (a.bf16) return launch_dependent(merge_kernel<true>, dim3(mgrid), dim3(kThreads), stream, mp);
+  return launch_dependent(merge_kernel<false>, dim3(mgrid), dim3(kThreads), stream, mp);
 }
 
 }  // namespace kld

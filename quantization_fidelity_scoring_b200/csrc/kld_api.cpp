@@ -148,6 +148,67 @@ kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp, const i
   return cuda_status(kld::launch_topk_tail(a, static_cast<cudaStream_t>(stream)));
 }
 
+static kld_status shared_head_impl(const void* h_ref, const void* h_cand, const void* head_w, int64_t n_rows,
+                                   int64_t hidden, int64_t vocab, const int32_t* target_ids, float* kl,
+                                   int32_t* ref_argmax, int32_t* cand_argmax, float* ref_target_lp,
+                                   float* cand_target_lp, void* workspace, size_t workspace_bytes,
+                                   int32_t* dev_status, void* stream, int withhold) {
+  if (n_rows < 0 || vocab < 1 || vocab > INT32_MAX || hidden < 8 || hidden > (1 << 20) || hidden % 8 != 0)
+    return KLD_ERR_INVALID_ARG;
+  if (!target_ids && (ref_target_lp || cand_target_lp)) return KLD_ERR_INVALID_ARG;
+  if (n_rows == 0) return KLD_OK;
+  if (n_rows > INT32_MAX / 2) return KLD_ERR_UNSUPPORTED;
+  if (!h_ref || !h_cand || !head_w || !kl) return KLD_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < kld::shared_head_workspace_bytes(n_rows, vocab)) return KLD_ERR_WORKSPACE;
+  if (!aligned(h_ref, 16) || !aligned(h_cand, 16) || !aligned(head_w, 16) || !aligned(workspace, 256))
+    return KLD_ERR_ALIGNMENT;
+  if (!aligned(kl, 4) || !aligned(ref_argmax, 4) || !aligned(cand_argmax, 4) || !aligned(ref_target_lp, 4) ||
+      !aligned(cand_target_lp, 4) || !aligned(target_ids, 4) || !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+  kld::SharedHeadArgs a;
+  a.h_ref = h_ref;
+  a.h_cand = h_cand;
+  a.head_w = head_w;
+  a.n_rows = n_rows;
+  a.hidden = hidden;
+  a.vocab = vocab;
+  a.targets = target_ids;
+  a.kl = kl;
+  a.ax = ref_argmax;
+  a.ay = cand_argmax;
+  a.lpx = ref_target_lp;
+  a.lpy = cand_target_lp;
+  a.workspace = workspace;
+  a.dev_status = dev_status;
+  a.withhold = withhold;
+  return cuda_status(kld::launch_shared_head(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t kld_shared_head_workspace_size(int64_t n_rows, int64_t hidden, int64_t vocab) {
+  (void)hidden;
+  if (n_rows < 0 || vocab < 1) return 0;
+  return kld::shared_head_workspace_bytes(n_rows, vocab);
+}
+
+kld_status kld_from_hidden_shared_head(const void* h_ref, const void* h_cand, const void* head_w, int64_t n_rows,
+                                       int64_t hidden, int64_t vocab, const int32_t* target_ids, float* kl,
+                                       int32_t* ref_argmax, int32_t* cand_argmax, float* ref_target_lp,
+                                       float* cand_target_lp, void* workspace, size_t workspace_bytes,
+                                       int32_t* dev_status, void* stream) {
+  return shared_head_impl(h_ref, h_cand, head_w, n_rows, hidden, vocab, target_ids, kl, ref_argmax, cand_argmax,
+                          ref_target_lp, cand_target_lp, workspace, workspace_bytes, dev_status, stream, 0);
+}
+
+// Test hook, not in kld.h: withhold the first TMA fill so that the kernel's
+// bounded waits run out and report KLD_DEV_TIMEOUT.
+kld_status kld_from_hidden_shared_head_withhold(const void* h_ref, const void* h_cand, const void* head_w,
+                                                int64_t n_rows, int64_t hidden, int64_t vocab, float* kl,
+                                                void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                                void* stream) {
+  return shared_head_impl(h_ref, h_cand, head_w, n_rows, hidden, vocab, nullptr, kl, nullptr, nullptr, nullptr,
+                          nullptr, workspace, workspace_bytes, dev_status, stream, 1);
+}
+
 size_t kld_reduce_workspace_size(int64_t n) { return kld::reduce_workspace_bytes(n); }
 
 kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,

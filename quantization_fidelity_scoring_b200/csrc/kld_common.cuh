@@ -177,4 +177,27 @@ __device__ __forceinline__ void set_dev_status(int32_t* dev_status, int bits) {
   if (dev_status) atomicOr(reinterpret_cast<int*>(dev_status), bits);
 }
 
+// Programmatic dependent launch.  A kernel launched with launch_dependent()
+// may be scheduled while the previous kernel on the stream is still
+// finishing, which hides its launch latency; it must call
+// wait_prior_grid() before touching memory the previous kernels use (the
+// wait returns at once when the kernel was launched the ordinary way).
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, cudaStream_t stream,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace kld

@@ -50,6 +50,24 @@ struct TopkTailArgs {
 };
 cudaError_t launch_topk_tail(const TopkTailArgs& a, cudaStream_t stream);
 
+struct SharedHeadArgs {
+  const void* h_ref;   // bf16 [n_rows, hidden]
+  const void* h_cand;  // bf16 [n_rows, hidden]
+  const void* head_w;  // bf16 [vocab, hidden]
+  int64_t n_rows, hidden, vocab;
+  const int32_t* targets;
+  float* kl;
+  int32_t* ax;
+  int32_t* ay;
+  float* lpx;
+  float* lpy;
+  void* workspace;     // >= shared_head_workspace_bytes(n_rows, vocab)
+  int32_t* dev_status;
+  int withhold;        // tests only (see shared_head.cu)
+};
+size_t shared_head_workspace_bytes(int64_t n_rows, int64_t vocab);
+cudaError_t launch_shared_head(const SharedHeadArgs& a, cudaStream_t stream);
+
 struct ReduceArgs {
   const float* kl;
   const int32_t* ref_argmax;

@@ -28,7 +28,7 @@ constexpr int kPasses = 4;
 constexpr int64_t kSmallN = 65536;
 constexpr int kBigThreads = 256;
 constexpr int kMaxBigBlocks = 1024;
-constexpr int kSmallThreads = 1024;
+constexpr int kSmallThreads = 256;
 
 struct Partial {  // per-CTA sums of the first pass
   double kl, nll_r, nll_c;
@@ -220,28 +220,46 @@ __device__ __forceinline__ void partial_add(Partial& a, const Partial& b) {
   for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) a.exceed[j] += b.exceed[j];
 }
 
-// Fixed-order CTA reduction of per-thread partials: warp butterfly, then the
-// warps in order.  Result valid in thread 0.
-__device__ void block_sum(Partial& acc, Partial* sh_warp) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+__device__ __forceinline__ Partial shfl_down_partial(const Partial& a, int off, int nt) {
+  Partial o;
+  o.kl = __shfl_down_sync(0xffffffffu, a.kl, off);
+  o.nll_r = __shfl_down_sync(0xffffffffu, a.nll_r, off);
+  o.nll_c = __shfl_down_sync(0xffffffffu, a.nll_c, off);
+  o.n = __shfl_down_sync(0xffffffffu, a.n, off);
+  o.n_nan = __shfl_down_sync(0xffffffffu, a.n_nan, off);
+  o.agree = __shfl_down_sync(0xffffffffu, a.agree, off);
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j)
+    o.exceed[j] = (j < nt) ? __shfl_down_sync(0xffffffffu, a.exceed[j], off) : 0;
+  return o;
+}
+
+// Fixed-order CTA reduction of per-thread partials: a butterfly in every
+// warp, then warp 0 does the same over the warp totals.  Result valid in
+// thread 0.  Call from every thread.
+__device__ void block_sum(Partial& acc, Partial* sh_warp, int nt) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    Partial o;
-    o.kl = __shfl_down_sync(0xffffffffu, acc.kl, off);
-    o.nll_r = __shfl_down_sync(0xffffffffu, acc.nll_r, off);
-    o.nll_c = __shfl_down_sync(0xffffffffu, acc.nll_c, off);
-    o.n = __shfl_down_sync(0xffffffffu, acc.n, off);
-    o.n_nan = __shfl_down_sync(0xffffffffu, acc.n_nan, off);
-    o.agree = __shfl_down_sync(0xffffffffu, acc.agree, off);
-    for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) o.exceed[j] = __shfl_down_sync(0xffffffffu, acc.exceed[j], off);
+    const Partial o = shfl_down_partial(acc, off, nt);
     if (lane < off) partial_add(acc, o);
   }
   if (lane == 0) sh_warp[w] = acc;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    Partial t = sh_warp[0];
-    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) partial_add(t, sh_warp[i]);
-    acc = t;
+  if (w == 0) {
+    Partial t;
+    if (lane < nw) {
+      t = sh_warp[lane];
+    } else {
+      t.kl = t.nll_r = t.nll_c = 0.0;
+      t.n = t.n_nan = t.agree = 0;
+      for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) t.exceed[j] = 0;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const Partial o = shfl_down_partial(t, off, nt);
+      if (lane < off) partial_add(t, o);
+    }
+    if (lane == 0) acc = t;
   }
   __syncthreads();
 }
@@ -283,13 +301,14 @@ __device__ void write_stats(const ReduceParams& p, const Partial& tot, const Sel
 // ---------------------------------------------------------------- one CTA
 
 __global__ void __launch_bounds__(kSmallThreads) reduce_small_kernel(const ReduceParams p) {
+  wait_prior_grid();
   __shared__ unsigned sh[kMaxTargets * kBins];
   __shared__ Partial sh_warp[kSmallThreads / 32];
   __shared__ Select sel;
 
   Partial acc;
   thread_sums(p, threadIdx.x, blockDim.x, acc);
-  block_sum(acc, sh_warp);
+  block_sum(acc, sh_warp, p.nt);
   if (threadIdx.x == 0) {
     select_init(sel, p, acc.n);
   }
@@ -308,6 +327,7 @@ __global__ void __launch_bounds__(kSmallThreads) reduce_small_kernel(const Reduc
 // ---------------------------------------------------------------- many CTAs
 
 __global__ void reduce_zero_kernel(unsigned* hist) {
+  wait_prior_grid();
   for (int i = threadIdx.x; i < kPasses * kMaxTargets * kBins; i += blockDim.x) hist[i] = 0u;
 }
 
@@ -325,6 +345,7 @@ __device__ void select_replay(Select& s, const ReduceParams& p, int pass) {
 }
 
 __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReduceParams p, int pass) {
+  wait_prior_grid();
   __shared__ unsigned sh[kMaxTargets * kBins];
   __shared__ Select sel;
   __shared__ Partial sh_warp[kBigThreads / 32];
@@ -344,7 +365,7 @@ __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReducePa
   if (pass == 0) {
     Partial acc;
     thread_sums(p, begin, stride, acc);
-    block_sum(acc, sh_warp);
+    block_sum(acc, sh_warp, p.nt);
     if (threadIdx.x == 0) p.partials[blockIdx.x] = acc;
   }
   __syncthreads();
@@ -355,6 +376,7 @@ __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReducePa
 }
 
 __global__ void __launch_bounds__(kBigThreads) reduce_final_kernel(const ReduceParams p, int n_partials) {
+  wait_prior_grid();
   __shared__ Select sel;
   select_replay(sel, p, kPasses);
   if (threadIdx.x != 0) return;
@@ -398,15 +420,13 @@ cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
   p.partials = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes);
   p.dev_status = a.dev_status;
 
-  if (a.n <= kSmallN) {
-    reduce_small_kernel<<<1, kSmallThreads, 0, stream>>>(p);
-    return cudaGetLastError();
-  }
+  if (a.n <= kSmallN) return launch_dependent(reduce_small_kernel, dim3(1), dim3(kSmallThreads), stream, p);
   const int grid = big_grid(a.n);
-  reduce_zero_kernel<<<1, 1024, 0, stream>>>(p.hist);
-  for (int pass = 0; pass < kPasses; ++pass) reduce_pass_kernel<<<grid, kBigThreads, 0, stream>>>(p, pass);
-  reduce_final_kernel<<<1, kBigThreads, 0, stream>>>(p, grid);
-  return cudaGetLastError();
+  cudaError_t e = launch_dependent(reduce_zero_kernel, dim3(1), dim3(1024), stream, p.hist);
+  for (int pass = 0; pass < kPasses && e == cudaSuccess; ++pass)
+    e = launch_dependent(reduce_pass_kernel, dim3(grid), dim3(kBigThreads), stream, p, pass);
+  if (e != cudaSuccess) return e;
+  return launch_dependent(reduce_final_kernel, dim3(1), dim3(kBigThreads), stream, p, grid);
 }
 
 }  // namespace kld
