@@ -28,7 +28,7 @@ constexpr int kPasses = 4;
 constexpr int64_t kSmallN = 65536;
 constexpr int kBigThreads = 256;
 constexpr int kMaxBigBlocks = 1024;
-constexpr int kSmallThreads = 256;
+constexpr int kSmallThreads = 512;
 
 struct Partial {  // per-CTA sums of the first pass
   double kl, nll_r, nll_c;
@@ -300,24 +300,55 @@ __device__ void write_stats(const ReduceParams& p, const Partial& tot, const Sel
 
 // ---------------------------------------------------------------- one CTA
 
+// Up to kCacheN scored keys stay in shared memory across the passes; key 0
+// marks a position that is not scored (only NaN bit patterns map to 0).
+constexpr int kCacheN = 6144;
+
 __global__ void __launch_bounds__(kSmallThreads) reduce_small_kernel(const ReduceParams p) {
-  wait_prior_grid();
   __shared__ unsigned sh[kMaxTargets * kBins];
+  __shared__ uint32_t keys[kCacheN];
   __shared__ Partial sh_warp[kSmallThreads / 32];
   __shared__ Select sel;
 
+  wait_prior_grid();
+  const bool cached = p.n <= kCacheN;
   Partial acc;
   thread_sums(p, threadIdx.x, blockDim.x, acc);
-  block_sum(acc, sh_warp, p.nt);
-  if (threadIdx.x == 0) {
-    select_init(sel, p, acc.n);
+  if (cached) {
+    for (int i = threadIdx.x; i < (int)p.n; i += blockDim.x) {
+      float v;
+      keys[i] = scored(p, i, v) ? f2key(v) : 0u;
+    }
   }
+  block_sum(acc, sh_warp, p.nt);
+  if (threadIdx.x == 0) select_init(sel, p, acc.n);
   __syncthreads();
   select_unique(sel);
   for (int pass = 0; pass < kPasses; ++pass) {
     for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) sh[i] = 0u;
     __syncthreads();
-    if (sel.nt > 0) hist_pass(p, sel, pass, threadIdx.x, blockDim.x, sh);
+    if (sel.nt > 0) {
+      if (cached) {
+        const int shift = 24 - 8 * pass;
+        for (int i = threadIdx.x; i < (int)p.n; i += blockDim.x) {
+          const uint32_t key = keys[i];
+          if (key == 0u) continue;
+          const uint32_t digit = (key >> shift) & 0xffu;
+          if (pass == 0) {
+            atomicAdd(&sh[digit], 1u);
+          } else {
+            const uint32_t pre = key >> (shift + 8);
+            for (int u = 0; u < sel.nu; ++u)
+              if (sel.uprefix[u] == pre) {
+                atomicAdd(&sh[u * kBins + digit], 1u);
+                break;
+              }
+          }
+        }
+      } else {
+        hist_pass(p, sel, pass, threadIdx.x, blockDim.x, sh);
+      }
+    }
     __syncthreads();
     select_step(sel, sh);
   }

@@ -1,4 +1,4 @@
-// Top-k + one tail bucket KL, one warp per position.
+// Top-k + one tail bucket KL, a half-warp per position.
 //
 // "Qwopus3.8-27B-Coder-Flash: quality-eval reference", section "Method": the
 // KL runs over the reference's top-64 ids plus one tail bucket; a reference id
@@ -7,11 +7,15 @@
 // is an exact argmax match (the first stored slot, lists being sorted per
 // section "Files").
 //
-// Matching: the candidate's k ids are inserted into a 128-slot open-address
-// table in shared memory (key = id, value = first slot holding it), then each
-// reference id is looked up.  The table gives the same answer whatever order
-// the lanes insert in, so the result is deterministic.  Mass sums are f64
-// butterfly reductions in a fixed lane order.
+// Each 16-lane half of a warp scores one position, so one warp instruction
+// advances two positions; lane l of a half holds list slots l, l+16, l+32,
+// l+48 of both lists.  Matching: the candidate's ids go into a 128-slot
+// open-addressed table in shared memory (key = id, value = first slot holding
+// it; atomicMin keeps the first slot of a repeated id), then each reference
+// id is looked up.  The table gives the same answer whatever order the lanes
+// insert in, so the result is deterministic.  The three masses that feed
+// 1 - sum (candidate list, reference list, matched candidate cells) are f64
+// butterflies in fixed lane order; the KL terms are f32.
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -23,7 +27,9 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSlots = 128;  // >= 2 * 64: probe chains stay short and always end
+constexpr int kHalves = 2 * kWarps;  // positions in flight per CTA
+constexpr int kPer = 4;              // list slots per lane
+constexpr int kSlots = 128;          // >= 2 * 64: probe chains stay short and always end
 constexpr uint32_t kEmpty = 0xffffffffu;
 constexpr double kQFloor = 1e-12;
 
@@ -31,9 +37,15 @@ __device__ __forceinline__ uint32_t slot_of(uint32_t id) { return (id * 0x9E3779
 
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
-__device__ __forceinline__ double warp_sum(double v) {
+// Butterfly sums inside a 16-lane half (offsets 8, 4, 2, 1 stay in the half).
+__device__ __forceinline__ double half_sum(double v) {
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  for (int off = 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+__device__ __forceinline__ float half_sum(float v) {
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   return v;
 }
 
@@ -52,48 +64,57 @@ struct TopkParams {
 };
 
 __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p) {
-  __shared__ uint32_t table[kWarps][kSlots];
-  __shared__ float cand_lp_s[kWarps][64];
+  __shared__ uint32_t table[kHalves][kSlots];
+  __shared__ float cand_lp_s[kHalves][64];
 
+  wait_prior_grid();
   const int lane = threadIdx.x & 31;
-  const int w = threadIdx.x >> 5;
+  const int hl = lane & 15;                       // lane within the half
+  const int half = (threadIdx.x >> 4);            // half index in the CTA
+  const unsigned half_mask = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
   const int k = p.k;
-  uint32_t* tab = table[w];
-  float* clps = cand_lp_s[w];
+  const uint32_t V = (uint32_t)p.vocab;
+  uint32_t* tab = table[half];
+  float* clps = cand_lp_s[half];
 
-  for (int64_t pos = (int64_t)blockIdx.x * kWarps + w; pos < p.n_rows; pos += (int64_t)gridDim.x * kWarps) {
+  const int64_t n_pairs = (p.n_rows + 1) / 2;
+  for (int64_t pair = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); pair < n_pairs;
+       pair += (int64_t)gridDim.x * kWarps) {
+    const int64_t pos = 2 * pair + (lane >> 4);
+    const bool live = pos < p.n_rows;             // the odd tail position's second half idles
     const int64_t base = pos * k;
-    const int j0 = lane, j1 = lane + 32;
-    const bool v0 = j0 < k, v1 = j1 < k;
-    const int32_t r0 = v0 ? p.ref_ids[base + j0] : 0;
-    const int32_t r1 = v1 ? p.ref_ids[base + j1] : 0;
-    const int32_t c0 = v0 ? p.cand_ids[base + j0] : 0;
-    const int32_t c1 = v1 ? p.cand_ids[base + j1] : 0;
-    const float a0 = v0 ? h2f(p.ref_lp[base + j0]) : 0.f;
-    const float a1 = v1 ? h2f(p.ref_lp[base + j1]) : 0.f;
-    const float b0 = v0 ? h2f(p.cand_lp[base + j0]) : 0.f;
-    const float b1 = v1 ? h2f(p.cand_lp[base + j1]) : 0.f;
 
-    const uint32_t V = (uint32_t)p.vocab;
-    const bool bad_lane = (v0 && ((uint32_t)r0 >= V || (uint32_t)c0 >= V)) ||
-                          (v1 && ((uint32_t)r1 >= V || (uint32_t)c1 >= V));
-    const bool bad = __any_sync(0xffffffffu, bad_lane);
-
-    // clear this warp's table, publish candidate log-probs
+    int32_t r[kPer], c[kPer];
+    float a[kPer], b[kPer];
+    bool valid[kPer];
 #pragma unroll
-    for (int s = lane; s < kSlots; s += 32) tab[s] = kEmpty;
-    if (v0) clps[j0] = b0;
-    if (v1) clps[j1] = b1;
+    for (int i = 0; i < kPer; ++i) {
+      const int j = hl + 16 * i;
+      valid[i] = live && j < k;
+      r[i] = valid[i] ? p.ref_ids[base + j] : 0;
+      c[i] = valid[i] ? p.cand_ids[base + j] : 0;
+      a[i] = valid[i] ? h2f(p.ref_lp[base + j]) : 0.f;
+      b[i] = valid[i] ? h2f(p.cand_lp[base + j]) : 0.f;
+    }
+    bool bad_lane = false;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      bad_lane |= valid[i] && ((uint32_t)r[i] >= V || (uint32_t)c[i] >= V);
+    const bool bad = (__ballot_sync(0xffffffffu, bad_lane) & half_mask) != 0;
+
+    // clear this half's table, publish the candidate log-probs
+#pragma unroll
+    for (int s = hl; s < kSlots; s += 16) tab[s] = kEmpty;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (valid[i]) clps[hl + 16 * i] = b[i];
     __syncwarp();
-
     if (!bad) {
-      // insert candidate ids; a repeated id keeps its lowest slot
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const bool valid = h == 0 ? v0 : v1;
-        if (!valid) continue;
-        const uint32_t id = (uint32_t)(h == 0 ? c0 : c1);
-        const uint32_t entry = (id << 6) | (uint32_t)(h == 0 ? j0 : j1);
+      for (int i = 0; i < kPer; ++i) {
+        if (!valid[i]) continue;
+        const uint32_t id = (uint32_t)c[i];
+        const uint32_t entry = (id << 6) | (uint32_t)(hl + 16 * i);
         uint32_t s = slot_of(id);
         for (int probe = 0; probe < kSlots; ++probe) {
           const uint32_t old = atomicCAS(&tab[s], kEmpty, entry);
@@ -108,15 +129,14 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
     }
     __syncwarp();
 
-    // per reference slot: matched candidate slot or -1
-    double p_sum = 0.0, c_sum = 0.0, qm_sum = 0.0, pu_sum = 0.0, pau_sum = 0.0, klm = 0.0;
-    int unmatched = 0, matched = 0;
+    double c_sum = 0.0, p_sum = 0.0, qm_sum = 0.0;
+    float klm = 0.f, pau = 0.f, pu = 0.f;
+    int matched = 0;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const bool valid = h == 0 ? v0 : v1;
-      if (!valid || bad) continue;
-      const uint32_t id = (uint32_t)(h == 0 ? r0 : r1);
-      const float a = h == 0 ? a0 : a1;
+    for (int i = 0; i < kPer; ++i) {
+      if (!valid[i] || bad) continue;
+      c_sum += (double)expf(b[i]);
+      const uint32_t id = (uint32_t)r[i];
       int slot = -1;
       uint32_t s = slot_of(id);
       for (int probe = 0; probe < kSlots; ++probe) {
@@ -128,32 +148,29 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
         }
         s = (s + 1) & (kSlots - 1);
       }
-      const double pj = (double)expf(a);
-      p_sum += pj;
+      const float pj = expf(a[i]);
+      p_sum += (double)pj;
       if (slot >= 0) {
-        const float b = clps[slot];
-        qm_sum += (double)expf(b);
-        klm += pj * ((double)a - (double)b);
+        const float bm = clps[slot];
+        qm_sum += (double)expf(bm);
+        klm += pj * (a[i] - bm);
         ++matched;
       } else {
-        pu_sum += pj;
-        pau_sum += pj * (double)a;
-        ++unmatched;
+        pu += pj;
+        pau += pj * a[i];
       }
     }
-    if (v0) c_sum += (double)expf(b0);
-    if (v1) c_sum += (double)expf(b1);
+    c_sum = half_sum(c_sum);
+    p_sum = half_sum(p_sum);
+    qm_sum = half_sum(qm_sum);
+    klm = half_sum(klm);
+    pau = half_sum(pau);
+    pu = half_sum(pu);
+    int m_total = matched;
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) m_total += __shfl_xor_sync(0xffffffffu, m_total, off);
 
-    p_sum = warp_sum(p_sum);
-    c_sum = warp_sum(c_sum);
-    qm_sum = warp_sum(qm_sum);
-    pu_sum = warp_sum(pu_sum);
-    pau_sum = warp_sum(pau_sum);
-    klm = warp_sum(klm);
-    unmatched = __reduce_add_sync(0xffffffffu, unmatched);
-    matched = __reduce_add_sync(0xffffffffu, matched);
-
-    if (lane == 0) {
+    if (hl == 0 && live) {
       float out;
       if (bad) {
         out = CUDART_NAN_F;
@@ -161,19 +178,21 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
       } else {
         const double leftover = fmax(1.0 - c_sum, 0.0);
         const double spread = leftover / (double)(p.vocab - k);
-        const double log_spread = log(fmax(spread, kQFloor));
+        const float log_spread = logf((float)fmax(spread, kQFloor));
+        const int unmatched = k - m_total;
         const double q_sum = qm_sum + (double)unmatched * spread;
         const double p_tail = 1.0 - p_sum;
         const double q_tail = 1.0 - q_sum;
-        double kl = klm + pau_sum - log_spread * pu_sum;
-        if (p_tail > 0.0) kl += p_tail * (log(p_tail) - log(fmax(q_tail, kQFloor)));
-        out = (float)kl;
+        float kl = klm + pau - log_spread * pu;
+        if (p_tail > 0.0)
+          kl += (float)p_tail * (logf((float)p_tail) - logf((float)fmax(q_tail, kQFloor)));
+        out = kl;
       }
       p.kl[pos] = out;
-      if (p.top1) p.top1[pos] = (uint8_t)(r0 == c0);
-      if (p.n_matched) p.n_matched[pos] = bad ? -1 : matched;
+      if (p.top1) p.top1[pos] = (uint8_t)(r[0] == c[0]);
+      if (p.n_matched) p.n_matched[pos] = bad ? -1 : m_total;
     }
-    __syncwarp();  // the table is cleared again for the next position
+    __syncwarp();  // the tables are cleared again for the next pair
   }
 }
 
@@ -195,11 +214,11 @@ cudaError_t launch_topk_tail(const TopkTailArgs& a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t need = (a.n_rows + kWarps - 1) / kWarps;
+  const int64_t pairs = (a.n_rows + 1) / 2;
+  const int64_t need = (pairs + kWarps - 1) / kWarps;
   const int64_t cap = (int64_t)sms * 8;  // 8 resident CTAs of 256 threads per SM
   const unsigned grid = (unsigned)(need < cap ? need : cap);
-  topk_tail_kernel<<<grid, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(topk_tail_kernel, dim3(grid), dim3(kThreads), stream, p);
 }
 
 }  // namespace kld
