@@ -341,13 +341,13 @@ def launches_per_step(n: int) -> int:
     return 2 + (1 if n <= 65536 else 6)
 
 
-def measure_topk(args, kq, dev) -> dict:
+def measure_topk(args, kq, dev, windows=512, steps=None) -> dict:
     """Top-64 + tail bucket on its full workload (512 windows x 2047
     positions): kld_topk_tail + kld_reduce_stats (mean/p50/p99/p99.9, top-1,
     both perplexities), inputs resident, larger than L2."""
     import torch
     from synth import workloads as W
-    d = W.topk_tail_windows(seed=W.seed_for(4), device=dev)
+    d = W.topk_tail_windows(seed=W.seed_for(4), device=dev, windows=windows)
     ri, rl = d["ref_ids"].reshape(-1, 64), d["ref_lp"].reshape(-1, 64)
     ci, cl = d["cand_ids"].reshape(-1, 64), d["cand_lp"].reshape(-1, 64)
     rt, ct = d["ref_target_lp"].reshape(-1), d["cand_target_lp"].reshape(-1)
@@ -367,7 +367,7 @@ def measure_topk(args, kq, dev) -> dict:
         kq.kld_reduce_stats(kl, None, None, top1, rt, ct, None, QUANTILES, (), out=out, workspace=ws,
                             stream=stream, to_host=False)
 
-    steps = max(1, min(args.steps, 100))
+    steps = steps or max(1, min(args.steps, 100))
     for _ in range(max(3, args.warmup)):
         step()
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -382,7 +382,7 @@ def measure_topk(args, kq, dev) -> dict:
     k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
     alg = n * (2 * 64 * 4 + 2 * 64 * 2 + 4 + 1)   # both lists in, kl and top-1 out
     peak, _ = measured_peaks()
-    return {"workload": "top-64 + tail bucket: 512 windows x 2047 positions, V=248,320",
+    return {"workload": f"top-64 + tail bucket: {windows} windows x 2047 positions, V=248,320",
             "value": n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
             "step": "kld_topk_tail + kld_reduce_stats", "gpu_launches_per_step": 1 + launches_per_step(n) - 2,
             "roofline": {"bound": "hbm", "achieved": alg / (k_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
@@ -532,6 +532,8 @@ def main(argv=None) -> int:
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the top-64 and shared-head lines")
+    ap.add_argument("--profile-topk", type=int, metavar="WINDOWS",
+                    help="only time the top-64 + tail path on WINDOWS windows (for profiling)")
     ap.add_argument("--profile-head", nargs=2, type=int, metavar=("ROWS", "VOCAB"),
                     help="only time the shared-head path at a reduced size (for profiling)")
     ap.add_argument("--rows", type=int, default=N_ROWS,
@@ -541,6 +543,13 @@ def main(argv=None) -> int:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_topk:
+        import torch
+        import quantization_fidelity_scoring_b200 as kq
+        kq.load_library()
+        print(json.dumps(measure_topk(args, kq, torch.device("cuda:0"), windows=args.profile_topk,
+                                      steps=args.steps)), flush=True)
+        return 0
     if args.profile_head:
         import torch
         import quantization_fidelity_scoring_b200 as kq

@@ -1,4 +1,4 @@
-// Top-k + one tail bucket KL, a half-warp per position.
+// Top-k + one tail bucket KL, sixteen lanes per position.
 //
 // "Qwopus3.8-27B-Coder-Flash: quality-eval reference", section "Method": the
 // KL runs over the reference's top-64 ids plus one tail bucket; a reference id
@@ -8,14 +8,18 @@
 // section "Files").
 //
 // Each 16-lane half of a warp scores one position, so one warp instruction
-// advances two positions; lane l of a half holds list slots l, l+16, l+32,
-// l+48 of both lists.  Matching: the candidate's ids go into a 128-slot
-// open-addressed table in shared memory (key = id, value = first slot holding
-// it; atomicMin keeps the first slot of a repeated id), then each reference
-// id is looked up.  The table gives the same answer whatever order the lanes
-// insert in, so the result is deterministic.  The three masses that feed
-// 1 - sum (candidate list, reference list, matched candidate cells) are f64
-// butterflies in fixed lane order; the KL terms are f32.
+// advances two positions.  Lane l of a half holds list slots 4l .. 4l+3
+// (vector loads when k is a multiple of 4; element loads otherwise).
+// Matching: the candidate's ids go into a 256-slot open-addressed table in
+// shared memory whose 64-bit entries hold (id, slot, fp16 log-prob); the
+// load factor is at most 1/4, so almost every insert and lookup finishes at
+// its first probe and lanes rarely diverge, and the two halves' tables are
+// offset by 16 banks.  A repeated candidate id keeps its lowest slot
+// (atomicMin on the packed entry).  Results do not depend on the order of
+// insertion, so they are deterministic.  The three masses that feed 1 - sum
+// (candidate list, reference list, matched candidate cells) use the accurate
+// expf and are accumulated in f64, in fixed lane order; the KL terms are f32
+// and the tail term takes one logarithm of the f64 ratio p_tail / q_tail.
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
@@ -27,25 +31,38 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kHalves = 2 * kWarps;  // positions in flight per CTA
-constexpr int kPer = 4;              // list slots per lane
-constexpr int kSlots = 128;          // >= 2 * 64: probe chains stay short and always end
-constexpr uint32_t kEmpty = 0xffffffffu;
+constexpr int kGroup = 16;                   // lanes per position
+constexpr int kPerWarp = 32 / kGroup;        // positions per warp
+constexpr int kPer = 64 / kGroup;            // list slots per lane
+constexpr int kPositions = kWarps * kPerWarp;
+constexpr int kSlots = 256;                  // >= 4 * 64: short probe chains that always end
+constexpr int kTableStride = kSlots + 8;     // 64-bit words; next table starts 16 banks over
+constexpr unsigned long long kEmpty = ~0ull;
 constexpr double kQFloor = 1e-12;
+constexpr float kLn2 = 0.6931471805599453f;
 
-__device__ __forceinline__ uint32_t slot_of(uint32_t id) { return (id * 0x9E3779B1u) >> 25; }
+__device__ __forceinline__ uint32_t slot_of(uint32_t id) { return (id * 0x9E3779B1u) >> 24; }
 
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
-// Butterfly sums inside a 16-lane half (offsets 8, 4, 2, 1 stay in the half).
-__device__ __forceinline__ double half_sum(double v) {
-#pragma unroll
-  for (int off = 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
+__device__ __forceinline__ float fast_log(float x) {
+  float r;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r * kLn2;
 }
-__device__ __forceinline__ float half_sum(float v) {
+
+// Entry: id in bits 22..46, list slot in 16..21, fp16 log-prob bits in 0..15.
+// For equal ids the lower slot is the smaller entry.
+__device__ __forceinline__ unsigned long long pack(uint32_t id, int slot, uint16_t lp) {
+  return ((unsigned long long)id << 22) | ((unsigned long long)slot << 16) | lp;
+}
+__device__ __forceinline__ uint32_t entry_id(unsigned long long e) { return (uint32_t)(e >> 22); }
+
+// Butterfly sums inside a 16-lane group (offsets 8, 4, 2, 1 stay in the group).
+template <typename T>
+__device__ __forceinline__ T group_sum(T v) {
 #pragma unroll
-  for (int off = 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  for (int off = kGroup / 2; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
   return v;
 }
 
@@ -57,69 +74,94 @@ struct TopkParams {
   int64_t n_rows;
   int k;
   int vocab;
+  double inv_spread_ids;  // 1 / (vocab - k)
+  bool vec;               // aligned rows for vector loads: k % 4 == 0
   float* kl;
   uint8_t* top1;
   int32_t* n_matched;
   int32_t* dev_status;
 };
 
+// Load slots 4l .. 4l+3 of one list (ids int32, log-probs as fp16 bits).
+__device__ __forceinline__ void load_list(const TopkParams& p, const int32_t* ids, const uint16_t* lps,
+                                          int64_t base, int gl, bool live, int32_t (&id)[kPer],
+                                          uint16_t (&lp)[kPer], bool (&valid)[kPer]) {
+  const int j0 = gl * kPer;
+  if (p.vec && live && j0 + kPer <= p.k) {
+    const int4 i4 = __ldg(reinterpret_cast<const int4*>(ids + base + j0));
+    const uint2 l2 = __ldg(reinterpret_cast<const uint2*>(lps + base + j0));
+    id[0] = i4.x;
+    id[1] = i4.y;
+    id[2] = i4.z;
+    id[3] = i4.w;
+    lp[0] = (uint16_t)(l2.x & 0xffffu);
+    lp[1] = (uint16_t)(l2.x >> 16);
+    lp[2] = (uint16_t)(l2.y & 0xffffu);
+    lp[3] = (uint16_t)(l2.y >> 16);
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) valid[t] = true;
+    return;
+  }
+#pragma unroll
+  for (int t = 0; t < kPer; ++t) {
+    const int j = j0 + t;
+    valid[t] = live && j < p.k;
+    id[t] = valid[t] ? ids[base + j] : 0;
+    lp[t] = valid[t] ? lps[base + j] : (uint16_t)0;
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p) {
-  __shared__ uint32_t table[kHalves][kSlots];
-  __shared__ float cand_lp_s[kHalves][64];
+  __shared__ __align__(16) unsigned long long table[kPositions * kTableStride];
 
   wait_prior_grid();
   const int lane = threadIdx.x & 31;
-  const int hl = lane & 15;                       // lane within the half
-  const int half = (threadIdx.x >> 4);            // half index in the CTA
-  const unsigned half_mask = (lane < 16) ? 0x0000ffffu : 0xffff0000u;
+  const int gl = lane & (kGroup - 1);             // lane within the group
+  const int grp = lane / kGroup;                  // group within the warp
+  const int gslot = threadIdx.x / kGroup;         // group index in the CTA
+  const unsigned gmask = 0xffffu << (grp * kGroup);
   const int k = p.k;
   const uint32_t V = (uint32_t)p.vocab;
-  uint32_t* tab = table[half];
-  float* clps = cand_lp_s[half];
+  unsigned long long* tab = table + gslot * kTableStride;
 
-  const int64_t n_pairs = (p.n_rows + 1) / 2;
-  for (int64_t pair = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); pair < n_pairs;
-       pair += (int64_t)gridDim.x * kWarps) {
-    const int64_t pos = 2 * pair + (lane >> 4);
-    const bool live = pos < p.n_rows;             // the odd tail position's second half idles
+  const int64_t n_iter = (p.n_rows + kPerWarp - 1) / kPerWarp;
+  for (int64_t it = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); it < n_iter;
+       it += (int64_t)gridDim.x * kWarps) {
+    const int64_t pos = it * kPerWarp + grp;
+    const bool live = pos < p.n_rows;
     const int64_t base = pos * k;
 
     int32_t r[kPer], c[kPer];
-    float a[kPer], b[kPer];
-    bool valid[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int j = hl + 16 * i;
-      valid[i] = live && j < k;
-      r[i] = valid[i] ? p.ref_ids[base + j] : 0;
-      c[i] = valid[i] ? p.cand_ids[base + j] : 0;
-      a[i] = valid[i] ? h2f(p.ref_lp[base + j]) : 0.f;
-      b[i] = valid[i] ? h2f(p.cand_lp[base + j]) : 0.f;
-    }
+    uint16_t ra[kPer], cb[kPer];
+    bool valid[kPer], vc[kPer];
+    load_list(p, p.ref_ids, p.ref_lp, base, gl, live, r, ra, valid);
+    load_list(p, p.cand_ids, p.cand_lp, base, gl, live, c, cb, vc);
+
     bool bad_lane = false;
 #pragma unroll
     for (int i = 0; i < kPer; ++i)
       bad_lane |= valid[i] && ((uint32_t)r[i] >= V || (uint32_t)c[i] >= V);
-    const bool bad = (__ballot_sync(0xffffffffu, bad_lane) & half_mask) != 0;
+    const bool bad = (__ballot_sync(0xffffffffu, bad_lane) & gmask) != 0;
 
-    // clear this half's table, publish the candidate log-probs
+    // clear this group's table: 16 lanes x 8 stores of 16 bytes
+    {
+      ulonglong2* t2 = reinterpret_cast<ulonglong2*>(tab);
+      const ulonglong2 e2 = make_ulonglong2(kEmpty, kEmpty);
 #pragma unroll
-    for (int s = hl; s < kSlots; s += 16) tab[s] = kEmpty;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      if (valid[i]) clps[hl + 16 * i] = b[i];
+      for (int s = gl; s < kSlots / 2; s += kGroup) t2[s] = e2;
+    }
     __syncwarp();
     if (!bad) {
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
         if (!valid[i]) continue;
         const uint32_t id = (uint32_t)c[i];
-        const uint32_t entry = (id << 6) | (uint32_t)(hl + 16 * i);
+        const unsigned long long entry = pack(id, gl * kPer + i, cb[i]);
         uint32_t s = slot_of(id);
         for (int probe = 0; probe < kSlots; ++probe) {
-          const uint32_t old = atomicCAS(&tab[s], kEmpty, entry);
+          const unsigned long long old = atomicCAS(&tab[s], kEmpty, entry);
           if (old == kEmpty) break;
-          if ((old >> 6) == id) {
+          if (entry_id(old) == id) {
             atomicMin(&tab[s], entry);
             break;
           }
@@ -132,67 +174,60 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
     double c_sum = 0.0, p_sum = 0.0, qm_sum = 0.0;
     float klm = 0.f, pau = 0.f, pu = 0.f;
     int matched = 0;
+    if (!bad) {
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      if (!valid[i] || bad) continue;
-      c_sum += (double)expf(b[i]);
-      const uint32_t id = (uint32_t)r[i];
-      int slot = -1;
-      uint32_t s = slot_of(id);
-      for (int probe = 0; probe < kSlots; ++probe) {
-        const uint32_t e = tab[s];
-        if (e == kEmpty) break;
-        if ((e >> 6) == id) {
-          slot = (int)(e & 63u);
-          break;
+      for (int i = 0; i < kPer; ++i) {
+        if (!valid[i]) continue;
+        const float a = h2f(ra[i]);
+        const float pj = expf(a);
+        c_sum += (double)expf(h2f(cb[i]));
+        p_sum += (double)pj;
+        const uint32_t id = (uint32_t)r[i];
+        uint32_t s = slot_of(id);
+        unsigned long long e = tab[s];
+        for (int probe = 1; probe < kSlots && e != kEmpty && entry_id(e) != id; ++probe) {
+          s = (s + 1) & (kSlots - 1);  // rare at load factor 1/4
+          e = tab[s];
         }
-        s = (s + 1) & (kSlots - 1);
-      }
-      const float pj = expf(a[i]);
-      p_sum += (double)pj;
-      if (slot >= 0) {
-        const float bm = clps[slot];
-        qm_sum += (double)expf(bm);
-        klm += pj * (a[i] - bm);
-        ++matched;
-      } else {
-        pu += pj;
-        pau += pj * a[i];
+        if (e != kEmpty && entry_id(e) == id) {
+          const float bm = h2f((uint16_t)(e & 0xffffu));
+          qm_sum += (double)expf(bm);
+          klm += pj * (a - bm);
+          ++matched;
+        } else {
+          pu += pj;
+          pau += pj * a;
+        }
       }
     }
-    c_sum = half_sum(c_sum);
-    p_sum = half_sum(p_sum);
-    qm_sum = half_sum(qm_sum);
-    klm = half_sum(klm);
-    pau = half_sum(pau);
-    pu = half_sum(pu);
-    int m_total = matched;
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) m_total += __shfl_xor_sync(0xffffffffu, m_total, off);
+    c_sum = group_sum(c_sum);
+    p_sum = group_sum(p_sum);
+    qm_sum = group_sum(qm_sum);
+    klm = group_sum(klm);
+    pau = group_sum(pau);
+    pu = group_sum(pu);
+    matched = group_sum(matched);
 
-    if (hl == 0 && live) {
+    if (gl == 0 && live) {
       float out;
       if (bad) {
         out = CUDART_NAN_F;
         set_dev_status(p.dev_status, 0x2 /* KLD_DEV_BAD_ID */);
       } else {
-        const double leftover = fmax(1.0 - c_sum, 0.0);
-        const double spread = leftover / (double)(p.vocab - k);
-        const float log_spread = logf((float)fmax(spread, kQFloor));
-        const int unmatched = k - m_total;
-        const double q_sum = qm_sum + (double)unmatched * spread;
+        const double spread = fmax(1.0 - c_sum, 0.0) * p.inv_spread_ids;
+        const float log_spread = fast_log((float)fmax(spread, kQFloor));
+        const double q_sum = qm_sum + (double)(k - matched) * spread;
         const double p_tail = 1.0 - p_sum;
         const double q_tail = 1.0 - q_sum;
         float kl = klm + pau - log_spread * pu;
-        if (p_tail > 0.0)
-          kl += (float)p_tail * (logf((float)p_tail) - logf((float)fmax(q_tail, kQFloor)));
+        if (p_tail > 0.0) kl += (float)p_tail * logf((float)(p_tail / fmax(q_tail, kQFloor)));
         out = kl;
       }
       p.kl[pos] = out;
       if (p.top1) p.top1[pos] = (uint8_t)(r[0] == c[0]);
-      if (p.n_matched) p.n_matched[pos] = bad ? -1 : m_total;
+      if (p.n_matched) p.n_matched[pos] = bad ? -1 : matched;
     }
-    __syncwarp();  // the tables are cleared again for the next pair
+    __syncwarp();  // the tables are cleared again for the next positions
   }
 }
 
@@ -207,6 +242,10 @@ cudaError_t launch_topk_tail(const TopkTailArgs& a, cudaStream_t stream) {
   p.n_rows = a.n_rows;
   p.k = a.k;
   p.vocab = (int)a.vocab;
+  p.inv_spread_ids = 1.0 / (double)(a.vocab - a.k);
+  const auto al = [](const void* q, uintptr_t n) { return (reinterpret_cast<uintptr_t>(q) % n) == 0; };
+  // 4 ids (16 B) and 4 fp16 log-probs (8 B) per lane: rows aligned when k % 4 == 0
+  p.vec = (a.k % 4 == 0) && al(a.ref_ids, 16) && al(a.cand_ids, 16) && al(a.ref_lp, 8) && al(a.cand_lp, 8);
   p.kl = a.kl;
   p.top1 = a.top1;
   p.n_matched = a.n_matched;
@@ -214,9 +253,9 @@ cudaError_t launch_topk_tail(const TopkTailArgs& a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t pairs = (a.n_rows + 1) / 2;
-  const int64_t need = (pairs + kWarps - 1) / kWarps;
-  const int64_t cap = (int64_t)sms * 8;  // 8 resident CTAs of 256 threads per SM
+  const int64_t iters = (a.n_rows + kPerWarp - 1) / kPerWarp;
+  const int64_t need = (iters + kWarps - 1) / kWarps;
+  const int64_t cap = (int64_t)sms * 8;
   const unsigned grid = (unsigned)(need < cap ? need : cap);
   return launch_dependent(topk_tail_kernel, dim3(grid), dim3(kThreads), stream, p);
 }
