@@ -133,6 +133,36 @@ class ClockSampler:
                 "samples_in_timed_region": len(inside), "samples": len(use)}
 
 
+def rank_env(default_world: int = 1):
+    """(world size, rank, local rank) from the torchrun environment."""
+    world = int(os.environ.get("WORLD_SIZE", str(default_world)))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def window_seed(rank: int) -> int:
+    """Every rank scores its own window: distinct seeded inputs per rank."""
+    from synth import workloads as W
+    return W.seed_for(2) + 1000 * rank
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The slowest rank's time (all ranks take part; a no-op for one rank)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(n_per_rank: int, world: int, steps: int, seconds: float) -> float:
+    """Positions scored by all ranks per second of the slowest rank."""
+    return n_per_rank * world * steps / seconds
+
+
 def oracle_rows(ref, cand, targets, rows):
     """Run the f64 oracle on the given row indices (host copies); returns seconds."""
     import numpy as np
@@ -161,13 +191,12 @@ def run_reference(args) -> int:
     import torch
     from oracle import kld_oracle as O
     from synth import workloads as W
-    rank = int(os.environ.get("RANK", "0"))
+    world, rank, _ = rank_env(default_world=args.gpus)
     if rank != 0:
         return 0
-    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
     # inputs drawn on the GPU when there is one (same bytes as our arm), else on the host
     dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
-    budget_s = 90.0
+    budget_s = args.ref_seconds
     per_row_s = 0.02
     rows_per_step = max(1, min(256, int(budget_s / ((args.steps + args.warmup) * per_row_s))))
     d = W.window_full_vocab(seed=W.seed_for(2), device=dev, n_rows=min(N_ROWS, max(2 * rows_per_step, 64)))
@@ -221,9 +250,7 @@ def run_ours(args) -> int:
     import quantization_fidelity_scoring_b200 as kq
     from synth import workloads as W
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -231,7 +258,7 @@ def run_ours(args) -> int:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     kq.load_library()
 
-    d = W.window_full_vocab(seed=W.seed_for(2) + 1000 * rank, device=dev, n_rows=args.rows)
+    d = W.window_full_vocab(seed=window_seed(rank), device=dev, n_rows=args.rows)
     ref, cand, targets = d["ref"], d["cand"], d["targets"]
     n = ref.shape[0]
     stream = torch.cuda.current_stream()
@@ -285,14 +312,10 @@ def run_ours(args) -> int:
     sampler.stop()
     ms = start.elapsed_time(stop)
     k_ms = [a.elapsed_time(b) for a, b in kev]
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, dev, world)
     assert status.item() == 0, f"device status {status.item()}"
 
-    positions = n * world * args.steps
-    value = positions / (ms / 1e3)
+    value = whole_job_rate(n, world, args.steps, ms / 1e3)
 
     # roofline of the dominant kernel (full-vocabulary pass)
     alg_bytes = 2 * n * VOCAB * 2 + n * (4 + 4 * 5)   # both logit rows, targets, five outputs
@@ -510,13 +533,9 @@ def measure_e2e(args, kq, d, dev, world) -> dict:
     t0 = time.perf_counter()
     for _ in range(steps):
         step()
-    dt = time.perf_counter() - t0
-    if world > 1:
-        tt = torch.tensor([dt], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        dt = float(tt.item())
+    dt = max_over_ranks(time.perf_counter() - t0, dev, world)
     h2d = h_ref.numel() * 2 + h_cand.numel() * 2 + h_t.numel() * 4
-    return {"value": n * world * steps / dt, "unit": UNIT, "h2d_bytes_per_step": h2d,
+    return {"value": whole_job_rate(n, world, steps, dt), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": 280, "steps": steps,
             "how": "pinned host logits copied in 256-row chunks on a copy stream, overlapped with "
                    "scoring of earlier chunks; stats struct read back each step; wall clock"}
@@ -530,6 +549,8 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-rows", type=int, default=512)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--ref-seconds", type=float, default=90.0,
+                    help="reference arm: CPU seconds the timed and warm-up steps aim for")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the top-64 and shared-head lines")
     ap.add_argument("--profile-topk", type=int, metavar="WINDOWS",
