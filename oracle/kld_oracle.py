@@ -312,6 +312,73 @@ def topk_tail(ref_ids, ref_lp, cand_ids, cand_lp, vocab: int, chunk: int = 8192)
 
 
 # ---------------------------------------------------------------------------
+# candidate full logits against a sparse reference (the challenge score)
+# ---------------------------------------------------------------------------
+
+def sparse_ref_row(y, ref_ids, ref_lp, p_tail=None, target=None) -> dict:
+    """KL over the reference's K listed ids plus one tail cell, from the
+    candidate's full logits y, one position.
+
+    "Qwen3.8-27B Quantization Challenge", "Golden distributions": the
+    reference is stored sparse, as its K most likely ids with f32 log p (most
+    likely first) and, per row, the tail mass 1 - sum exp(top lp) summed
+    over the rest of the full row.  "The score": the candidate's q =
+    softmax(y) is coarsened onto the reference's K + 1 cells (the K listed
+    ids, and one cell holding all the rest of q's mass) and
+    KL(p || q) = sum over cells p_c (log p_c - log q_c).  Top-1 agreement is
+    an argmax match; the reference's argmax is its first listed id.
+
+    p_tail defaults to 1 - sum_R p when the row's stored tail mass is not
+    given.  Listed ids are distinct (a top-K of one distribution); an id
+    outside [0, V) or a repeated id makes the position invalid (KL NaN).
+    """
+    y = as_f64(y)
+    V = y.shape[0]
+    ids = np.asarray(ref_ids).astype(np.int64)
+    lp = as_f64(np.asarray(ref_lp))
+    K = ids.shape[0]
+    out = dict(kl=math.nan, cand_argmax=-1, top1=0, cand_target_lp=math.nan)
+    if not 0 < K <= V or lp.shape != (K,):
+        raise ValueError("need 0 < K <= V listed ids with one log-prob each")
+    if not _row_is_valid(y):
+        return out
+    lq_all = log_softmax(y)
+    out["cand_argmax"] = int(np.argmax(y))
+    out["top1"] = int(int(ids[0]) == out["cand_argmax"])
+    if target is not None and 0 <= int(target) < V:
+        out["cand_target_lp"] = float(lq_all[int(target)])
+    if np.any((ids < 0) | (ids >= V)) or np.unique(ids).shape[0] != K:
+        return out
+    p = np.exp(lp)
+    live = p > 0.0                                  # 0 * log 0 = 0
+    kl = float(np.sum(p[live] * (lp[live] - lq_all[ids][live])))
+    rest = np.ones(V, dtype=bool)
+    rest[ids] = False
+    q_tail = float(np.sum(np.exp(lq_all[rest])))    # the rest of q's mass
+    pt = (1.0 - float(np.sum(p))) if p_tail is None else float(p_tail)
+    if pt > 0.0:
+        kl += pt * (math.log(pt) - math.log(max(q_tail, Q_FLOOR)))
+    out["kl"] = kl
+    return out
+
+
+def sparse_ref(Y, ref_ids, ref_lp, p_tail=None, targets=None) -> dict:
+    """sparse_ref_row for every position: Y [n, V] candidate logits
+    (float64-exact), ref_ids / ref_lp [n, K], p_tail [n] or None."""
+    Y = np.asarray(Y)
+    n = Y.shape[0]
+    kl = np.full(n, np.nan)
+    ca = np.full(n, -1, dtype=np.int64)
+    top1 = np.zeros(n, dtype=np.uint8)
+    ct = np.full(n, np.nan)
+    for i in range(n):
+        r = sparse_ref_row(Y[i], ref_ids[i], ref_lp[i], None if p_tail is None else p_tail[i],
+                           None if targets is None else int(targets[i]))
+        kl[i], ca[i], top1[i], ct[i] = r["kl"], r["cand_argmax"], r["top1"], r["cand_target_lp"]
+    return dict(kl=kl, cand_argmax=ca, top1=top1, cand_target_lp=ct)
+
+
+# ---------------------------------------------------------------------------
 # reductions
 # ---------------------------------------------------------------------------
 

@@ -271,6 +271,111 @@ def pin_tail_self(O):
 
 
 # ---------------------------------------------------------------------------
+# candidate full logits against a sparse reference (K + 1 cells)
+# ---------------------------------------------------------------------------
+
+def _softmax_loop(y):
+    e = [math.exp(v) for v in y]
+    s = sum(e)
+    return [v / s for v in e]
+
+
+def _brute_force_cells_kl(p, q, listed):
+    """KL between p and q coarsened onto the listed singletons plus one cell
+    holding every other id, by enumerating the cells."""
+    cells = [[i] for i in listed] + [[i for i in range(len(p)) if i not in set(listed)]]
+    kl = 0.0
+    for c in cells:
+        P = sum(p[i] for i in c)
+        Q = sum(q[i] for i in c)
+        if P > 0:
+            kl += P * math.log(P / Q)
+    return kl
+
+
+def pin_sparse_brute_force(O):
+    rng = np.random.default_rng(21)
+    for trial in range(300):
+        V = int(rng.integers(2, 17))
+        K = int(rng.integers(1, V + 1))
+        p = list(rng.dirichlet(np.full(V, 0.6)))
+        y = list(rng.normal(0, 1.5, V))
+        q = _softmax_loop(y)
+        listed = sorted(range(V), key=lambda i: -p[i])[:K]
+        lp = np.log([p[i] for i in listed])
+        tail = sum(p[i] for i in range(V) if i not in set(listed))
+        want = _brute_force_cells_kl(p, q, listed)
+        given = O.sparse_ref_row(np.array(y), np.array(listed), lp, tail)
+        assert _close(given["kl"], want, rtol=1e-9, atol=1e-13), (V, K, given, want)
+        if trial % 3 == 0:   # stored tail absent: 1 - sum of the listed masses
+            dflt = O.sparse_ref_row(np.array(y), np.array(listed), lp)
+            assert _close(dflt["kl"], want, rtol=1e-9, atol=1e-12)
+        assert given["cand_argmax"] == max(range(V), key=lambda i: (y[i], -i))
+        assert given["top1"] == int(listed[0] == given["cand_argmax"])
+
+
+def pin_sparse_all_ids_is_full_kl(O):
+    # listing every id makes the coarsening the identity: the full KL
+    rng = np.random.default_rng(22)
+    for V in (5, 64, 1000):
+        x = rng.normal(0, 2, V)
+        y = x + rng.normal(0, 0.3, V)
+        m = x.max()
+        lp = x - (m + math.log(math.fsum(np.exp(x - m))))
+        ids = rng.permutation(V)
+        r = O.sparse_ref_row(y, ids, lp[ids], 0.0)
+        f = O.full_vocab_row(x, y)
+        assert _close(r["kl"], f["kl"], rtol=1e-10, atol=1e-15)
+        assert r["cand_argmax"] == f["cand_argmax"]
+
+
+def pin_sparse_lower_bound_and_self(O):
+    rng = np.random.default_rng(23)
+    for _ in range(50):
+        V = int(rng.integers(50, 400))
+        K = int(rng.integers(1, 40))
+        x = rng.normal(0, 2, V)
+        y = x + rng.normal(0, 0.2, V)
+        m = x.max()
+        lp = x - (m + math.log(math.fsum(np.exp(x - m))))
+        ids = np.argsort(-lp, kind="stable")[:K]
+        rest = np.setdiff1d(np.arange(V), ids)
+        tail = math.fsum(np.exp(lp[rest]))
+        s = O.sparse_ref_row(y, ids, lp[ids], tail)["kl"]
+        assert s <= O.full_vocab_row(x, y)["kl"] + 1e-13     # coarsening lowers KL
+        assert abs(O.sparse_ref_row(x, ids, lp[ids], tail)["kl"]) < 1e-13   # q = p
+
+
+def pin_sparse_binary_closed_form(O):
+    # V = 2, K = 1: cells {a} and {b}; KL = binary KL of p and sigmoid(y_a - y_b)
+    for p, ya, yb in ((0.7, 0.3, -0.4), (0.99, 2.0, 1.0), (0.2, -1.0, 3.0)):
+        q = 1.0 / (1.0 + math.exp(yb - ya))
+        want = p * math.log(p / q) + (1 - p) * math.log((1 - p) / (1 - q))
+        r = O.sparse_ref_row(np.array([ya, yb]), np.array([0]), np.array([math.log(p)]), 1 - p, target=1)
+        assert _close(r["kl"], want, rtol=1e-12)
+        assert _close(r["cand_target_lp"], math.log(1 - q), rtol=1e-12)
+
+
+def pin_sparse_edge_cases(O):
+    y = np.zeros(8)
+    lp = np.log([0.5, 0.25])
+    assert math.isnan(O.sparse_ref_row(y, np.array([0, 8]), lp, 0.25)["kl"])      # id out of range
+    assert math.isnan(O.sparse_ref_row(y, np.array([3, 3]), lp, 0.25)["kl"])      # repeated id
+    bad = y.copy()
+    bad[5] = np.nan
+    r = O.sparse_ref_row(bad, np.array([0, 1]), lp, 0.25)
+    assert math.isnan(r["kl"]) and r["cand_argmax"] == -1
+    ninf = y.copy()
+    ninf[1] = -np.inf                                  # p > 0 on a cell with q = 0
+    assert O.sparse_ref_row(ninf, np.array([0, 1]), lp, 0.25)["kl"] == math.inf
+    # no tail term when the stored tail is not positive; uniform q = 1/8
+    r = O.sparse_ref_row(y, np.array([2, 6]), np.log([0.75, 0.25]), 0.0, target=4)
+    assert _close(r["kl"], 0.75 * math.log(0.75 * 8) + 0.25 * math.log(0.25 * 8), rtol=1e-12)
+    assert _close(r["cand_target_lp"], -math.log(8), rtol=1e-14)
+    assert r["cand_argmax"] == 0 and r["top1"] == 0   # uniform row: lowest index wins
+
+
+# ---------------------------------------------------------------------------
 # reductions
 # ---------------------------------------------------------------------------
 
@@ -402,6 +507,14 @@ MUTANTS = [
     ("percentile index n q", "h = (n - 1) * float(q)", "h = n * float(q) - 0.5"),
     ("mean over all positions", "out[\"mean_kl\"] = exact_mean(vals)",
      "out[\"mean_kl\"] = exact_mean(kl.astype(np.float64))"),
+    ("tail cell keeps listed ids", "rest[ids] = False", "rest[ids[:1]] = False"),
+    ("sparse tail term dropped", "kl += pt * (math.log(pt) - math.log(max(q_tail, Q_FLOOR)))", "kl += 0.0"),
+    ("listed cells scored against p", "kl = float(np.sum(p[live] * (lp[live] - lq_all[ids][live])))",
+     "kl = float(np.sum(p[live] * (lp[live] - lp[live])))"),
+    ("default tail from the candidate", "pt = (1.0 - float(np.sum(p)))",
+     "pt = (1.0 - float(np.sum(np.exp(lq_all[ids]))))"),
+    ("reference top-1 from the last listed id", "out[\"top1\"] = int(int(ids[0]) == out[\"cand_argmax\"])",
+     "out[\"top1\"] = int(int(ids[-1]) == out[\"cand_argmax\"])"),
     ("transposed head", "return np.asarray(H, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T",
      "return (np.asarray(W, dtype=np.float64) @ np.asarray(H, dtype=np.float64).T).T[:, ::-1]"),
 ]
