@@ -36,7 +36,7 @@ QUANTILES = (0.5, 0.99, 0.999)
 WORKLOAD = "one-window full-vocabulary scoring: 2047 positions x 248,320 vocab, bf16 logits"
 PROFILE = os.path.join(ROOT, "profiles", "full_vocab_kernel_window_bf16.txt")
 KERNEL_SOURCES = [os.path.join(ROOT, "quantization_fidelity_scoring_b200", "csrc", f)
-                  for f in ("full_vocab.cu", "kld_common.cuh")]
+                  for f in ("full_vocab.cu", "kld_common.cuh", "stream_common.cuh")]
 
 
 def kernel_digest() -> str:
@@ -345,6 +345,7 @@ def run_ours(args) -> int:
         }
         if not args.no_extra:
             line["extra_paths"] = {"topk_tail": measure_topk(args, kq, dev),
+                                   "sparse_ref": measure_sparse_ref(args, kq, dev),
                                    "shared_head": measure_shared_head(args, kq, dev)}
         if world == 1 and not args.no_cpu_baseline:
             rows = list(range(0, n, max(1, n // args.cpu_rows)))[:args.cpu_rows]
@@ -410,6 +411,63 @@ def measure_topk(args, kq, dev, windows=512, steps=None) -> dict:
             "step": "kld_topk_tail + kld_reduce_stats", "gpu_launches_per_step": 1 + launches_per_step(n) - 2,
             "roofline": {"bound": "hbm", "achieved": alg / (k_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
                          "frac": alg / (k_ms / 1e3) / 1e9 / peak, "kernel": "kld::topk_tail_kernel",
+                         "kernel_ms": k_ms}}
+
+
+def measure_sparse_ref(args, kq, dev, n_rows=N_ROWS, k=512, steps=None) -> dict:
+    """The challenge score on one window: candidate full logits (2047 x
+    248,320 bf16) against a 512-id sparse reference with stored tail masses,
+    kld_sparse_ref_score + kld_reduce_stats, inputs resident, larger than L2."""
+    import torch
+    from synth import workloads as W
+    d = W.sparse_ref_window(seed=W.seed_for(6), device=dev, n_rows=n_rows, k=k)
+    cand, top, rows, tg = d["cand"], d["ref_top"], d["ref_rows"], d["targets"]
+    n = cand.shape[0]
+    kl = torch.empty(n, dtype=torch.float32, device=dev)
+    am = torch.empty(n, dtype=torch.int32, device=dev)
+    top1 = torch.empty(n, dtype=torch.uint8, device=dev)
+    lpc = torch.empty(n, dtype=torch.float32, device=dev)
+    lpr = torch.empty(n, dtype=torch.float32, device=dev)
+    sws = torch.empty(kq.kld_sparse_ref_workspace_size(n, k), dtype=torch.uint8, device=dev)
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    out = torch.empty(280, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kq.kld_sparse_ref_score(cand, top, rows, tg, kl=kl, cand_argmax=am, top1=top1, cand_target_lp=lpc,
+                                ref_target_lp=lpr, workspace=sws, dev_status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kq.kld_reduce_stats(kl, None, None, top1, lpr, lpc, None, QUANTILES, (), out=out, workspace=ws,
+                            stream=stream, to_host=False)
+
+    steps = steps or max(1, min(args.steps, 200))
+    for _ in range(max(3, args.warmup)):
+        step()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        step(kev[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item()}"
+    ms = start.elapsed_time(stop) / steps
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    # candidate row, reference entries and stored row, target in; five outputs
+    alg = n * (VOCAB * 2 + k * 8 + 12 + 4 + 17)
+    peak, _ = measured_peaks()
+    return {"workload": f"challenge score: {n} positions x 248,320 bf16 candidate logits vs "
+                        f"{k}-id sparse reference + tail cell",
+            "value": n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "step": "kld_sparse_ref_score + kld_reduce_stats", "gpu_launches_per_step": launches_per_step(n),
+            "roofline": {"bound": "hbm", "achieved": alg / (k_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": alg / (k_ms / 1e3) / 1e9 / peak,
+                         "kernel": "kld::sparse_stream_kernel<bf16> + kld::sparse_merge_kernel<bf16>",
                          "kernel_ms": k_ms}}
 
 
@@ -555,6 +613,8 @@ def main(argv=None) -> int:
     ap.add_argument("--no-extra", action="store_true", help="skip the top-64 and shared-head lines")
     ap.add_argument("--profile-topk", type=int, metavar="WINDOWS",
                     help="only time the top-64 + tail path on WINDOWS windows (for profiling)")
+    ap.add_argument("--profile-sparse", type=int, metavar="ROWS",
+                    help="only time the sparse-reference score on ROWS positions (for profiling)")
     ap.add_argument("--profile-head", nargs=2, type=int, metavar=("ROWS", "VOCAB"),
                     help="only time the shared-head path at a reduced size (for profiling)")
     ap.add_argument("--rows", type=int, default=N_ROWS,
@@ -570,6 +630,13 @@ def main(argv=None) -> int:
         kq.load_library()
         print(json.dumps(measure_topk(args, kq, torch.device("cuda:0"), windows=args.profile_topk,
                                       steps=args.steps)), flush=True)
+        return 0
+    if args.profile_sparse:
+        import torch
+        import quantization_fidelity_scoring_b200 as kq
+        kq.load_library()
+        print(json.dumps(measure_sparse_ref(args, kq, torch.device("cuda:0"), n_rows=args.profile_sparse,
+                                            steps=args.steps)), flush=True)
         return 0
     if args.profile_head:
         import torch

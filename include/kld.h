@@ -197,6 +197,64 @@ kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp,
                          int32_t* dev_status, void* stream);
 
 /*
+ * kld_sparse_ref_score - the challenge score: a candidate's full logits
+ * against a sparse reference, KL over K + 1 cells.
+ *
+ * Defines ("Qwen3.8-27B Quantization Challenge", "Golden distributions" for
+ * the reference layout, "The score" for the KL): per position, with
+ * reference entries (R_j, a_j), j < k, the k most likely ids and their f32
+ * log-probs (most likely first), reference tail mass p_tail (the mass of
+ * every unlisted id), and candidate logits y over the whole vocabulary,
+ *    q        = softmax(y) over all vocab ids
+ *    q_tail   = sum of q over the ids not in R      (the tail cell)
+ *    p_j      = exp(a_j)
+ *    kl       = sum_j p_j (a_j - log q_{R_j})
+ *             + [p_tail > 0] p_tail (log p_tail - log max(q_tail, 1e-12))
+ *    top1     = (R_0 == cand_argmax)
+ * cand_argmax is the lowest index of the candidate's maximum.  q_tail is
+ * summed over the unlisted ids directly (the listed ids are masked out of
+ * the streaming pass), never formed as 1 - sum_R q, so it stays accurate
+ * when the listed ids hold all but a millionth of the mass.
+ *
+ * Arguments:
+ *   cand_logits      DEVICE [n_rows, ld_cand] f32 or bf16, 16-byte aligned;
+ *                    ld_cand * element size a multiple of 16.
+ *   ref_top          DEVICE kld_top_entry [n_rows, k] (row stride k), 8-byte aligned.
+ *   k                1 .. KLD_SPARSE_MAX_K and k <= vocab; vocab <= 2^22.
+ *   ref_rows         DEVICE f32 [n_rows, 3] per row (NLL of the true next
+ *                    token, entropy, tail mass), or NULL: p_tail is then
+ *                    1 - sum_j p_j (in f64).
+ *   target_ids       DEVICE int32 [n_rows], required when cand_target_lp is given.
+ *   kl               DEVICE f32 [n_rows], required.
+ *   cand_argmax      DEVICE int32 [n_rows], or NULL.
+ *   top1             DEVICE uint8 [n_rows] (0/1), or NULL.
+ *   cand_target_lp   DEVICE f32 [n_rows]: log q of the target, or NULL.
+ *   ref_target_lp    DEVICE f32 [n_rows]: -NLL copied from ref_rows (so the
+ *                    reductions can form the perplexity ratio), or NULL;
+ *                    requires ref_rows.
+ *   workspace        DEVICE, >= kld_sparse_ref_workspace_size(n_rows, k)
+ *                    bytes, 256-byte aligned; holds nothing between calls.
+ * A candidate row holding NaN or +inf, or no finite logit, gives kl NaN,
+ * cand_argmax -1, top1 0 and NaN target log-prob.  A listed id outside
+ * [0, vocab), or repeated within a row, gives kl NaN and sets
+ * KLD_DEV_BAD_ID; a target outside [0, vocab) gives a NaN target log-prob
+ * and sets KLD_DEV_BAD_TARGET.
+ */
+#define KLD_SPARSE_MAX_K 1024
+typedef struct {
+  int32_t id;
+  float lp;
+} kld_top_entry;
+
+size_t kld_sparse_ref_workspace_size(int64_t n_rows, int32_t k);
+kld_status kld_sparse_ref_score(const void* cand_logits, kld_dtype dtype, int64_t n_rows, int64_t vocab,
+                                int64_t ld_cand, const kld_top_entry* ref_top, int32_t k,
+                                const float* ref_rows, const int32_t* target_ids, float* kl,
+                                int32_t* cand_argmax, uint8_t* top1, float* cand_target_lp,
+                                float* ref_target_lp, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, void* stream);
+
+/*
  * kld_from_hidden_shared_head - full-vocabulary scoring from final hidden
  * states pushed through one shared LM head.
  *

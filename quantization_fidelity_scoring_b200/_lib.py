@@ -54,6 +54,8 @@ class KldStats(ctypes.Structure):
 
 assert ctypes.sizeof(KldStats) == 280
 
+KLD_SPARSE_MAX_K = 1024
+
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _I32 = ctypes.c_int32
@@ -69,6 +71,9 @@ PROTOTYPES = {
     "kld_full_vocab_noalloc": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
                                               _P, _P, _P, _P, _P]),
     "kld_topk_tail": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I64, _P, _P, _P, _P, _P]),
+    "kld_sparse_ref_workspace_size": (_SZ, [_I64, _I32]),
+    "kld_sparse_ref_score": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _I32, _P, _P, _P, _P, _P,
+                                            _P, _P, _P, _SZ, _P, _P]),
     "kld_shared_head_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "kld_from_hidden_shared_head": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                                    _SZ, _P, _P]),
@@ -79,6 +84,8 @@ PROTOTYPES = {
 
 # exported for tests only (not part of the public header)
 TEST_PROTOTYPES = {
+    "kld_sparse_ref_score_split": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _I32, _P, _P, _P, _P,
+                                                  _P, _P, _P, _P, _SZ, _P, _P, _I32]),
     "kld_from_hidden_shared_head_withhold": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P, _P]),
     "kld_full_vocab_split": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
                                             _P, _P, _P, _P, _SZ, _P, _P, _I32]),

@@ -122,6 +122,54 @@ def kld_topk_tail(ref_ids, ref_lp, cand_ids, cand_lp, vocab: int, *, kl=None, to
     return dict(kl=kl, top1=top1, n_matched=n_matched)
 
 
+def kld_sparse_ref_score(cand: torch.Tensor, ref_top: torch.Tensor, ref_rows=None, targets=None, *,
+                         kl=None, cand_argmax=None, top1=None, cand_target_lp=None, ref_target_lp=None,
+                         workspace=None, dev_status=None, stream=None, warps: int = 0) -> dict:
+    """Challenge score of candidate logit rows [n, V] (f32 or bf16, unit
+    stride along V) against a sparse reference: ref_top int32 [n, k, 2]
+    holding (id, f32 log-prob bits) pairs, contiguous; ref_rows f32 [n, 3]
+    (NLL, entropy, tail mass) or None.  Outputs and the workspace are
+    allocated when not given.  `warps` forces the number of streaming warps
+    (tests of long pieces and of the piece merge)."""
+    _need_cuda("cand", cand, ndim=2)
+    if cand.dtype not in _DTYPES:
+        raise ValueError("cand must be float32 or bfloat16")
+    if cand.stride(1) != 1:
+        raise ValueError("logit rows must be contiguous along the vocabulary")
+    _need_cuda("ref_top", ref_top, torch.int32, 3)
+    n, V = cand.shape
+    if ref_top.shape[0] != n or ref_top.shape[2] != 2 or not ref_top.is_contiguous():
+        raise ValueError("ref_top must be a contiguous int32 [n, k, 2] tensor")
+    k = ref_top.shape[1]
+    if ref_rows is not None:
+        _need_cuda("ref_rows", ref_rows, torch.float32, 2)
+        if tuple(ref_rows.shape) != (n, 3) or not ref_rows.is_contiguous():
+            raise ValueError("ref_rows must be a contiguous float32 [n, 3] tensor")
+    dev = cand.device
+    kl = _out(kl, n, torch.float32, dev)
+    cand_argmax = _out(cand_argmax, n, torch.int32, dev)
+    top1 = _out(top1, n, torch.uint8, dev)
+    if targets is not None:
+        _need_cuda("targets", targets, torch.int32, 1)
+        cand_target_lp = _out(cand_target_lp, n, torch.float32, dev)
+    if ref_rows is not None:
+        ref_target_lp = _out(ref_target_lp, n, torch.float32, dev)
+    lib = _lib.load()
+    if workspace is None:
+        workspace = torch.empty(lib.kld_sparse_ref_workspace_size(n, k), dtype=torch.uint8, device=dev)
+    args = (_ptr(cand), _DTYPES[cand.dtype], n, V, cand.stride(0), _ptr(ref_top), k, _ptr(ref_rows),
+            _ptr(targets), _ptr(kl), _ptr(cand_argmax), _ptr(top1), _ptr(cand_target_lp), _ptr(ref_target_lp),
+            _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream_handle(stream))
+    st = lib.kld_sparse_ref_score_split(*args, warps) if warps else lib.kld_sparse_ref_score(*args)
+    _check(st, "kld_sparse_ref_score")
+    return dict(kl=kl, cand_argmax=cand_argmax, top1=top1, cand_target_lp=cand_target_lp,
+                ref_target_lp=ref_target_lp)
+
+
+def kld_sparse_ref_workspace_size(n_rows: int, k: int) -> int:
+    return int(_lib.load().kld_sparse_ref_workspace_size(n_rows, k))
+
+
 def kld_from_hidden_shared_head(h_ref, h_cand, head_w, targets=None, *, argmax: bool = True, kl=None,
                                 ref_argmax=None, cand_argmax=None, ref_target_lp=None, cand_target_lp=None,
                                 workspace=None, dev_status=None, stream=None) -> dict:

@@ -148,6 +148,81 @@ kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp, const i
   return cuda_status(kld::launch_topk_tail(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t kld_sparse_ref_workspace_size(int64_t n_rows, int32_t k) {
+  if (n_rows < 0 || k < 1 || k > KLD_SPARSE_MAX_K) return 0;
+  return kld::sparse_ref_workspace_bytes(n_rows, k);
+}
+
+static kld_status sparse_ref_impl(const void* cand_logits, kld_dtype dtype, int64_t n_rows, int64_t vocab,
+                                  int64_t ld_cand, const kld_top_entry* ref_top, int32_t k,
+                                  const float* ref_rows, const int32_t* target_ids, float* kl,
+                                  int32_t* cand_argmax, uint8_t* top1, float* cand_target_lp,
+                                  float* ref_target_lp, void* workspace, size_t workspace_bytes,
+                                  int32_t* dev_status, void* stream, int warps) {
+  if (warps < 0) return KLD_ERR_INVALID_ARG;
+  if (dtype != KLD_F32 && dtype != KLD_BF16) return KLD_ERR_UNSUPPORTED;
+  if (n_rows < 0 || vocab < 1 || ld_cand < vocab || k < 1 || k > KLD_SPARSE_MAX_K || k > vocab)
+    return KLD_ERR_INVALID_ARG;
+  if (vocab > (int64_t(1) << 22)) return KLD_ERR_UNSUPPORTED;
+  if (!target_ids && cand_target_lp) return KLD_ERR_INVALID_ARG;
+  if (!ref_rows && ref_target_lp) return KLD_ERR_INVALID_ARG;
+  if (n_rows == 0) return KLD_OK;
+  if (!cand_logits || !ref_top || !kl) return KLD_ERR_INVALID_ARG;
+  if (n_rows > (int64_t)INT32_MAX - kld::kFullVocabMaxWarps) return KLD_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < kld::sparse_ref_workspace_bytes(n_rows, k)) return KLD_ERR_WORKSPACE;
+  const int64_t esize = dtype == KLD_BF16 ? 2 : 4;
+  if (!aligned(workspace, 256) || !aligned(cand_logits, 16) || (ld_cand * esize) % 16 != 0)
+    return KLD_ERR_ALIGNMENT;
+  if (!aligned(ref_top, 8) || !aligned(ref_rows, 4) || !aligned(target_ids, 4) || !aligned(kl, 4) ||
+      !aligned(cand_argmax, 4) || !aligned(cand_target_lp, 4) || !aligned(ref_target_lp, 4) ||
+      !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+  kld::SparseRefArgs a;
+  a.y = cand_logits;
+  a.bf16 = dtype == KLD_BF16;
+  a.n_rows = n_rows;
+  a.vocab = vocab;
+  a.ld = ld_cand;
+  a.ref_top = ref_top;
+  a.k = k;
+  a.ref_rows = ref_rows;
+  a.targets = target_ids;
+  a.kl = kl;
+  a.argmax = cand_argmax;
+  a.top1 = top1;
+  a.lp_cand = cand_target_lp;
+  a.lp_ref = ref_target_lp;
+  a.workspace = workspace;
+  a.dev_status = dev_status;
+  a.warps_override = warps;
+  return cuda_status(kld::launch_sparse_ref(a, static_cast<cudaStream_t>(stream)));
+}
+
+kld_status kld_sparse_ref_score(const void* cand_logits, kld_dtype dtype, int64_t n_rows, int64_t vocab,
+                                int64_t ld_cand, const kld_top_entry* ref_top, int32_t k,
+                                const float* ref_rows, const int32_t* target_ids, float* kl,
+                                int32_t* cand_argmax, uint8_t* top1, float* cand_target_lp,
+                                float* ref_target_lp, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, void* stream) {
+  return sparse_ref_impl(cand_logits, dtype, n_rows, vocab, ld_cand, ref_top, k, ref_rows, target_ids, kl,
+                         cand_argmax, top1, cand_target_lp, ref_target_lp, workspace, workspace_bytes,
+                         dev_status, stream, 0);
+}
+
+// kld_sparse_ref_score with the number of streaming warps forced (0 =
+// automatic), to test long pieces and many-piece merges.  Exported for
+// tests; not in kld.h.
+kld_status kld_sparse_ref_score_split(const void* cand_logits, kld_dtype dtype, int64_t n_rows, int64_t vocab,
+                                      int64_t ld_cand, const kld_top_entry* ref_top, int32_t k,
+                                      const float* ref_rows, const int32_t* target_ids, float* kl,
+                                      int32_t* cand_argmax, uint8_t* top1, float* cand_target_lp,
+                                      float* ref_target_lp, void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, void* stream, int32_t warps) {
+  return sparse_ref_impl(cand_logits, dtype, n_rows, vocab, ld_cand, ref_top, k, ref_rows, target_ids, kl,
+                         cand_argmax, top1, cand_target_lp, ref_target_lp, workspace, workspace_bytes,
+                         dev_status, stream, warps);
+}
+
 static kld_status shared_head_impl(const void* h_ref, const void* h_cand, const void* head_w, int64_t n_rows,
                                    int64_t hidden, int64_t vocab, const int32_t* target_ids, float* kl,
                                    int32_t* ref_argmax, int32_t* cand_argmax, float* ref_target_lp,

@@ -50,6 +50,26 @@ struct TopkTailArgs {
 };
 cudaError_t launch_topk_tail(const TopkTailArgs& a, cudaStream_t stream);
 
+struct SparseRefArgs {
+  const void* y;          // candidate logits [n_rows, ld]
+  bool bf16;
+  int64_t n_rows, vocab, ld;
+  const kld_top_entry* ref_top;  // [n_rows, k]
+  int k;
+  const float* ref_rows;  // [n_rows, 3] or null
+  const int32_t* targets;
+  float* kl;
+  int32_t* argmax;
+  uint8_t* top1;
+  float* lp_cand;
+  float* lp_ref;
+  void* workspace;        // >= sparse_ref_workspace_bytes(n_rows, k)
+  int32_t* dev_status;
+  int warps_override;     // 0: choose from the problem size
+};
+size_t sparse_ref_workspace_bytes(int64_t n_rows, int k);
+cudaError_t launch_sparse_ref(const SparseRefArgs& a, cudaStream_t stream);
+
 struct SharedHeadArgs {
   const void* h_ref;   // bf16 [n_rows, hidden]
   const void* h_cand;  // bf16 [n_rows, hidden]

@@ -13,8 +13,10 @@ in here"; "Qwopus3.8-27B-Coder-Flash: quality-eval reference", "Method");
 top-64 ids + fp16 log-probs sorted descending and f32 target log-probs over
 512 windows ("Qwopus...", "Files"); final hidden states of width 5120 and
 one bf16 LM head ("Qwen3.8-27B fidelity suite v5", "What is in here" and
-"What we preserve").  No corpus, model or capture is reproduced: the
-distributions below stand in for them.
+"What we preserve"); a sparse reference of the 512 most likely ids with f32
+log-probs, most likely first, and per row (NLL, entropy, tail mass)
+("Qwen3.8-27B Quantization Challenge", "Golden distributions").  No corpus,
+model or capture is reproduced: the distributions below stand in for them.
 
 Reference rows are Gumbel-perturbed Zipf(s = 1.1) log-weights over a
 per-row pseudo-random assignment of ranks to vocabulary ids, scaled by
@@ -32,6 +34,7 @@ ZIPF_S = 1.1
 SEED_BASE = 0x5EED0000
 TOPK = 64
 HIDDEN = 5120
+SPARSE_K = 512
 
 # rank -> vocabulary id bijection: id = (rank * RANK_MUL + offset) mod V.
 # 7919 is prime and does not divide 248,320 = 2^9 * 5 * 97.
@@ -253,3 +256,73 @@ def shared_head_states(seed: int = seed_for(5), device="cpu", n_rows: int = 8192
         W[a:b] = (w_std * torch.randn((b - a, hidden), generator=g, device=device)).to(torch.bfloat16)
     targets = torch.randint(0, vocab, (n_rows,), generator=g, device=device, dtype=torch.int32)
     return dict(h_ref=h_ref, h_cand=h_cand, W=W, targets=targets)
+
+
+def sparse_ref_window(seed: int = seed_for(6), device="cpu", n_rows: int = 2047, vocab: int = VOCAB,
+                      k: int = SPARSE_K, dtype=torch.bfloat16, sigma: float = 0.05,
+                      chunk: int = 256) -> dict:
+    """A sparse reference and a candidate's full logits for one window.
+
+    Reference, per row: a tail mass p_tail with log10 p_tail ~ U(-10, -3)
+    (median ~3e-7: the pages put the median below 1e-6 at 512 ids), and k
+    listed probabilities proportional to (j + 1)^-s e^{0.3 g_j} (g Gumbel,
+    s ~ U(1.5, 4) per row), sorted descending and summing to 1 - p_tail.
+    Listed ids are ranks 0 .. k-1 mapped through the row's id bijection, so
+    they are distinct; with k = vocab every id is listed and p_tail = 0.  ref_top is int32 [n, k, 2]: (id, f32 log-prob bits).
+    ref_rows is f32 [n, 3]: (NLL of the target, 0.0 in place of the entropy,
+    which the score does not read, p_tail).
+
+    Candidate full logits, per row: listed ids get log p_j + N(0, sigma^2),
+    the other ids log(p_tail c / (V - k)) + N(0, 1) with c = e^{N(0, 0.5^2)},
+    all shifted by U(-5, 5); 1% of rows swap the candidate values of the two
+    most likely listed ids.  Targets are drawn from the listed distribution
+    by Gumbel-max (an unlisted uniform id with probability p_tail)."""
+    g = _gen(seed, device)
+    n = n_rows
+    ref_top = torch.empty((n, k, 2), device=device, dtype=torch.int32)
+    ref_rows = torch.zeros((n, 3), device=device, dtype=torch.float32)
+    cand = torch.empty((n, vocab), device=device, dtype=dtype)
+    targets = torch.empty(n, device=device, dtype=torch.int32)
+    j = torch.arange(k, device=device, dtype=torch.float32)
+    for a in range(0, n, chunk):
+        b = min(n, a + chunk)
+        m = b - a
+        log_tail = math.log(10.0) * (-10.0 + 7.0 * torch.rand(m, generator=g, device=device, dtype=torch.float64))
+        if k >= vocab:          # every id listed: nothing is left for the tail
+            log_tail = torch.full_like(log_tail, -math.inf)
+        steep = 1.5 + 2.5 * torch.rand((m, 1), generator=g, device=device)
+        logw = -steep * torch.log1p(j)[None, :] + 0.3 * _gumbel((m, k), g, device)
+        logw = torch.sort(logw.double(), dim=1, descending=True).values
+        lp = logw - torch.logsumexp(logw, dim=1, keepdim=True) + torch.log1p(-torch.exp(log_tail))[:, None]
+        lp32 = lp.float()
+        off = torch.randint(0, vocab, (m,), generator=g, device=device, dtype=torch.int64)
+        ids = _ids_of_ranks(torch.arange(k, device=device)[None, :].expand(m, k), off, vocab)
+        ref_top[a:b, :, 0] = ids.to(torch.int32)
+        ref_top[a:b, :, 1] = lp32.view(torch.int32)
+        ref_rows[a:b, 2] = torch.exp(log_tail).float()
+
+        shift = -5.0 + 10.0 * torch.rand((m, 1), generator=g, device=device)
+        c_tail = log_tail + 0.5 * torch.randn(m, generator=g, device=device, dtype=torch.float64)
+        rest = (c_tail - math.log(max(vocab - k, 1))).float()[:, None]
+        y = rest + torch.randn((m, vocab), generator=g, device=device)
+        listed = lp32 + sigma * torch.randn((m, k), generator=g, device=device)
+        swap = torch.rand(m, generator=g, device=device) < 0.01
+        if k > 1 and bool(swap.any()):
+            top2 = listed[swap, :2].flip(1)
+            listed[swap, :2] = top2
+        y.scatter_(1, ids, listed)
+        cand[a:b] = (y + shift).to(dtype)
+
+        pick = torch.argmax(lp32 + _gumbel((m, k), g, device), dim=1)
+        t = torch.gather(ids, 1, pick[:, None]).squeeze(1)
+        nll = -torch.gather(lp32, 1, pick[:, None]).squeeze(1)
+        in_tail = torch.rand(m, generator=g, device=device, dtype=torch.float64) < torch.exp(log_tail)
+        if bool(in_tail.any()):
+            r = torch.randint(k, vocab, (m,), generator=g, device=device)
+            t = torch.where(in_tail, _ids_of_ranks(r[:, None], off, vocab).squeeze(1), t)
+            nll = torch.where(in_tail, (math.log(vocab - k) - log_tail).float(), nll)
+        targets[a:b] = t.to(torch.int32)
+        ref_rows[a:b, 0] = nll
+        del y, listed
+    return dict(cand=cand, ref_top=ref_top, ref_ids=ref_top[:, :, 0], ref_lp=ref_top[:, :, 1].view(torch.float32),
+                ref_rows=ref_rows, targets=targets, vocab=vocab)

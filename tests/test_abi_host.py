@@ -127,3 +127,36 @@ def test_reduce_validation(lib):
     assert rd(lib, wsb=16) == _lib.KLD_ERR_WORKSPACE
     assert rd(lib, ws=A16 + 128) == _lib.KLD_ERR_ALIGNMENT
     assert rd(lib, out=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
+
+
+def sr(lib, **kw):
+    a = dict(cand=A16, dtype=_lib.KLD_BF16, n=4, V=4096, ld=4096, top=A16 + 65536, k=512, rows=None, tgt=None,
+             kl=A16 + 131072, am=None, t1=None, lpc=None, lpr=None, ws=A16 + (1 << 19), wsb=None, st=None)
+    a.update(kw)
+    wsb = lib.kld_sparse_ref_workspace_size(max(a["n"], 0), max(a["k"], 1)) if a["wsb"] is None else a["wsb"]
+    return lib.kld_sparse_ref_score(a["cand"], a["dtype"], a["n"], a["V"], a["ld"], a["top"], a["k"], a["rows"],
+                                    a["tgt"], a["kl"], a["am"], a["t1"], a["lpc"], a["lpr"], a["ws"], wsb,
+                                    a["st"], None)
+
+
+def test_sparse_ref_validation(lib):
+    assert sr(lib, dtype=3) == _lib.KLD_ERR_UNSUPPORTED
+    assert sr(lib, k=0) == _lib.KLD_ERR_INVALID_ARG
+    assert sr(lib, k=_lib.KLD_SPARSE_MAX_K + 1) == _lib.KLD_ERR_INVALID_ARG
+    assert sr(lib, k=100, V=64, ld=64) == _lib.KLD_ERR_INVALID_ARG       # more listed ids than the vocabulary
+    assert sr(lib, V=(1 << 22) + 8, ld=(1 << 22) + 8) == _lib.KLD_ERR_UNSUPPORTED
+    assert sr(lib, ld=4000) == _lib.KLD_ERR_INVALID_ARG
+    assert sr(lib, n=-1) == _lib.KLD_ERR_INVALID_ARG
+    assert sr(lib, lpc=A16) == _lib.KLD_ERR_INVALID_ARG                  # target lp without targets
+    assert sr(lib, lpr=A16) == _lib.KLD_ERR_INVALID_ARG                  # reference lp without its rows
+    assert sr(lib, top=None) == _lib.KLD_ERR_INVALID_ARG
+    assert sr(lib, kl=None) == _lib.KLD_ERR_INVALID_ARG
+    assert sr(lib, ws=None) == _lib.KLD_ERR_WORKSPACE
+    assert sr(lib, wsb=1024) == _lib.KLD_ERR_WORKSPACE
+    assert sr(lib, cand=MIS) == _lib.KLD_ERR_ALIGNMENT
+    assert sr(lib, ld=4100) == _lib.KLD_ERR_ALIGNMENT                    # 8200-byte rows
+    assert sr(lib, top=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
+    assert sr(lib, ws=A16 + 64) == _lib.KLD_ERR_ALIGNMENT
+    assert sr(lib, n=0) == _lib.KLD_OK
+    assert lib.kld_sparse_ref_workspace_size(10, 512) > lib.kld_sparse_ref_workspace_size(10, 64)
+    assert lib.kld_sparse_ref_workspace_size(10, 0) == 0
