@@ -20,12 +20,13 @@
 // Pass 1 (persistent warps over the flattened (row, 16-byte vector) space,
 // as the full-vocabulary kernel): for each row piece a warp buckets the
 // listed ids that fall in the piece by streaming step (a counting sort in
-// shared memory, 256 steps at a time).  While streaming, the lane that holds
-// a listed id writes its logit to the workspace and masks it to -inf before
-// the step's maximum and weights are taken.  A repeated id is seen as a
-// second mask of the same slot and flags the row.  Pass 2 (one warp per
-// row) merges the pieces in index order, adds the ragged end of the row,
-// reads the listed logits and forms the outputs.
+// shared memory, 256 steps at a time); a repeated id shows up twice in one
+// bucket and flags the row.  A step that holds listed ids is staged through
+// shared memory, where up to 32 of its ids at once have their logits written
+// to the workspace and replaced by -inf, before the step's maximum and
+// weights are taken.  Pass 2 (one warp per row) merges the pieces in index
+// order, adds the ragged end of the row, reads the listed logits and forms
+// the outputs.
 #include <cuda_bf16.h>
 #include <cfloat>
 
@@ -38,13 +39,17 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarpsPerCta = kThreads / 32;
+constexpr int kMergeThreads = 128;           // one warp per row, four rows per CTA
+constexpr int kMergeWarps = kMergeThreads / 32;
 constexpr int kVecs = 4;                         // 16-byte vectors per lane per step
 constexpr int kStepVecs = 32 * kVecs;            // vectors per warp step
 constexpr int kMinVecsPerWarp = 4 * kStepVecs;
-constexpr int kMaxStreamWarps = 148 * 32;
+constexpr int kStreamCtasPerSm = 3;
+constexpr int kMaxStreamWarps = 148 * kStreamCtasPerSm * kWarpsPerCta;
 constexpr int kWin = 256;                        // steps per bucket window
 constexpr int kMaxK = KLD_SPARSE_MAX_K;
 constexpr int kFlagRepeat = 1;
+constexpr uint32_t kSkip = 0x80000000u;
 constexpr double kQFloor = 1e-12;
 
 // Tail state of one warp over one row piece (16 bytes).
@@ -85,42 +90,49 @@ struct MergeParams {
   int32_t* dev_status;
 };
 
+// Per-warp shared memory (6 KB): the bucketed list of a window, and either
+// the bucket counts (while the list is built) or one step's vectors (while
+// the listed elements of that step are captured and masked).
 struct WarpLists {
-  uint32_t entry[kMaxK];     // (step in window << 20) | (element in step << 10) | list slot
-  uint32_t count[kWin + 1];
+  // (step in window << 20) | (element in step << 10) | list slot, and
+  // kSkip on the later copies of a repeated id
+  uint32_t entry[kMaxK];
+  union {
+    uint32_t count[kWin + 1];
+    uint4 stage[kStepVecs];
+  };
 };
+static_assert(sizeof(uint32_t) * (kWin + 1) <= sizeof(uint4) * kStepVecs, "counts fit in the stage");
 
-// Element e of a 16-byte vector as f32, and the same slot set to -inf.
-template <bool kBF16>
-__device__ __forceinline__ float take_and_mask(uint4& v, int e) {
-  float out = 0.f;
-  if (kBF16) {
-    const int word = e >> 1, hi = e & 1;
+// Weights exp(y - mo) of a lane's step, added to r2.  With kMasked the
+// element slot `excl` (a new argmax) is weighed as -inf.
+template <bool kBF16, bool kMasked>
+__device__ __forceinline__ void accumulate(const uint4 (&v)[kVecs], float mo, int excl, float2& r2) {
+  using El = Elems<kBF16>;
+  constexpr int E = El::E;
+  const float2 nm = make_float2(-mo, -mo);
+  const float2 l2 = make_float2(kLog2e, kLog2e);
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      if (w != word) continue;
-      uint32_t& x = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
-      out = __uint_as_float(hi ? (x & 0xffff0000u) : (x << 16));
-      x = hi ? ((x & 0x0000ffffu) | 0xff800000u) : ((x & 0xffff0000u) | 0x0000ff80u);
-    }
-  } else {
+  for (int q = 0; q < kVecs; ++q) {
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      if (w != e) continue;
-      uint32_t& x = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
-      out = __uint_as_float(x);
-      x = 0xff800000u;
+    for (int k = 0; k < E / 2; ++k) {
+      float2 Y = El::pair(v[q], k);
+      if (kMasked) {
+        if (excl == q * E + 2 * k) Y.x = -CUDART_INF_F;
+        if (excl == q * E + 2 * k + 1) Y.y = -CUDART_INF_F;
+      }
+      const float2 t = __fmul2_rn(__fadd2_rn(Y, nm), l2);
+      r2 = __fadd2_rn(r2, make_float2(ex2(t.x), ex2(t.y)));
     }
   }
-  return out;
 }
 
 // Bucket the listed ids of elements [elo, ehi) by step (kStepVecs * E
-// elements each) for the window's steps; returns the number of entries.
-// Entries of one step are contiguous; their order inside a step is not fixed
-// and does not matter.
+// elements each) for the window's steps; returns the number of entries and
+// sets `repeat` when an id is listed twice.  Entries of one step are
+// contiguous; their order inside a step is not fixed and does not matter.
 __device__ int build_window(WarpLists& L, const int2* top, int K, int64_t elo, int64_t ehi, int step_elems,
-                            int lane) {
+                            int lane, bool& repeat) {
   for (int s = lane; s <= kWin; s += 32) L.count[s] = 0u;
   __syncwarp();
   for (int j = lane; j < K; j += 32) {
@@ -161,6 +173,23 @@ __device__ int build_window(WarpLists& L, const int2* top, int K, int64_t elo, i
     }
   }
   __syncwarp();
+  // a repeated id lands twice in one bucket: compare every entry with the
+  // later entries of its bucket (count[s] now holds the bucket's end) and
+  // mark the later copies, which then record -inf instead of the logit so
+  // the row's sums hold the id once
+  bool rep = false;
+  for (int i = lane; i < total; i += 32) {
+    const uint32_t key = (L.entry[i] >> 10) & 0x3ffffu;
+    const int end = (int)L.count[key >> 10];
+    for (int t = i + 1; t < end; ++t) {
+      if (((L.entry[t] >> 10) & 0x3ffffu) == key) {
+        rep = true;
+        atomicOr(&L.entry[t], kSkip);
+      }
+    }
+  }
+  repeat = __any_sync(0xffffffffu, rep);
+  __syncwarp();
   return total;
 }
 
@@ -189,10 +218,12 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
     const int64_t elo = (int64_t)(a + w0 * kStepVecs) * E;
     const int wend = min(nsteps, w0 + kWin);
     const int64_t ehi = (int64_t)min(b, a + wend * kStepVecs) * E;
-    const int cnt = build_window(L, top, p.K, elo, ehi, kStepElems, lane);
+    bool repeat;
+    const int cnt = build_window(L, top, p.K, elo, ehi, kStepElems, lane, repeat);
+    flags |= repeat ? kFlagRepeat : 0;
     int ptr = 0;
-    for (int st = w0; st < wend; ++st) {
-      uint4 v[kVecs];
+    // one step of loads stays in flight while the previous step is processed
+    auto load_step = [&](int st, uint4 (&v)[kVecs]) {
       const int64_t o = (int64_t)st * kStepVecs * 16;
       if ((st + 1) * kStepVecs <= n) {
 #pragma unroll
@@ -202,25 +233,47 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
         for (int q = 0; q < kVecs; ++q) v[q] = (st * kStepVecs + lane + 32 * q < n) ? ld_stream(yl + o + q * 32 * 16)
                                                                                    : neg_inf;
       }
-      // listed ids of this step: capture the logit, then mask it
-      uint32_t seen = 0u;
-      while (ptr < cnt) {
-        const uint32_t e = L.entry[ptr];
-        if ((int)(e >> 20) != st - w0) break;
-        const int off = (int)((e >> 10) & 1023u);
-        const int vec = off / E, el = off % E;
-        if (lane == (vec & 31)) {
-          const int slot = vec >> 5;
-          const uint32_t bit = 1u << (slot * E + el);
-          flags |= (seen & bit) ? kFlagRepeat : 0;
-          seen |= bit;
-          float val = 0.f;
+    };
+    uint4 nx[kVecs];
+    load_step(w0, nx);
+    for (int st = w0; st < wend; ++st) {
+      uint4 v[kVecs];
 #pragma unroll
-          for (int q = 0; q < kVecs; ++q)
-            if (q == slot) val = take_and_mask<kBF16>(v[q], el);
-          gy[e & 1023u] = val;
+      for (int q = 0; q < kVecs; ++q) v[q] = nx[q];
+      if (st + 1 < wend) load_step(st + 1, nx);
+      // listed ids of this step: stage the step's vectors so that element
+      // `off` of the step has a fixed shared-memory address (vector v of the
+      // step is lane v % 32's vector v / 32), capture and mask up to 32 ids
+      // at once, and reload
+      if (ptr < cnt && (int)((L.entry[ptr] >> 20) & 0xffu) == st - w0) {
+#pragma unroll
+        for (int q = 0; q < kVecs; ++q) L.stage[lane + 32 * q] = v[q];
+        __syncwarp();
+        for (;;) {
+          const int i = ptr + lane;
+          const uint32_t e = (i < cnt) ? L.entry[i] : 0xffffffffu;
+          const bool act = (i < cnt) && (int)((e >> 20) & 0xffu) == st - w0;
+          if (act && (e & kSkip)) {
+            gy[e & 1023u] = -CUDART_INF_F;
+          } else if (act) {
+            const int off = (int)((e >> 10) & 1023u);
+            if (kBF16) {
+              unsigned short* el = reinterpret_cast<unsigned short*>(L.stage) + off;
+              gy[e & 1023u] = __uint_as_float((uint32_t)*el << 16);
+              *el = (unsigned short)0xff80u;
+            } else {
+              uint32_t* el = reinterpret_cast<uint32_t*>(L.stage) + off;
+              gy[e & 1023u] = __uint_as_float(*el);
+              *el = 0xff800000u;
+            }
+          }
+          const int nact = __popc(__ballot_sync(0xffffffffu, act));
+          ptr += nact;
+          if (nact < 32) break;
         }
-        ++ptr;
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < kVecs; ++q) v[q] = L.stage[lane + 32 * q];
       }
       float c[kVecs];
       float cm = -CUDART_INF_F;
@@ -230,58 +283,44 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
         cm = fmaxf(cm, c[q]);
       }
       const float CM = warp_max(cm);
-      int excl = -1;
-      if (CM > s.m) {  // warp-uniform: a new maximum
-        s.r += r2.x + r2.y;
-        r2 = make_float2(0.f, 0.f);
-        const float sc = (s.a < 0) ? 0.f : ex2((s.m - CM) * kLog2e);
-        s.r = s.r * sc + ((lane == 0 && s.a >= 0) ? sc : 0.f);
-        int part = kVecs - 1, src = 0;
-#pragma unroll
-        for (int q = kVecs - 1; q >= 0; --q) {
-          const unsigned bq = __ballot_sync(0xffffffffu, c[q] == CM);
-          if (bq) {
-            part = q;
-            src = __ffs(bq) - 1;
-          }
-        }
-        int idx = 0;
-        if (lane == src) {
-          uint4 vv = v[0];
-#pragma unroll
-          for (int q = 1; q < kVecs; ++q)
-            if (q == part) vv = v[q];
-          int jj = E - 1;
-#pragma unroll
-          for (int k = E / 2 - 1; k >= 0; --k) {
-            const float2 pr = El::pair(vv, k);
-            if (pr.y == CM) jj = 2 * k + 1;
-            if (pr.x == CM) jj = 2 * k;
-          }
-          excl = part * E + jj;
-          idx = (a + st * kStepVecs + src + 32 * part) * E + jj;
-        }
-        s.a = __shfl_sync(0xffffffffu, idx, src);
-        s.m = CM;
+      if (!(CM > s.m)) {  // warp-uniform: the common step
+        accumulate<kBF16, false>(v, (s.a < 0) ? 0.f : s.m, -1, r2);
+        continue;
       }
-      // weights exp(y - m); a side with no finite value yet has only -inf
-      // (weight 0) or NaN (poisons r), so any finite offset serves
-      const float mo = (s.a < 0) ? 0.f : s.m;
-      const float2 nm = make_float2(-mo, -mo);
-      const float2 l2 = make_float2(kLog2e, kLog2e);
+      // a new maximum: fold the pair sums, rescale to the new maximum, hand
+      // the old maximum's own term to lane 0, find the first occurrence
+      s.r += r2.x + r2.y;
+      r2 = make_float2(0.f, 0.f);
+      const float sc = (s.a < 0) ? 0.f : ex2((s.m - CM) * kLog2e);
+      s.r = s.r * sc + ((lane == 0 && s.a >= 0) ? sc : 0.f);
+      int part = kVecs - 1, src = 0;
 #pragma unroll
-      for (int q = 0; q < kVecs; ++q) {
-#pragma unroll
-        for (int k = 0; k < E / 2; ++k) {
-          float2 Y = El::pair(v[q], k);
-          if (excl >= 0) {
-            if (excl == q * E + 2 * k) Y.x = -CUDART_INF_F;
-            if (excl == q * E + 2 * k + 1) Y.y = -CUDART_INF_F;
-          }
-          const float2 t = __fmul2_rn(__fadd2_rn(Y, nm), l2);
-          r2 = __fadd2_rn(r2, make_float2(ex2(t.x), ex2(t.y)));
+      for (int q = kVecs - 1; q >= 0; --q) {
+        const unsigned bq = __ballot_sync(0xffffffffu, c[q] == CM);
+        if (bq) {
+          part = q;
+          src = __ffs(bq) - 1;
         }
       }
+      int idx = 0, excl = -1;
+      if (lane == src) {
+        uint4 vv = v[0];
+#pragma unroll
+        for (int q = 1; q < kVecs; ++q)
+          if (q == part) vv = v[q];
+        int jj = E - 1;
+#pragma unroll
+        for (int k = E / 2 - 1; k >= 0; --k) {
+          const float2 pr = El::pair(vv, k);
+          if (pr.y == CM) jj = 2 * k + 1;
+          if (pr.x == CM) jj = 2 * k;
+        }
+        excl = part * E + jj;
+        idx = (a + st * kStepVecs + src + 32 * part) * E + jj;
+      }
+      s.a = __shfl_sync(0xffffffffu, idx, src);
+      s.m = CM;
+      accumulate<kBF16, true>(v, s.m, excl, r2);
     }
     __syncwarp();  // the lists are rebuilt for the next window
   }
@@ -293,7 +332,7 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
 }
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads) sparse_stream_kernel(const StreamParams p) {
+__global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) sparse_stream_kernel(const StreamParams p) {
   __shared__ WarpLists lists[kWarpsPerCta];
   const int lane = threadIdx.x & 31;
   const int wl = threadIdx.x >> 5;
@@ -343,20 +382,22 @@ __device__ __forceinline__ double warp_sum(double v) {
 
 // One warp per row.
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads) sparse_merge_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(kMergeThreads) sparse_merge_kernel(const MergeParams p) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
   constexpr int kElemBytes = kBF16 ? 2 : 4;
-  __shared__ float ys[kWarpsPerCta][kMaxK];
+  __shared__ float ys[kMergeWarps][kMaxK];   // listed logits
+  __shared__ float lps[kMergeWarps][kMaxK];  // listed reference log-probs
   wait_prior_grid();
   const int lane = threadIdx.x & 31;
   const int wl = threadIdx.x >> 5;
-  const int row = blockIdx.x * kWarpsPerCta + wl;
+  const int row = blockIdx.x * kMergeWarps + wl;
   if (row >= p.n_rows) return;
   const char* yrow = reinterpret_cast<const char*>(p.y) + (int64_t)row * p.ld * kElemBytes;
   const int2* top = p.top + (int64_t)row * p.K;
   const float* gy = p.gy + (int64_t)row * p.K;
   float* ysw = ys[wl];
+  float* lpw = lps[wl];
   const int64_t listed_end = (int64_t)p.nvec * E;  // ids below this were captured by the stream
 
   // tail state of the unlisted ids covered by the stream
@@ -377,14 +418,17 @@ __global__ void __launch_bounds__(kThreads) sparse_merge_kernel(const MergeParam
   bool bad = false;   // an id outside [0, V), or a repeated id
   bool nan = false;
   float lm = -CUDART_INF_F;
+#pragma unroll 4
   for (int j = lane; j < p.K; j += 32) {
-    const int id = top[j].x;
+    const int2 t = top[j];
+    const float g = gy[j];
     float y = -CUDART_INF_F;
-    if (id < 0 || id >= p.vocab) bad = true;
-    else y = (id < listed_end) ? gy[j] : El::load1(yrow, id);
+    if (t.x < 0 || t.x >= p.vocab) bad = true;
+    else y = (t.x < listed_end) ? g : El::load1(yrow, t.x);
     nan |= (y != y);
     lm = fmaxf(lm, y);
     ysw[j] = y;
+    lpw[j] = __int_as_float(t.y);
   }
   __syncwarp();
   bad = __any_sync(0xffffffffu, bad) || (acc.flags & kFlagRepeat);
@@ -420,8 +464,9 @@ __global__ void __launch_bounds__(kThreads) sparse_merge_kernel(const MergeParam
   const float m = have_tail ? fmaxf(acc.m, m_listed) : m_listed;
   int cand = INT32_MAX;
   for (int j = lane; j < p.K; j += 32) {
+    if (ysw[j] != m) continue;
     const int id = top[j].x;
-    if (ysw[j] == m && id >= 0 && id < cand) cand = id;
+    if (id >= 0 && id < cand) cand = id;
   }
   cand = __reduce_min_sync(0xffffffffu, cand);
   if (have_tail && acc.m == m && acc.a < cand) cand = acc.a;
@@ -430,6 +475,7 @@ __global__ void __launch_bounds__(kThreads) sparse_merge_kernel(const MergeParam
 
   // S = sum_R e^{y_j - m} + T, with T the tail mass relative to m
   double sw = 0.0;
+#pragma unroll 4
   for (int j = lane; j < p.K; j += 32) sw += exp((double)ysw[j] - (double)m);
   sw = warp_sum(sw);
   const double T = have_tail ? (1.0 + (double)acc.r) * exp((double)acc.m - (double)m) : 0.0;
@@ -437,8 +483,9 @@ __global__ void __launch_bounds__(kThreads) sparse_merge_kernel(const MergeParam
   const double logS = log(S);
 
   double kl = 0.0, psum = 0.0;
+#pragma unroll 4
   for (int j = lane; j < p.K; j += 32) {
-    const double lp = (double)__int_as_float(top[j].y);
+    const double lp = (double)lpw[j];
     const double pj = exp(lp);
     psum += pj;
     if (pj > 0.0) kl += pj * (lp - (((double)ysw[j] - (double)m) - logS));
@@ -509,9 +556,9 @@ cudaError_t launch_sparse_ref(const SparseRefArgs& a, cudaStream_t stream) {
   }
   MergeParams mp{a.y, a.ld, (int)a.vocab, nvec, (int)a.n_rows, nwarps, total, pieces, top, a.k, gy,
                  a.ref_rows, a.targets, a.kl, a.argmax, a.top1, a.lp_cand, a.lp_ref, a.dev_status};
-  const unsigned mgrid = (unsigned)((a.n_rows + kWarpsPerCta - 1) / kWarpsPerCta);
-  if (a.bf16) return launch_dependent(sparse_merge_kernel<true>, dim3(mgrid), dim3(kThreads), stream, mp);
-  return launch_dependent(sparse_merge_kernel<false>, dim3(mgrid), dim3(kThreads), stream, mp);
+  const unsigned mgrid = (unsigned)((a.n_rows + kMergeWarps - 1) / kMergeWarps);
+  if (a.bf16) return launch_dependent(sparse_merge_kernel<true>, dim3(mgrid), dim3(kMergeThreads), stream, mp);
+  return launch_dependent(sparse_merge_kernel<false>, dim3(mgrid), dim3(kMergeThreads), stream, mp);
 }
 
 }  // namespace kld
