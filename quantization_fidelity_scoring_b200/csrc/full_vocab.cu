@@ -228,12 +228,15 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
     accumulate<kBF16, true>(cur, sx.a < 0 ? 0.f : sx.m, sy.a < 0 ? 0.f : sy.m, ex_x, ex_y, rx2, ry2, a2);
   };
 
-  // full steps: the warp's four 16-byte loads per lane are issued together
-  // at the top of each step; other warps cover the latency
-  StepRaw A;
+  // full steps: the warp's four 16-byte loads per lane for step st + 1 are
+  // issued before step st is processed, so one step of loads is always in
+  // flight per warp; other warps cover the rest of the latency
+  StepRaw A, B;
   int st = 0;
+  if (nfull > 0) load_full(B, 0);
   for (; st < nfull; ++st) {
-    load_full(A, st);
+    A = B;
+    if (st + 1 < nfull) load_full(B, st + 1);  // next step's loads stay in flight
     step(A, st);
   }
   // ragged last step: lanes past b read -inf
@@ -260,7 +263,7 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
 }
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads) stream_kernel(const StreamParams p) {
+__global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) stream_kernel(const StreamParams p) {
   constexpr int kElemBytes = kBF16 ? 2 : 4;
   const int lane = threadIdx.x & 31;
   const int w = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);

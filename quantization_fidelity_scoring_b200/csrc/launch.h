@@ -25,8 +25,10 @@ struct FullVocabArgs {
   void* workspace;       // >= full_vocab_workspace_bytes(n_rows)
   int warps_override;    // 0: choose from the problem size
 };
-// Upper bound on the streaming warps (fixed, so results do not depend on the device).
-constexpr int kFullVocabMaxWarps = 148 * 32;
+// Upper bound on the streaming warps (fixed, so results do not depend on the
+// device): three CTAs of eight warps per SM on 148 SMs.
+constexpr int kStreamCtasPerSm = 3;
+constexpr int kFullVocabMaxWarps = 148 * kStreamCtasPerSm * 8;
 size_t full_vocab_workspace_bytes(int64_t n_rows);
 cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream);
 // Rows the library-owned scratch of kld_full_vocab_noalloc can hold.
