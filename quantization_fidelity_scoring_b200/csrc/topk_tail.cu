@@ -17,8 +17,8 @@
 // offset by 16 banks.  A repeated candidate id keeps its lowest slot
 // (atomicMin on the packed entry).  Results do not depend on the order of
 // insertion, so they are deterministic.  The three masses that feed 1 - sum
-// (candidate list, reference list, matched candidate cells) use the accurate
-// expf and are accumulated in f64, in fixed lane order; the KL terms are f32
+// (candidate list, reference list, matched candidate cells) are exp on the
+// MUFU unit accumulated in f64, in fixed lane order; the KL terms are f32
 // and the tail term takes one logarithm of the f64 ratio p_tail / q_tail.
 #include <cuda_fp16.h>
 #include <math_constants.h>
@@ -44,6 +44,10 @@ constexpr float kLn2 = 0.6931471805599453f;
 __device__ __forceinline__ uint32_t slot_of(uint32_t id) { return (id * 0x9E3779B1u) >> 24; }
 
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+
+// exp(lp) of a stored log-prob on the MUFU unit (relative error a few units
+// in the last place; the sums that use it are f64).
+__device__ __forceinline__ float mass(float lp) { return ex2(lp * kLog2e); }
 
 __device__ __forceinline__ float fast_log(float x) {
   float r;
@@ -179,8 +183,8 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
       for (int i = 0; i < kPer; ++i) {
         if (!valid[i]) continue;
         const float a = h2f(ra[i]);
-        const float pj = expf(a);
-        c_sum += (double)expf(h2f(cb[i]));
+        const float pj = mass(a);
+        c_sum += (double)mass(h2f(cb[i]));
         p_sum += (double)pj;
         const uint32_t id = (uint32_t)r[i];
         uint32_t s = slot_of(id);
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
         }
         if (e != kEmpty && entry_id(e) == id) {
           const float bm = h2f((uint16_t)(e & 0xffffu));
-          qm_sum += (double)expf(bm);
+          qm_sum += (double)mass(bm);
           klm += pj * (a - bm);
           ++matched;
         } else {
