@@ -379,6 +379,60 @@ def sparse_ref(Y, ref_ids, ref_lp, p_tail=None, targets=None) -> dict:
 
 
 # ---------------------------------------------------------------------------
+# sparse capture of a reference distribution
+# ---------------------------------------------------------------------------
+
+def sparse_capture_row(x, k: int, target=None) -> dict:
+    """The sparse record of one position, from the reference's full logits x.
+
+    "Qwen3.8-27B Quantization Challenge", "Golden distributions": per scored
+    position the reference keeps its k most likely tokens with their f32 log
+    p, most likely first, and a row of (NLL of the true next token, entropy
+    in nats, tail mass 1 - sum exp(top lp) summed over the rest of the full
+    row).  Equal log-probs keep the lower id first (a reading: the page does
+    not order ties).  A row holding NaN or +inf, or no finite logit, gives ids
+    -1 and NaN everywhere else.
+    """
+    x = as_f64(x)
+    V = x.shape[0]
+    if not 0 < k <= V:
+        raise ValueError("need 0 < k <= V")
+    out = dict(ids=np.full(k, -1, dtype=np.int64), lp=np.full(k, np.nan), nll=math.nan,
+               entropy=math.nan, tail=math.nan)
+    if not _row_is_valid(x):
+        return out
+    lp = log_softmax(x)
+    order = np.lexsort((np.arange(V), -lp))        # by log-prob descending, then id ascending
+    top = order[:k]
+    p = np.exp(lp)
+    live = p > 0.0                                  # 0 * log 0 = 0
+    rest = np.ones(V, dtype=bool)
+    rest[top] = False
+    out["ids"] = top.astype(np.int64)
+    out["lp"] = lp[top]
+    out["entropy"] = -math.fsum((p[live] * lp[live]).tolist())
+    out["tail"] = math.fsum(p[rest].tolist())
+    if target is not None and 0 <= int(target) < V:
+        out["nll"] = -float(lp[int(target)])
+    return out
+
+
+def sparse_capture(X, k: int, targets=None) -> dict:
+    """sparse_capture_row for every row of X [n, V] (float64-exact): ids and
+    lp [n, k], rows [n, 3] = (NLL, entropy, tail)."""
+    X = np.asarray(X)
+    n = X.shape[0]
+    ids = np.empty((n, k), dtype=np.int64)
+    lp = np.empty((n, k))
+    rows = np.empty((n, 3))
+    for i in range(n):
+        r = sparse_capture_row(X[i], k, None if targets is None else int(targets[i]))
+        ids[i], lp[i] = r["ids"], r["lp"]
+        rows[i] = (r["nll"], r["entropy"], r["tail"])
+    return dict(ids=ids, lp=lp, rows=rows)
+
+
+# ---------------------------------------------------------------------------
 # reductions
 # ---------------------------------------------------------------------------
 

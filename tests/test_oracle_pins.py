@@ -376,6 +376,69 @@ def pin_sparse_edge_cases(O):
 
 
 # ---------------------------------------------------------------------------
+# sparse capture of a reference distribution
+# ---------------------------------------------------------------------------
+
+def pin_capture_uniform_and_peak(O):
+    # uniform row: ties keep the lowest ids, every lp = -ln V, entropy ln V,
+    # tail (V - k) / V, NLL ln V
+    for V, k in ((10, 3), (64, 64), (1000, 17)):
+        r = O.sparse_capture_row(np.full(V, 2.5), k, target=V - 1)
+        assert list(r["ids"]) == list(range(k))
+        assert np.allclose(r["lp"], -math.log(V), rtol=0, atol=1e-14)
+        assert _close(r["entropy"], math.log(V)) and _close(r["nll"], math.log(V))
+        assert _close(r["tail"], (V - k) / V, atol=1e-15)
+    # one raised logit: p0 = e^c / (e^c + V - 1)
+    V, c = 50, 3.0
+    x = np.zeros(V)
+    x[7] = c
+    p0 = math.exp(c) / (math.exp(c) + V - 1)
+    q = 1.0 / (math.exp(c) + V - 1)
+    r = O.sparse_capture_row(x, 2, target=7)
+    assert list(r["ids"]) == [7, 0]
+    assert _close(r["lp"][0], math.log(p0)) and _close(r["lp"][1], math.log(q))
+    assert _close(r["entropy"], -(p0 * math.log(p0) + (V - 1) * q * math.log(q)))
+    assert _close(r["tail"], (V - 2) * q) and _close(r["nll"], -math.log(p0))
+
+
+def pin_capture_brute_force(O):
+    import scipy.stats
+    rng = np.random.default_rng(31)
+    for _ in range(200):
+        V = int(rng.integers(2, 40))
+        k = int(rng.integers(1, V + 1))
+        x = np.round(rng.normal(0, 2, V), 1)          # rounding makes ties common
+        p = _softmax_loop(list(x))
+        want = sorted(range(V), key=lambda i: (-p[i], i))[:k]
+        t = int(rng.integers(0, V))
+        r = O.sparse_capture_row(x, k, target=t)
+        # ids equal where the probabilities differ; equal logits give exactly equal lp
+        assert [x[i] for i in r["ids"]] == [x[i] for i in want]
+        assert sorted(r["ids"][np.array([x[i] for i in r["ids"]]) == x[want[-1]]]) == list(r["ids"][
+            np.array([x[i] for i in r["ids"]]) == x[want[-1]]])
+        assert np.allclose(np.exp(r["lp"]), [p[i] for i in r["ids"]], rtol=1e-12, atol=0)
+        assert _close(r["entropy"], float(scipy.stats.entropy(p)), rtol=1e-10, atol=1e-14)
+        assert _close(r["tail"], sum(p[i] for i in range(V) if i not in set(r["ids"])), rtol=1e-10, atol=1e-15)
+        assert _close(r["nll"], -math.log(p[t]))
+
+
+def pin_capture_round_trip(O):
+    # a candidate identical to the captured reference scores 0 against it,
+    # and the listed masses plus the tail make 1
+    rng = np.random.default_rng(32)
+    for _ in range(20):
+        V, k = int(rng.integers(20, 300)), int(rng.integers(1, 20))
+        x = rng.normal(0, 3, V)
+        r = O.sparse_capture_row(x, k)
+        assert abs(O.sparse_ref_row(x, r["ids"], r["lp"], r["tail"])["kl"]) < 1e-13
+        assert _close(math.fsum(np.exp(r["lp"]).tolist()) + r["tail"], 1.0, atol=1e-14)
+    bad = O.sparse_capture_row(np.array([0.0, np.nan, 1.0]), 2, target=0)
+    assert list(bad["ids"]) == [-1, -1] and math.isnan(bad["tail"]) and math.isnan(bad["nll"])
+    ninf = O.sparse_capture_row(np.array([0.0, -np.inf, 1.0]), 3, target=1)
+    assert list(ninf["ids"]) == [2, 0, 1] and ninf["nll"] == math.inf and ninf["tail"] == 0.0
+
+
+# ---------------------------------------------------------------------------
 # reductions
 # ---------------------------------------------------------------------------
 
@@ -515,6 +578,13 @@ MUTANTS = [
      "pt = (1.0 - float(np.sum(np.exp(lq_all[ids]))))"),
     ("reference top-1 from the last listed id", "out[\"top1\"] = int(int(ids[0]) == out[\"cand_argmax\"])",
      "out[\"top1\"] = int(int(ids[-1]) == out[\"cand_argmax\"])"),
+    ("capture tail from the listed ids", "out[\"tail\"] = math.fsum(p[rest].tolist())",
+     "out[\"tail\"] = math.fsum(p[top].tolist())"),
+    ("capture entropy sign", "out[\"entropy\"] = -math.fsum((p[live] * lp[live]).tolist())",
+     "out[\"entropy\"] = math.fsum((p[live] * lp[live]).tolist())"),
+    ("capture ties keep the higher id", "order = np.lexsort((np.arange(V), -lp))",
+     "order = np.lexsort((-np.arange(V), -lp))"),
+    ("capture NLL sign", "out[\"nll\"] = -float(lp[int(target)])", "out[\"nll\"] = float(lp[int(target)])"),
     ("transposed head", "return np.asarray(H, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T",
      "return (np.asarray(W, dtype=np.float64) @ np.asarray(H, dtype=np.float64).T).T[:, ::-1]"),
 ]
