@@ -255,6 +255,41 @@ kld_status kld_sparse_ref_score(const void* cand_logits, kld_dtype dtype, int64_
                                 int32_t* dev_status, void* stream);
 
 /*
+ * kld_sparse_capture - the sparse record of a reference distribution, from
+ * its full logits: the producer of kld_sparse_ref_score's reference.
+ *
+ * Defines ("Qwen3.8-27B Quantization Challenge", "Golden distributions"): per
+ * row, with lp = log-softmax of the logits over all vocab ids and p = exp(lp),
+ *    top[j], j < k   the k ids of largest lp with their lp (f32), most
+ *                    likely first; equal lp keep the lower id first
+ *    rows[0]         -lp[target], the NLL of the true next token
+ *    rows[1]         -sum_i p_i lp_i, the entropy in nats
+ *    rows[2]         sum of p_i over the ids not in top, summed over those
+ *                    ids (never formed as 1 - sum of the listed masses)
+ *
+ * Arguments:
+ *   logits       DEVICE [n_rows, ld] f32 or bf16, 16-byte aligned; ld * element
+ *                size a multiple of 16.
+ *   k            1 .. KLD_SPARSE_MAX_K and k <= vocab; vocab <= 2^22.
+ *   target_ids   DEVICE int32 [n_rows], or NULL (rows[0] is then NaN).
+ *   top          DEVICE kld_top_entry [n_rows, k], 8-byte aligned (output).
+ *   rows         DEVICE f32 [n_rows, 3], 4-byte aligned (output).
+ *   workspace    DEVICE, >= kld_sparse_capture_workspace_size(n_rows, k)
+ *                bytes, 256-byte aligned; holds nothing between calls.
+ * A row holding NaN or +inf, or no finite logit, gives ids -1 and NaN lp and
+ * rows.  A target outside [0, vocab) gives NaN NLL and sets
+ * KLD_DEV_BAD_TARGET.  Up to KLD_CAPTURE_CANDIDATES ids per row are kept as
+ * candidates in one streaming pass; a row that needs more (many equal
+ * logits, or its largest logits missed by the threshold sample) is redone
+ * exactly from its logits, which is slower but gives the same result.
+ */
+#define KLD_CAPTURE_CANDIDATES 8192
+size_t kld_sparse_capture_workspace_size(int64_t n_rows, int32_t k);
+kld_status kld_sparse_capture(const void* logits, kld_dtype dtype, int64_t n_rows, int64_t vocab, int64_t ld,
+                              int32_t k, const int32_t* target_ids, kld_top_entry* top, float* rows,
+                              void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * kld_from_hidden_shared_head - full-vocabulary scoring from final hidden
  * states pushed through one shared LM head.
  *

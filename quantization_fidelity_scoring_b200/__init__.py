@@ -6,10 +6,12 @@ of include/kld.h); this package is its Python binding.
 from . import _lib
 from .api import (KldError, kld_from_hidden_shared_head, kld_full_vocab, kld_full_vocab_workspace_size,
                   kld_reduce_stats, kld_reduce_workspace_size, kld_shared_head_workspace_size,
-                  kld_sparse_ref_score, kld_sparse_ref_workspace_size, kld_topk_tail, stats_to_dict)
+                  kld_sparse_capture, kld_sparse_capture_workspace_size, kld_sparse_ref_score,
+                  kld_sparse_ref_workspace_size, kld_topk_tail, stats_to_dict)
 
 __all__ = ["KldError", "kld_from_hidden_shared_head", "kld_shared_head_workspace_size", "kld_full_vocab", "kld_full_vocab_workspace_size", "kld_topk_tail", "kld_reduce_stats",
-           "kld_sparse_ref_score", "kld_sparse_ref_workspace_size",
+           "kld_sparse_ref_score", "kld_sparse_ref_workspace_size", "kld_sparse_capture",
+           "kld_sparse_capture_workspace_size",
            "kld_reduce_workspace_size", "stats_to_dict", "load_library"]
 
 

@@ -55,6 +55,7 @@ class KldStats(ctypes.Structure):
 assert ctypes.sizeof(KldStats) == 280
 
 KLD_SPARSE_MAX_K = 1024
+KLD_CAPTURE_CANDIDATES = 8192
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -74,6 +75,8 @@ PROTOTYPES = {
     "kld_sparse_ref_workspace_size": (_SZ, [_I64, _I32]),
     "kld_sparse_ref_score": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _I32, _P, _P, _P, _P, _P,
                                             _P, _P, _P, _SZ, _P, _P]),
+    "kld_sparse_capture_workspace_size": (_SZ, [_I64, _I32]),
+    "kld_sparse_capture": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _SZ, _P, _P]),
     "kld_shared_head_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "kld_from_hidden_shared_head": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                                    _SZ, _P, _P]),
@@ -84,6 +87,8 @@ PROTOTYPES = {
 
 # exported for tests only (not part of the public header)
 TEST_PROTOTYPES = {
+    "kld_sparse_capture_exact": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _SZ,
+                                                _P, _P]),
     "kld_sparse_ref_score_split": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _I32, _P, _P, _P, _P,
                                                   _P, _P, _P, _P, _SZ, _P, _P, _I32]),
     "kld_from_hidden_shared_head_withhold": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P, _P]),

@@ -170,6 +170,38 @@ def kld_sparse_ref_workspace_size(n_rows: int, k: int) -> int:
     return int(_lib.load().kld_sparse_ref_workspace_size(n_rows, k))
 
 
+def kld_sparse_capture(logits: torch.Tensor, k: int, targets=None, *, top=None, rows=None, workspace=None,
+                       dev_status=None, stream=None, exact: bool = False) -> dict:
+    """Sparse record of reference logit rows [n, V] (f32 or bf16, unit
+    stride along V): top int32 [n, k, 2] of (id, f32 log-prob bits), most
+    likely first, and rows f32 [n, 3] of (NLL, entropy, tail mass).  Outputs
+    and the workspace are allocated when not given.  `exact` sends every row
+    down the exact path (tests)."""
+    _need_cuda("logits", logits, ndim=2)
+    if logits.dtype not in _DTYPES:
+        raise ValueError("logits must be float32 or bfloat16")
+    if logits.stride(1) != 1:
+        raise ValueError("logit rows must be contiguous along the vocabulary")
+    n, V = logits.shape
+    dev = logits.device
+    if targets is not None:
+        _need_cuda("targets", targets, torch.int32, 1)
+    top = torch.empty((n, k, 2), dtype=torch.int32, device=dev) if top is None else top
+    rows = torch.empty((n, 3), dtype=torch.float32, device=dev) if rows is None else rows
+    lib = _lib.load()
+    if workspace is None:
+        workspace = torch.empty(max(lib.kld_sparse_capture_workspace_size(n, k), 1), dtype=torch.uint8, device=dev)
+    fn = lib.kld_sparse_capture_exact if exact else lib.kld_sparse_capture
+    st = fn(_ptr(logits), _DTYPES[logits.dtype], n, V, logits.stride(0), k, _ptr(targets), _ptr(top), _ptr(rows),
+            _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream_handle(stream))
+    _check(st, "kld_sparse_capture")
+    return dict(top=top, ids=top[:, :, 0], lp=top[:, :, 1].view(torch.float32), rows=rows)
+
+
+def kld_sparse_capture_workspace_size(n_rows: int, k: int) -> int:
+    return int(_lib.load().kld_sparse_capture_workspace_size(n_rows, k))
+
+
 def kld_from_hidden_shared_head(h_ref, h_cand, head_w, targets=None, *, argmax: bool = True, kl=None,
                                 ref_argmax=None, cand_argmax=None, ref_target_lp=None, cand_target_lp=None,
                                 workspace=None, dev_status=None, stream=None) -> dict:

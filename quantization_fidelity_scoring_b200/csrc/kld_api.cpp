@@ -223,6 +223,60 @@ kld_status kld_sparse_ref_score_split(const void* cand_logits, kld_dtype dtype, 
                          dev_status, stream, warps);
 }
 
+size_t kld_sparse_capture_workspace_size(int64_t n_rows, int32_t k) {
+  if (n_rows < 0 || k < 1 || k > KLD_SPARSE_MAX_K) return 0;
+  return kld::sparse_capture_workspace_bytes(n_rows);
+}
+
+static kld_status sparse_capture_impl(const void* logits, kld_dtype dtype, int64_t n_rows, int64_t vocab,
+                                      int64_t ld, int32_t k, const int32_t* target_ids, kld_top_entry* top,
+                                      float* rows, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                      void* stream, int force_exact) {
+  if (dtype != KLD_F32 && dtype != KLD_BF16) return KLD_ERR_UNSUPPORTED;
+  if (n_rows < 0 || vocab < 1 || ld < vocab || k < 1 || k > KLD_SPARSE_MAX_K || k > vocab)
+    return KLD_ERR_INVALID_ARG;
+  if (vocab > (int64_t(1) << 22)) return KLD_ERR_UNSUPPORTED;
+  if (n_rows == 0) return KLD_OK;
+  if (!logits || !top || !rows) return KLD_ERR_INVALID_ARG;
+  if (n_rows > (int64_t)INT32_MAX - kld::kFullVocabMaxWarps) return KLD_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < kld::sparse_capture_workspace_bytes(n_rows)) return KLD_ERR_WORKSPACE;
+  const int64_t esize = dtype == KLD_BF16 ? 2 : 4;
+  if (!aligned(workspace, 256) || !aligned(logits, 16) || (ld * esize) % 16 != 0) return KLD_ERR_ALIGNMENT;
+  if (!aligned(top, 8) || !aligned(rows, 4) || !aligned(target_ids, 4) || !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+  kld::SparseCaptureArgs a;
+  a.x = logits;
+  a.bf16 = dtype == KLD_BF16;
+  a.n_rows = n_rows;
+  a.vocab = vocab;
+  a.ld = ld;
+  a.k = k;
+  a.targets = target_ids;
+  a.top = top;
+  a.rows = rows;
+  a.workspace = workspace;
+  a.dev_status = dev_status;
+  a.force_exact = force_exact;
+  return cuda_status(kld::launch_sparse_capture(a, static_cast<cudaStream_t>(stream)));
+}
+
+kld_status kld_sparse_capture(const void* logits, kld_dtype dtype, int64_t n_rows, int64_t vocab, int64_t ld,
+                              int32_t k, const int32_t* target_ids, kld_top_entry* top, float* rows,
+                              void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return sparse_capture_impl(logits, dtype, n_rows, vocab, ld, k, target_ids, top, rows, workspace,
+                             workspace_bytes, dev_status, stream, 0);
+}
+
+// kld_sparse_capture with every row on the exact path (the one a row takes
+// when its candidates do not fit or fall short).  Exported for tests; not in
+// kld.h.
+kld_status kld_sparse_capture_exact(const void* logits, kld_dtype dtype, int64_t n_rows, int64_t vocab, int64_t ld,
+                                    int32_t k, const int32_t* target_ids, kld_top_entry* top, float* rows,
+                                    void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  return sparse_capture_impl(logits, dtype, n_rows, vocab, ld, k, target_ids, top, rows, workspace,
+                             workspace_bytes, dev_status, stream, 1);
+}
+
 static kld_status shared_head_impl(const void* h_ref, const void* h_cand, const void* head_w, int64_t n_rows,
                                    int64_t hidden, int64_t vocab, const int32_t* target_ids, float* kl,
                                    int32_t* ref_argmax, int32_t* cand_argmax, float* ref_target_lp,

@@ -72,6 +72,21 @@ struct SparseRefArgs {
 size_t sparse_ref_workspace_bytes(int64_t n_rows, int k);
 cudaError_t launch_sparse_ref(const SparseRefArgs& a, cudaStream_t stream);
 
+struct SparseCaptureArgs {
+  const void* x;           // reference logits [n_rows, ld]
+  bool bf16;
+  int64_t n_rows, vocab, ld;
+  int k;
+  const int32_t* targets;  // or null
+  kld_top_entry* top;      // [n_rows, k]
+  float* rows;             // [n_rows, 3]
+  void* workspace;         // >= sparse_capture_workspace_bytes(n_rows)
+  int32_t* dev_status;
+  int force_exact;         // tests only: every row takes the exact path
+};
+size_t sparse_capture_workspace_bytes(int64_t n_rows);
+cudaError_t launch_sparse_capture(const SparseCaptureArgs& a, cudaStream_t stream);
+
 struct SharedHeadArgs {
   const void* h_ref;   // bf16 [n_rows, hidden]
   const void* h_cand;  // bf16 [n_rows, hidden]

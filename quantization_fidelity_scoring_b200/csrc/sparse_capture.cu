@@ -1,0 +1,691 @@
+// Sparse capture of a reference distribution from its full logits.
+//
+// "Qwen3.8-27B Quantization Challenge", "Golden distributions": per scored
+// position the reference keeps its K most likely tokens with f32 log p, most
+// likely first, and a row (NLL of the true next token, entropy in nats, tail
+// mass summed over the rest of the full row).  Equal log-probs keep the lower
+// id first.
+//
+// Three kernels:
+//  1. sample (one warp per row): 1024 evenly spaced elements of the row; the
+//     threshold tau is their 10th largest, so about 10 / 1024 of the row is
+//     at or above it (~2,400 ids at V = 248,320) while the row's top 512 are
+//     all above it unless the sample holds 10 of them (about 3e-5 for a
+//     random layout).  tau = -inf when the whole row fits the candidate
+//     buffer.
+//  2. stream (persistent warps over the flattened (row, 16-byte vector)
+//     space): elements >= tau are appended, as (value, id), to the row's
+//     candidate buffer; every other element feeds the row's tail mass
+//     T = sum e^{x - m} and entropy term B = sum e^{x - m} (x - m) with a
+//     warp-uniform running maximum m over all elements.  Neither sum ever
+//     holds a candidate, so the tail never comes from 1 - sum of the listed
+//     masses (which cancels when they hold all but ~1e-6 of the mass).
+//  3. finalize (one CTA per row): exact selection of the K largest among
+//     the candidates (bitwise radix select on the value bits, then on the ids
+//     of the values tied at the boundary), a bitonic sort of the K, and the
+//     outputs.  The listed terms are summed in sorted order and the unlisted
+//     candidates in fixed point scaled to the K-th weight, so every sum is
+//     exact up to rounding and independent of the order candidates arrived
+//     in.  A row whose candidates at or above tau are fewer than K, or
+//     overflow the buffer, is redone exactly from the full row by the same
+//     CTA (every element a candidate).
+#include <cuda_bf16.h>
+#include <cfloat>
+
+#include "kld_common.cuh"
+#include "launch.h"
+#include "stream_common.cuh"
+
+namespace kld {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarpsPerCta = kThreads / 32;
+constexpr int kVecs = 4;                      // 16-byte vectors per lane per step
+constexpr int kStepVecs = 32 * kVecs;
+constexpr int kMinVecsPerWarp = 4 * kStepVecs;
+constexpr int kStreamCtasPerSm = 3;
+constexpr int kMaxStreamWarps = 148 * kStreamCtasPerSm * kWarpsPerCta;
+constexpr int kSampleElems = 1024;
+constexpr int kSampleRank = 10;
+constexpr int kCap = KLD_CAPTURE_CANDIDATES;  // candidates kept per row
+constexpr int kFinThreads = 256;
+constexpr int kMaxK = KLD_SPARSE_MAX_K;
+
+// Tail state of one warp over one row piece (16 bytes): running maximum m
+// over all elements, and over the non-candidates T = sum e^{x-m},
+// B = sum e^{x-m} (x - m).
+struct CapPiece {
+  float m, T, B;
+  int pad;
+};
+
+struct CapParams {
+  const void* x;
+  int64_t ld;          // elements
+  int vocab, nvec, n_rows, nwarps;
+  int64_t total;       // n_rows * nvec
+  int K;
+  const int32_t* targets;
+  float* tau;          // [n_rows]
+  int* count;          // [n_rows] candidates appended (may exceed kCap)
+  int2* cand;          // [n_rows][kCap] (f32 value bits, id)
+  CapPiece* pieces;    // slot row + warp
+  kld_top_entry* top;  // [n_rows, K]
+  float* rows;         // [n_rows, 3] NLL, entropy, tail
+  int32_t* dev_status;
+  int force_exact;     // tests only: every row takes the exact path
+};
+
+// 1. one warp per row: tau = the kSampleRank-th largest of kSampleElems
+// evenly spaced elements (counted with multiplicity); also clears the row's
+// candidate count.
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads) cap_sample_kernel(const CapParams p) {
+  using El = Elems<kBF16>;
+  constexpr int E = El::E;
+  constexpr int kSampleVecs = kSampleElems / E;       // 128 (bf16) or 256 (f32)
+  constexpr int kPerLane = kSampleVecs / 32;
+  constexpr int kElemBytes = kBF16 ? 2 : 4;
+  wait_prior_grid();
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (row >= p.n_rows) return;
+  if (lane == 0) p.count[row] = 0;
+  if ((int64_t)p.nvec * E <= kCap || p.nvec < kSampleVecs) {
+    if (lane == 0) p.tau[row] = -CUDART_INF_F;  // every element fits the buffer
+    return;
+  }
+  const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld * kElemBytes;
+  float v[kPerLane * E];
+#pragma unroll
+  for (int q = 0; q < kPerLane; ++q) {
+    const int s = lane + 32 * q;
+    const int64_t vec = ((int64_t)s * p.nvec) / kSampleVecs;
+    const uint4 w = *reinterpret_cast<const uint4*>(xrow + vec * 16);
+#pragma unroll
+    for (int k = 0; k < E / 2; ++k) {
+      const float2 pr = El::pair(w, k);
+      v[q * E + 2 * k] = pr.x;
+      v[q * E + 2 * k + 1] = pr.y;
+    }
+  }
+  // peel off the largest values until kSampleRank of them are counted
+  int need = kSampleRank;
+  float thr = -CUDART_INF_F;
+  for (int round = 0; round < kSampleRank; ++round) {
+    float lm = -CUDART_INF_F;
+#pragma unroll
+    for (int i = 0; i < kPerLane * E; ++i) lm = fmaxf(lm, v[i]);
+    const float M = warp_max(lm);
+    thr = M;
+    if (!(M > -CUDART_INF_F)) break;  // only -inf (or NaN) left
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kPerLane * E; ++i) {
+      const bool hit = v[i] == M;
+      c += hit ? 1 : 0;
+      v[i] = hit ? -CUDART_INF_F : v[i];
+    }
+    need -= __reduce_add_sync(0xffffffffu, c);
+    if (need <= 0) break;
+  }
+  if (lane == 0) p.tau[row] = thr;
+}
+
+// 2. stream vectors [a, b) of one row; returns the piece's tail state
+// (identical in every lane) and appends the piece's candidates.
+template <bool kBF16>
+__device__ CapPiece cap_piece(const CapParams& p, int row, int a, int b, int lane, float tau) {
+  using El = Elems<kBF16>;
+  constexpr int E = El::E;
+  constexpr int kElemBytes = kBF16 ? 2 : 4;
+  constexpr uint32_t kNegInfWord = kBF16 ? 0xff80ff80u : 0xff800000u;
+  const uint4 neg_inf = make_uint4(kNegInfWord, kNegInfWord, kNegInfWord, kNegInfWord);
+  const char* yl = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld * kElemBytes + (int64_t)(a + lane) * 16;
+  int2* cand = p.cand + (int64_t)row * kCap;
+
+  float m = -CUDART_INF_F;  // warp-uniform
+  float2 T2 = make_float2(0.f, 0.f), B2 = T2;
+  const int n = b - a;
+  const int nsteps = (n + kStepVecs - 1) / kStepVecs;
+  auto load_step = [&](int st, uint4 (&v)[kVecs]) {
+    const int64_t o = (int64_t)st * kStepVecs * 16;
+    if ((st + 1) * kStepVecs <= n) {
+#pragma unroll
+      for (int q = 0; q < kVecs; ++q) v[q] = ld_stream(yl + o + q * 32 * 16);
+    } else {
+#pragma unroll
+      for (int q = 0; q < kVecs; ++q)
+        v[q] = (st * kStepVecs + lane + 32 * q < n) ? ld_stream(yl + o + q * 32 * 16) : neg_inf;
+    }
+  };
+  uint4 nx[kVecs];
+  if (nsteps > 0) load_step(0, nx);
+  for (int st = 0; st < nsteps; ++st) {
+    uint4 v[kVecs];
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q) v[q] = nx[q];
+    if (st + 1 < nsteps) load_step(st + 1, nx);
+
+    float c[kVecs];
+    float cm = -CUDART_INF_F;
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q) {
+      c[q] = El::vmax(v[q]);
+      cm = fmaxf(cm, c[q]);
+    }
+    const float CM = warp_max(cm);
+    if (CM > m) {  // warp-uniform: a new maximum; rescale both sums to it
+      float T = T2.x + T2.y, B = B2.x + B2.y;
+      if (m != -CUDART_INF_F) {  // else nothing finite yet: the sums hold 0, or NaN, and stay
+        const float sc = ex2((m - CM) * kLog2e);
+        B = sc * (B + (m - CM) * T);
+        T = sc * T;
+      }
+      T2 = make_float2(T, 0.f);
+      B2 = make_float2(B, 0.f);
+      m = CM;
+    }
+
+    // candidates: the lanes whose vectors reach tau append their elements
+    // that do, at positions reserved by one atomic per warp
+    unsigned hitq = 0u;
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q) hitq |= (c[q] >= tau) ? (1u << q) : 0u;
+    if (__any_sync(0xffffffffu, hitq != 0u)) {
+      uint32_t emask = 0u;
+#pragma unroll
+      for (int q = 0; q < kVecs; ++q) {
+        if (!((hitq >> q) & 1u)) continue;
+#pragma unroll
+        for (int k = 0; k < E / 2; ++k) {
+          const float2 pr = El::pair(v[q], k);
+          emask |= (pr.x >= tau) ? (1u << (q * E + 2 * k)) : 0u;
+          emask |= (pr.y >= tau) ? (1u << (q * E + 2 * k + 1)) : 0u;
+        }
+      }
+      const int nc = __popc(emask);
+      int incl = nc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const int tot = __shfl_sync(0xffffffffu, incl, 31);
+      int base = 0;
+      if (lane == 0) base = atomicAdd(p.count + row, tot);
+      int pos = __shfl_sync(0xffffffffu, base, 0) + incl - nc;
+      while (emask) {
+        const int bit = __ffs(emask) - 1;
+        emask &= emask - 1u;
+        const int q = bit / E, e = bit % E;
+        uint4 vv = v[0];
+#pragma unroll
+        for (int qq = 1; qq < kVecs; ++qq)
+          if (qq == q) vv = v[qq];
+        const float2 pr = El::pair(vv, e >> 1);
+        const float val = (e & 1) ? pr.y : pr.x;
+        if (pos < kCap)
+          cand[pos] = make_int2(__float_as_int(val), (a + st * kStepVecs + lane + 32 * q) * E + e);
+        ++pos;
+      }
+    }
+
+    // tail and entropy sums over the non-candidates; a row with no finite
+    // value yet has only -inf (weight 0) or NaN (poisons T), so any finite
+    // offset serves
+    const float mo = (m == -CUDART_INF_F) ? 0.f : m;
+    const float2 nm = make_float2(-mo, -mo);
+    const float2 l2 = make_float2(kLog2e, kLog2e);
+#pragma unroll
+    for (int q = 0; q < kVecs; ++q) {
+#pragma unroll
+      for (int k = 0; k < E / 2; ++k) {
+        const float2 X = El::pair(v[q], k);
+        float2 d = __fadd2_rn(X, nm);
+        if (X.x >= tau) d.x = -CUDART_INF_F;
+        if (X.y >= tau) d.y = -CUDART_INF_F;
+        const float2 t = __fmul2_rn(d, l2);
+        const float2 w = make_float2(ex2(t.x), ex2(t.y));
+        T2 = __fadd2_rn(T2, w);
+        d.x = fmaxf(d.x, -FLT_MAX);
+        d.y = fmaxf(d.y, -FLT_MAX);
+        B2 = __ffma2_rn(w, d, B2);
+      }
+    }
+  }
+  float T = T2.x + T2.y, B = B2.x + B2.y;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    T += __shfl_xor_sync(0xffffffffu, T, off);
+    B += __shfl_xor_sync(0xffffffffu, B, off);
+  }
+  return CapPiece{m, T, B, 0};
+}
+
+template <bool kBF16>
+__global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) cap_stream_kernel(const CapParams p) {
+  wait_prior_grid();
+  const int lane = threadIdx.x & 31;
+  const int w = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  if (w >= p.nwarps) return;  // the whole warp leaves together
+  int64_t pos = warp_begin(w, p.total, p.nwarps);
+  const int64_t end = warp_begin(w + 1, p.total, p.nwarps);
+  while (pos < end) {
+    const int row = (int)(pos / p.nvec);
+    const int64_t row0 = (int64_t)row * p.nvec;
+    const int a = (int)(pos - row0);
+    const int b = (int)min((int64_t)p.nvec, end - row0);
+    const CapPiece pc = cap_piece<kBF16>(p, row, a, b, lane, p.tau[row]);
+    if (lane == 0) p.pieces[row + w] = pc;
+    pos = row0 + b;
+  }
+}
+
+// ---------------------------------------------------------------- finalize
+
+// Order-preserving 32-bit key of a non-NaN f32 value (-0 sorts with +0).
+__device__ __forceinline__ uint32_t vkey(float f) {
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float keyv(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Block sums in a fixed order (butterfly in each warp, then the warp totals
+// in warp order): every thread gets the same, reproducible result.
+template <typename T>
+__device__ T block_sum(T v, T* sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  T t = sh[0];
+  for (int i = 1; i < kFinThreads / 32; ++i) t += sh[i];
+  return t;
+}
+
+__device__ float block_max(float v, float* sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  float t = sh[0];
+  for (int i = 1; i < kFinThreads / 32; ++i) t = fmaxf(t, sh[i]);
+  return t;
+}
+
+// Merge of two pieces' tail states (the larger maximum wins; a side that has
+// seen nothing finite holds 0 or NaN and is added as it is).
+__device__ __forceinline__ CapPiece piece_merge(const CapPiece& a, const CapPiece& b) {
+  const float M = fmaxf(a.m, b.m);
+  float T = 0.f, B = 0.f;
+  if (a.m == -CUDART_INF_F || M == -CUDART_INF_F) {
+    T += a.T;
+    B += a.B;
+  } else {
+    const float s = ex2((a.m - M) * kLog2e);
+    T += s * a.T;
+    B += s * (a.B + (a.m - M) * a.T);
+  }
+  if (b.m == -CUDART_INF_F || M == -CUDART_INF_F) {
+    T += b.T;
+    B += b.B;
+  } else {
+    const float s = ex2((b.m - M) * kLog2e);
+    T += s * b.T;
+    B += s * (b.B + (b.m - M) * b.T);
+  }
+  return CapPiece{M, T, B, 0};
+}
+
+// Candidates held in shared memory.
+struct SmemCands {
+  const float* v;
+  const int* id;
+  int n;
+  __device__ __forceinline__ float val(int i) const { return v[i]; }
+  __device__ __forceinline__ int idx(int i) const { return id[i]; }
+};
+
+// Every element of a row, read from global memory (the exact path).
+template <bool kBF16>
+struct RowCands {
+  const void* row;
+  int n;
+  __device__ __forceinline__ float val(int i) const { return Elems<kBF16>::load1(row, i); }
+  __device__ __forceinline__ int idx(int i) const { return i; }
+};
+
+struct FinScratch {
+  double d[kFinThreads / 32];
+  long long ll[kFinThreads / 32];
+  int i[kFinThreads / 32];
+  float f[kFinThreads / 32];
+  int n_sel;
+};
+
+// The outputs of one row from its candidates `src` and, on the streaming
+// path, the tail state (mT, T, B) of every element that is not a candidate
+// (mT = -inf and T = B = 0 when every element is a candidate).  Every
+// thread of the CTA calls this.
+template <bool kBF16, class Src>
+__device__ void capture_finish(const CapParams& p, int row, const Src& src, float mT, float T, float B,
+                               unsigned long long* sel, FinScratch& sc) {
+  const int tid = threadIdx.x;
+  const int K = p.K;
+  const int n = src.n;
+  const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld * (kBF16 ? 2 : 4);
+  kld_top_entry* top = p.top + (int64_t)row * K;
+  float* out = p.rows + (int64_t)row * 3;
+
+  // the row's maximum; NaN or +inf anywhere makes the row invalid
+  float lm = -CUDART_INF_F;
+  int bad = 0;
+  for (int i = tid; i < n; i += kFinThreads) {
+    const float v = src.val(i);
+    bad |= (v != v) || (v == CUDART_INF_F);
+    lm = fmaxf(lm, v);
+  }
+  bad = __syncthreads_or(bad);
+  const float m = fmaxf(block_max(lm, sc.f), mT);
+  if (bad || T != T || B != B || !(m > -CUDART_INF_F) || m == CUDART_INF_F) {
+    for (int j = tid; j < K; j += kFinThreads) top[j] = kld_top_entry{-1, CUDART_NAN_F};
+    if (tid == 0) {
+      out[0] = out[1] = out[2] = CUDART_NAN_F;
+      if (p.targets) {
+        const int t = p.targets[row];
+        if (t < 0 || t >= p.vocab) set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
+      }
+    }
+    return;
+  }
+
+  // the K-th largest value key: the largest key with at least K keys >= it
+  uint32_t pre = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t t = pre | (1u << bit);
+    int c = 0;
+    for (int i = tid; i < n; i += kFinThreads) c += (vkey(src.val(i)) >= t) ? 1 : 0;
+    if (block_sum(c, sc.i) >= K) pre = t;
+  }
+  int gt = 0, eq = 0;
+  for (int i = tid; i < n; i += kFinThreads) {
+    const uint32_t k = vkey(src.val(i));
+    gt += (k > pre) ? 1 : 0;
+    eq += (k == pre) ? 1 : 0;
+  }
+  gt = block_sum(gt, sc.i);
+  eq = block_sum(eq, sc.i);
+  const int need = K - gt;  // 1 .. eq values tied at the boundary join, lowest ids first
+  uint32_t id_cut = 0xffffffffu;
+  if (need < eq) {
+    uint32_t lo = 0u;  // ends as the need-th smallest tied id
+    for (int bit = 22; bit >= 0; --bit) {
+      const uint32_t t = lo | (1u << bit);
+      int c = 0;
+      for (int i = tid; i < n; i += kFinThreads)
+        c += (vkey(src.val(i)) == pre && (uint32_t)src.idx(i) < t) ? 1 : 0;
+      if (block_sum(c, sc.i) < need) lo = t;
+    }
+    id_cut = lo;
+  }
+
+  // gather the K selected as descending-sortable keys (value key, ~id)
+  if (tid == 0) sc.n_sel = 0;
+  int P = 1;
+  while (P < K) P <<= 1;
+  for (int j = K + tid; j < P; j += kFinThreads) sel[j] = 0ull;
+  __syncthreads();
+  for (int i = tid; i < n; i += kFinThreads) {
+    const uint32_t k = vkey(src.val(i));
+    const uint32_t id = (uint32_t)src.idx(i);
+    if (k > pre || (k == pre && id <= id_cut)) {
+      const int at = atomicAdd(&sc.n_sel, 1);
+      if (at < K) sel[at] = ((unsigned long long)k << 32) | (unsigned long long)(~id);
+    }
+  }
+  __syncthreads();
+  // bitonic sort, descending
+  for (int kk = 2; kk <= P; kk <<= 1) {
+    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+      for (int i = tid; i < P; i += kFinThreads) {
+        const int ixj = i ^ jj;
+        if (ixj > i) {
+          const unsigned long long a = sel[i], b = sel[ixj];
+          const bool desc = (i & kk) == 0;
+          if (desc ? (a < b) : (a > b)) {
+            sel[i] = b;
+            sel[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // listed terms in sorted order (a fixed share per thread): the largest
+  // has weight exactly 1 and is left out of s1 so that log S = log1p(S - 1)
+  const double md = (double)m;
+  double s1 = 0.0, b1 = 0.0;
+  for (int j = tid; j < K; j += kFinThreads) {
+    const double v = (double)keyv((uint32_t)(sel[j] >> 32));
+    const double w = exp(v - md);
+    if (j > 0) s1 += w;
+    if (w > 0.0) b1 += w * (v - md);
+  }
+  s1 = block_sum(s1, sc.d);
+  b1 = block_sum(b1, sc.d);
+
+  // candidates left out of the list: every one weighs at most the K-th
+  // weight wK, so their sums go to 64-bit fixed point scaled to that bound
+  // (exact integer sums: the order candidates arrived in does not matter)
+  const unsigned long long kth = sel[K - 1];
+  const uint32_t kkey = (uint32_t)(kth >> 32), kid = ~(uint32_t)kth;
+  const double dK = (double)keyv(kkey) - md;
+  const double wK = exp(dK);
+  double s_ns = 0.0, b_ns = 0.0;
+  if (wK > 0.0 && n > K) {
+    int lg = 0;
+    while ((1 << lg) < n + 1) ++lg;
+    const double unit = ldexp(1.0, 62 - lg);                    // n * unit < 2^62
+    const double bw = (dK <= -1.0) ? wK * -dK : exp(-1.0);    // max of w |d| over d <= dK
+    long long aw = 0, ab = 0;
+    for (int i = tid; i < n; i += kFinThreads) {
+      const float v = src.val(i);
+      const uint32_t k = vkey(v);
+      const uint32_t id = (uint32_t)src.idx(i);
+      if (k > kkey || (k == kkey && id <= kid)) continue;       // listed
+      const double d = (double)v - md;
+      const double w = exp(d);
+      if (w > 0.0) {
+        aw += __double2ll_rn(w / wK * unit);
+        ab += __double2ll_rn(w * -d / bw * unit);
+      }
+    }
+    aw = block_sum(aw, sc.ll);
+    ab = block_sum(ab, sc.ll);
+    s_ns = (double)aw / unit * wK;
+    b_ns = -(double)ab / unit * bw;
+  }
+
+  // the streamed tail, moved to the row's maximum
+  double Ts = 0.0, Bs = 0.0;
+  if (mT == -CUDART_INF_F) {
+    Ts = (double)T;
+    Bs = (double)B;
+  } else {
+    const double e = exp((double)mT - md);
+    Ts = e * (double)T;
+    Bs = e * ((double)B + ((double)mT - md) * (double)T);
+  }
+  const double s_minus_1 = s1 + s_ns + Ts;
+  const double logS = log1p(s_minus_1);
+  const double S = 1.0 + s_minus_1;
+
+  for (int j = tid; j < K; j += kFinThreads) {
+    const unsigned long long e = sel[j];
+    const double v = (double)keyv((uint32_t)(e >> 32));
+    top[j] = kld_top_entry{(int32_t)(~(uint32_t)e), (float)((v - md) - logS)};
+  }
+  if (tid == 0) {
+    float nll = CUDART_NAN_F;
+    if (p.targets) {
+      const int t = p.targets[row];
+      if (t >= 0 && t < p.vocab) nll = (float)(logS - ((double)Elems<kBF16>::load1(xrow, t) - md));
+      else set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
+    }
+    out[0] = nll;
+    out[1] = (float)(logS - (b1 + b_ns + Bs) / S);
+    out[2] = (float)((s_ns + Ts) / S);
+  }
+}
+
+constexpr size_t kFinSmem = sizeof(float) * (kCap + 8) + sizeof(int) * (kCap + 8) +
+                            sizeof(unsigned long long) * kMaxK;
+
+// 3. one CTA per row.
+template <bool kBF16>
+__global__ void __launch_bounds__(kFinThreads) cap_finalize_kernel(const CapParams p) {
+  using El = Elems<kBF16>;
+  constexpr int E = El::E;
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* cv = reinterpret_cast<float*>(smem);
+  int* ci = reinterpret_cast<int*>(cv + kCap + 8);
+  unsigned long long* sel = reinterpret_cast<unsigned long long*>(ci + kCap + 8);
+  __shared__ FinScratch sc;
+  __shared__ CapPiece merged;
+  __shared__ int sh_n;
+  wait_prior_grid();
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld * (kBF16 ? 2 : 4);
+
+  // the streamed tail state: the row's pieces merged in index order (warp 0)
+  if (tid < 32) {
+    const int lane = tid;
+    CapPiece acc{-CUDART_INF_F, 0.f, 0.f, 0};
+    if (p.nvec > 0) {
+      const int64_t f = (int64_t)row * p.nvec;
+      const int w0 = warp_of(f, p.total, p.nwarps);
+      const int w1 = warp_of(f + p.nvec - 1, p.total, p.nwarps);
+      for (int c = w0; c <= w1; c += 32) {
+        const int w = c + lane;
+        CapPiece s = (w <= w1) ? p.pieces[row + w] : CapPiece{-CUDART_INF_F, 0.f, 0.f, 0};
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const CapPiece o{__shfl_xor_sync(0xffffffffu, s.m, off), __shfl_xor_sync(0xffffffffu, s.T, off),
+                           __shfl_xor_sync(0xffffffffu, s.B, off), 0};
+          s = (lane & off) ? piece_merge(o, s) : piece_merge(s, o);
+        }
+        acc = (c == w0) ? s : piece_merge(acc, s);
+      }
+    }
+    if (lane == 0) merged = acc;
+  }
+
+  // candidates: the streamed ones, then the ragged end of the row
+  const int cnt = p.count[row];
+  const int ns = min(cnt, kCap);
+  const int2* cand = p.cand + (int64_t)row * kCap;
+  for (int i = tid; i < ns; i += kFinThreads) {
+    const int2 c = cand[i];
+    cv[i] = __int_as_float(c.x);
+    ci[i] = c.y;
+  }
+  const int ragged = p.vocab - p.nvec * E;
+  const float tau = p.tau[row];
+  int ge = 0;
+  if (tid < ragged) {
+    const int id = p.nvec * E + tid;
+    const float v = El::load1(xrow, id);
+    cv[ns + tid] = v;
+    ci[ns + tid] = id;
+    ge = v >= tau ? 1 : 0;
+  }
+  ge = __syncthreads_count(ge);
+  const bool exact = p.force_exact || cnt > kCap || ns + ge < p.K;
+  if (!exact) {
+    capture_finish<kBF16>(p, row, SmemCands{cv, ci, ns + ragged}, merged.m, merged.T, merged.B, sel, sc);
+  } else {
+    // every element of the row is a candidate; nothing was left to the tail
+    capture_finish<kBF16>(p, row, RowCands<kBF16>{xrow, p.vocab}, -CUDART_INF_F, 0.f, 0.f, sel, sc);
+  }
+  (void)sh_n;
+}
+
+int stream_warps(int64_t total) {
+  int64_t w = total / kMinVecsPerWarp;
+  if (w < 1) w = 1;
+  if (w > kMaxStreamWarps) w = kMaxStreamWarps;
+  return (int)w;
+}
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+}  // namespace
+
+size_t sparse_capture_workspace_bytes(int64_t n_rows) {
+  return align256(sizeof(float) * n_rows) + align256(sizeof(int) * n_rows) +
+         align256(sizeof(CapPiece) * (n_rows + kMaxStreamWarps)) + sizeof(int2) * (size_t)n_rows * kCap;
+}
+
+cudaError_t launch_sparse_capture(const SparseCaptureArgs& a, cudaStream_t stream) {
+  const int E = a.bf16 ? 8 : 4;
+  CapParams p;
+  p.x = a.x;
+  p.ld = a.ld;
+  p.vocab = (int)a.vocab;
+  p.nvec = (int)(a.vocab / E);
+  p.n_rows = (int)a.n_rows;
+  p.total = a.n_rows * (int64_t)p.nvec;
+  p.nwarps = stream_warps(p.total);
+  p.K = a.k;
+  p.targets = a.targets;
+  char* ws = reinterpret_cast<char*>(a.workspace);
+  p.tau = reinterpret_cast<float*>(ws);
+  ws += align256(sizeof(float) * a.n_rows);
+  p.count = reinterpret_cast<int*>(ws);
+  ws += align256(sizeof(int) * a.n_rows);
+  p.pieces = reinterpret_cast<CapPiece*>(ws);
+  ws += align256(sizeof(CapPiece) * (a.n_rows + kMaxStreamWarps));
+  p.cand = reinterpret_cast<int2*>(ws);
+  p.top = a.top;
+  p.rows = a.rows;
+  p.dev_status = a.dev_status;
+  p.force_exact = a.force_exact;
+
+  const unsigned sgrid = (unsigned)((a.n_rows + kWarpsPerCta - 1) / kWarpsPerCta);
+  cudaError_t e;
+  if (a.bf16) e = launch_dependent(cap_sample_kernel<true>, dim3(sgrid), dim3(kThreads), stream, p);
+  else e = launch_dependent(cap_sample_kernel<false>, dim3(sgrid), dim3(kThreads), stream, p);
+  if (e != cudaSuccess) return e;
+  if (p.total > 0) {
+    const unsigned grid = (unsigned)((p.nwarps + kWarpsPerCta - 1) / kWarpsPerCta);
+    if (a.bf16) e = launch_dependent(cap_stream_kernel<true>, dim3(grid), dim3(kThreads), stream, p);
+    else e = launch_dependent(cap_stream_kernel<false>, dim3(grid), dim3(kThreads), stream, p);
+    if (e != cudaSuccess) return e;
+  }
+  auto fin = a.bf16 ? cap_finalize_kernel<true> : cap_finalize_kernel<false>;
+  e = cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinSmem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.n_rows);
+  cfg.blockDim = dim3(kFinThreads);
+  cfg.dynamicSmemBytes = kFinSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fin, p);
+}
+
+}  // namespace kld

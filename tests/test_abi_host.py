@@ -160,3 +160,32 @@ def test_sparse_ref_validation(lib):
     assert sr(lib, n=0) == _lib.KLD_OK
     assert lib.kld_sparse_ref_workspace_size(10, 512) > lib.kld_sparse_ref_workspace_size(10, 64)
     assert lib.kld_sparse_ref_workspace_size(10, 0) == 0
+
+
+def cp(lib, **kw):
+    a = dict(x=A16, dtype=_lib.KLD_BF16, n=4, V=4096, ld=4096, k=512, tgt=None, top=A16 + 65536,
+             rows=A16 + 131072, ws=A16 + (1 << 19), wsb=None, st=None)
+    a.update(kw)
+    wsb = lib.kld_sparse_capture_workspace_size(max(a["n"], 0), max(a["k"], 1)) if a["wsb"] is None else a["wsb"]
+    return lib.kld_sparse_capture(a["x"], a["dtype"], a["n"], a["V"], a["ld"], a["k"], a["tgt"], a["top"],
+                                  a["rows"], a["ws"], wsb, a["st"], None)
+
+
+def test_sparse_capture_validation(lib):
+    assert cp(lib, dtype=2) == _lib.KLD_ERR_UNSUPPORTED
+    assert cp(lib, k=0) == _lib.KLD_ERR_INVALID_ARG
+    assert cp(lib, k=_lib.KLD_SPARSE_MAX_K + 1) == _lib.KLD_ERR_INVALID_ARG
+    assert cp(lib, k=65, V=64, ld=64) == _lib.KLD_ERR_INVALID_ARG
+    assert cp(lib, V=(1 << 22) + 8, ld=(1 << 22) + 8) == _lib.KLD_ERR_UNSUPPORTED
+    assert cp(lib, ld=4000) == _lib.KLD_ERR_INVALID_ARG
+    assert cp(lib, n=-2) == _lib.KLD_ERR_INVALID_ARG
+    assert cp(lib, top=None) == _lib.KLD_ERR_INVALID_ARG
+    assert cp(lib, rows=None) == _lib.KLD_ERR_INVALID_ARG
+    assert cp(lib, ws=None) == _lib.KLD_ERR_WORKSPACE
+    assert cp(lib, wsb=4096) == _lib.KLD_ERR_WORKSPACE
+    assert cp(lib, x=MIS) == _lib.KLD_ERR_ALIGNMENT
+    assert cp(lib, ld=4100) == _lib.KLD_ERR_ALIGNMENT
+    assert cp(lib, top=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
+    assert cp(lib, ws=A16 + 32) == _lib.KLD_ERR_ALIGNMENT
+    assert cp(lib, n=0) == _lib.KLD_OK
+    assert lib.kld_sparse_capture_workspace_size(2, 64) > _lib.KLD_CAPTURE_CANDIDATES * 8
