@@ -7,12 +7,13 @@
 // id first.
 //
 // Three kernels:
-//  1. sample (one warp per row): 1024 evenly spaced elements of the row; the
-//     threshold tau is their 10th largest, so about 10 / 1024 of the row is
-//     at or above it (~2,400 ids at V = 248,320) while the row's top 512 are
-//     all above it unless the sample holds 10 of them (about 3e-5 for a
-//     random layout).  tau = -inf when the whole row fits the candidate
-//     buffer.
+//  1. sample (one CTA per row): 4096 evenly spaced elements of the row, 16
+//     per thread; the threshold tau is the 25th largest of the 256 thread
+//     maxima, at most the sample's own 25th largest, so about 25 / 4096 of
+//     the row is at or above it (~1,500 ids at V = 248,320) while the row's
+//     top 512 are all above it unless the sample holds 25 of them (mean 8.4
+//     for a random layout: about 1e-7).  tau = -inf when the whole row fits
+//     the candidate buffer.
 //  2. stream (persistent warps over the flattened (row, 16-byte vector)
 //     space): elements >= tau are appended, as (value, id), to the row's
 //     candidate buffer; every other element feeds the row's tail mass
@@ -46,8 +47,8 @@ constexpr int kStepVecs = 32 * kVecs;
 constexpr int kMinVecsPerWarp = 4 * kStepVecs;
 constexpr int kStreamCtasPerSm = 3;
 constexpr int kMaxStreamWarps = 148 * kStreamCtasPerSm * kWarpsPerCta;
-constexpr int kSampleElems = 1024;
-constexpr int kSampleRank = 10;
+constexpr int kSampleElems = 4096;
+constexpr int kSampleRank = 25;
 constexpr int kCap = KLD_CAPTURE_CANDIDATES;  // candidates kept per row
 constexpr int kFinThreads = 256;
 constexpr int kMaxK = KLD_SPARSE_MAX_K;
@@ -77,73 +78,71 @@ struct CapParams {
   int force_exact;     // tests only: every row takes the exact path
 };
 
-// 1. one warp per row: tau = the kSampleRank-th largest of kSampleElems
-// evenly spaced elements (counted with multiplicity); also clears the row's
-// candidate count.
+// Per-warp shared memory of the stream: the 16-byte vectors that hold
+// candidates, with their vector index in the row, gathered until the ring
+// is full and then unpacked together.
+constexpr int kRing = 256;
+struct CapRing {
+  uint4 vec[kRing];
+  int vid[kRing];
+};
+
+// Append the elements >= tau of the ring's `fill` vectors to the row's
+// candidate buffer (one atomic per 32 vectors reserves their places).
 template <bool kBF16>
-__global__ void __launch_bounds__(kThreads) cap_sample_kernel(const CapParams p) {
+__device__ void ring_flush(const CapParams& p, CapRing& R, int fill, int row, float tau, int lane) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
-  constexpr int kSampleVecs = kSampleElems / E;       // 128 (bf16) or 256 (f32)
-  constexpr int kPerLane = kSampleVecs / 32;
-  constexpr int kElemBytes = kBF16 ? 2 : 4;
-  wait_prior_grid();
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-  if (row >= p.n_rows) return;
-  if (lane == 0) p.count[row] = 0;
-  if ((int64_t)p.nvec * E <= kCap || p.nvec < kSampleVecs) {
-    if (lane == 0) p.tau[row] = -CUDART_INF_F;  // every element fits the buffer
-    return;
-  }
-  const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld * kElemBytes;
-  float v[kPerLane * E];
+  int2* cand = p.cand + (int64_t)row * kCap;
+  __syncwarp();
+  for (int j0 = 0; j0 < fill; j0 += 32) {  // warp-uniform
+    const int j = j0 + lane;
+    uint32_t em = 0u;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    int vid = 0;
+    if (j < fill) {
+      v = R.vec[j];
+      vid = R.vid[j];
 #pragma unroll
-  for (int q = 0; q < kPerLane; ++q) {
-    const int s = lane + 32 * q;
-    const int64_t vec = ((int64_t)s * p.nvec) / kSampleVecs;
-    const uint4 w = *reinterpret_cast<const uint4*>(xrow + vec * 16);
+      for (int k = 0; k < E / 2; ++k) {
+        const float2 pr = El::pair(v, k);
+        em |= (pr.x >= tau) ? (1u << (2 * k)) : 0u;
+        em |= (pr.y >= tau) ? (1u << (2 * k + 1)) : 0u;
+      }
+    }
+    const int nc = __popc(em);
+    int incl = nc;
 #pragma unroll
-    for (int k = 0; k < E / 2; ++k) {
-      const float2 pr = El::pair(w, k);
-      v[q * E + 2 * k] = pr.x;
-      v[q * E + 2 * k + 1] = pr.y;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+    int base = 0;
+    if (lane == 0 && tot > 0) base = atomicAdd(p.count + row, tot);
+    int pos = __shfl_sync(0xffffffffu, base, 0) + incl - nc;
+    while (em) {
+      const int e = __ffs(em) - 1;
+      em &= em - 1u;
+      const float2 pr = El::pair(v, e >> 1);
+      if (pos < kCap) cand[pos] = make_int2(__float_as_int((e & 1) ? pr.y : pr.x), vid * E + e);
+      ++pos;
     }
   }
-  // peel off the largest values until kSampleRank of them are counted
-  int need = kSampleRank;
-  float thr = -CUDART_INF_F;
-  for (int round = 0; round < kSampleRank; ++round) {
-    float lm = -CUDART_INF_F;
-#pragma unroll
-    for (int i = 0; i < kPerLane * E; ++i) lm = fmaxf(lm, v[i]);
-    const float M = warp_max(lm);
-    thr = M;
-    if (!(M > -CUDART_INF_F)) break;  // only -inf (or NaN) left
-    int c = 0;
-#pragma unroll
-    for (int i = 0; i < kPerLane * E; ++i) {
-      const bool hit = v[i] == M;
-      c += hit ? 1 : 0;
-      v[i] = hit ? -CUDART_INF_F : v[i];
-    }
-    need -= __reduce_add_sync(0xffffffffu, c);
-    if (need <= 0) break;
-  }
-  if (lane == 0) p.tau[row] = thr;
+  __syncwarp();
 }
 
 // 2. stream vectors [a, b) of one row; returns the piece's tail state
 // (identical in every lane) and appends the piece's candidates.
 template <bool kBF16>
-__device__ CapPiece cap_piece(const CapParams& p, int row, int a, int b, int lane, float tau) {
+__device__ CapPiece cap_piece(const CapParams& p, CapRing& R, int row, int a, int b, int lane, float tau) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
   constexpr int kElemBytes = kBF16 ? 2 : 4;
   constexpr uint32_t kNegInfWord = kBF16 ? 0xff80ff80u : 0xff800000u;
   const uint4 neg_inf = make_uint4(kNegInfWord, kNegInfWord, kNegInfWord, kNegInfWord);
   const char* yl = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld * kElemBytes + (int64_t)(a + lane) * 16;
-  int2* cand = p.cand + (int64_t)row * kCap;
+  int fill = 0;  // vectors in the ring (warp-uniform)
 
   float m = -CUDART_INF_F;  // warp-uniform
   float2 T2 = make_float2(0.f, 0.f), B2 = T2;
@@ -188,48 +187,33 @@ __device__ CapPiece cap_piece(const CapParams& p, int row, int a, int b, int lan
       m = CM;
     }
 
-    // candidates: the lanes whose vectors reach tau append their elements
-    // that do, at positions reserved by one atomic per warp
+    // candidates: vectors that reach tau go to the warp's ring
     unsigned hitq = 0u;
 #pragma unroll
     for (int q = 0; q < kVecs; ++q) hitq |= (c[q] >= tau) ? (1u << q) : 0u;
     if (__any_sync(0xffffffffu, hitq != 0u)) {
-      uint32_t emask = 0u;
-#pragma unroll
-      for (int q = 0; q < kVecs; ++q) {
-        if (!((hitq >> q) & 1u)) continue;
-#pragma unroll
-        for (int k = 0; k < E / 2; ++k) {
-          const float2 pr = El::pair(v[q], k);
-          emask |= (pr.x >= tau) ? (1u << (q * E + 2 * k)) : 0u;
-          emask |= (pr.y >= tau) ? (1u << (q * E + 2 * k + 1)) : 0u;
-        }
-      }
-      const int nc = __popc(emask);
-      int incl = nc;
+      const int nh = __popc(hitq);
+      int incl = nh;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, off);
         if (lane >= off) incl += o;
       }
       const int tot = __shfl_sync(0xffffffffu, incl, 31);
-      int base = 0;
-      if (lane == 0) base = atomicAdd(p.count + row, tot);
-      int pos = __shfl_sync(0xffffffffu, base, 0) + incl - nc;
-      while (emask) {
-        const int bit = __ffs(emask) - 1;
-        emask &= emask - 1u;
-        const int q = bit / E, e = bit % E;
-        uint4 vv = v[0];
-#pragma unroll
-        for (int qq = 1; qq < kVecs; ++qq)
-          if (qq == q) vv = v[qq];
-        const float2 pr = El::pair(vv, e >> 1);
-        const float val = (e & 1) ? pr.y : pr.x;
-        if (pos < kCap)
-          cand[pos] = make_int2(__float_as_int(val), (a + st * kStepVecs + lane + 32 * q) * E + e);
-        ++pos;
+      if (fill + tot > kRing) {
+        ring_flush<kBF16>(p, R, fill, row, tau, lane);
+        fill = 0;
       }
+      int pos = fill + incl - nh;
+#pragma unroll
+      for (int q = 0; q < kVecs; ++q) {
+        if ((hitq >> q) & 1u) {
+          R.vec[pos] = v[q];
+          R.vid[pos] = a + st * kStepVecs + lane + 32 * q;
+          ++pos;
+        }
+      }
+      fill += tot;
     }
 
     // tail and entropy sums over the non-candidates; a row with no finite
@@ -255,6 +239,7 @@ __device__ CapPiece cap_piece(const CapParams& p, int row, int a, int b, int lan
       }
     }
   }
+  if (fill > 0) ring_flush<kBF16>(p, R, fill, row, tau, lane);
   float T = T2.x + T2.y, B = B2.x + B2.y;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -266,6 +251,7 @@ __device__ CapPiece cap_piece(const CapParams& p, int row, int a, int b, int lan
 
 template <bool kBF16>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) cap_stream_kernel(const CapParams p) {
+  __shared__ CapRing rings[kWarpsPerCta];
   wait_prior_grid();
   const int lane = threadIdx.x & 31;
   const int w = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
@@ -277,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) cap_stream_kernel(
     const int64_t row0 = (int64_t)row * p.nvec;
     const int a = (int)(pos - row0);
     const int b = (int)min((int64_t)p.nvec, end - row0);
-    const CapPiece pc = cap_piece<kBF16>(p, row, a, b, lane, p.tau[row]);
+    const CapPiece pc = cap_piece<kBF16>(p, rings[threadIdx.x >> 5], row, a, b, lane, p.tau[row]);
     if (lane == 0) p.pieces[row + w] = pc;
     pos = row0 + b;
   }
@@ -369,7 +355,120 @@ struct FinScratch {
   int i[kFinThreads / 32];
   float f[kFinThreads / 32];
   int n_sel;
+  unsigned hist[256];
+  unsigned digit, rank, eq;
 };
+
+// The r-th largest (1-based) of the 32-bit keys of the elements i < n for
+// which key(i, k) returns true: an MSB-first radix select, 8 bits per pass,
+// with shared-memory histograms (lanes with equal digits add once, by
+// __match_any_sync).  Returns the key; eq = elements equal to it, rank = its
+// rank among them (eq - rank of the equal keys come after position r); rank
+// is 0 when fewer than r elements take part.
+// Every thread of the CTA calls this.
+template <class KeyFn>
+__device__ uint32_t rth_largest(int n, int r, KeyFn key, FinScratch& sc, int& eq, int& rank) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0u, pmask = 0u;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 256; b += kFinThreads) sc.hist[b] = 0u;
+    __syncthreads();
+    for (int i0 = threadIdx.x & ~31; i0 < n; i0 += kFinThreads) {  // warp-uniform trip count
+      const int i = i0 + lane;
+      uint32_t k = 0u;
+      const bool ok = i < n && key(i, k) && (k & pmask) == prefix;
+      const unsigned digit = ok ? ((k >> shift) & 255u) : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, digit);
+      if (ok && lane == __ffs(peers) - 1) atomicAdd(&sc.hist[digit], (unsigned)__popc(peers));
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane l holds bins 255 - 8l .. 248 - 8l (descending); scan from the top
+      unsigned c[8], run = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = sc.hist[255 - 8 * lane - j];
+        run += c[j];
+      }
+      unsigned incl = run;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      const unsigned base = incl - run;
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= (unsigned)r && base < (unsigned)r);
+      if (hit == 0u && lane == 0) {  // fewer than r keys: report rank 0
+        sc.digit = 0u;
+        sc.rank = 0u;
+        sc.eq = 0u;
+      }
+      if (lane == __ffs(hit) - 1) {
+        unsigned before = base, j = 0u, cj = 0u;
+        bool found = false;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          if (!found && before + c[jj] >= (unsigned)r) {
+            found = true;
+            j = (unsigned)jj;
+            cj = c[jj];
+          } else if (!found) {
+            before += c[jj];
+          }
+        }
+        sc.digit = 255u - 8u * lane - j;
+        sc.rank = (unsigned)r - before;
+        sc.eq = cj;
+      }
+    }
+    __syncthreads();
+    prefix |= sc.digit << shift;
+    pmask |= 255u << shift;
+    r = (int)sc.rank;
+  }
+  eq = (int)sc.eq;
+  rank = r;
+  return prefix;
+}
+
+// 1. one CTA per row: tau = the kSampleRank-th largest of kSampleElems
+// evenly spaced elements (counted with multiplicity); also clears the row's
+// candidate count.
+template <bool kBF16>
+__global__ void __launch_bounds__(kFinThreads) cap_sample_kernel(const CapParams p) {
+  using El = Elems<kBF16>;
+  constexpr int E = El::E;
+  constexpr int kSampleVecs = kSampleElems / E;  // 512 (bf16) or 1024 (f32)
+  __shared__ float tmax[kFinThreads];
+  __shared__ FinScratch sc;
+  wait_prior_grid();
+  const int row = blockIdx.x;
+  if (threadIdx.x == 0) p.count[row] = 0;
+  if ((int64_t)p.nvec * E <= kCap || p.nvec < kSampleVecs) {
+    if (threadIdx.x == 0) p.tau[row] = -CUDART_INF_F;  // every element fits the buffer
+    return;
+  }
+  const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld * (kBF16 ? 2 : 4);
+  // each thread keeps the largest of its sampled values; the kSampleRank-th
+  // largest of those maxima is at most the sample's own kSampleRank-th
+  // largest (a subset's), so tau only errs low: more candidates, never fewer
+  float mx = -CUDART_INF_F;
+  for (int s = threadIdx.x; s < kSampleVecs; s += kFinThreads) {
+    const int64_t vec = ((int64_t)s * p.nvec) / kSampleVecs;
+    mx = fmaxf(mx, El::vmax(*reinterpret_cast<const uint4*>(xrow + vec * 16)));
+  }
+  tmax[threadIdx.x] = mx;
+  __syncthreads();
+  int eq = 0, rank = 0;
+  const uint32_t kk = rth_largest(kFinThreads, kSampleRank, [&](int i, uint32_t& k) {
+    const float v = tmax[i];
+    k = vkey(v);
+    return v == v;  // NaN (an invalid row) takes no part
+  }, sc, eq, rank);
+  // too few sampled values to rank (NaN): every element becomes a candidate,
+  // which sends the row down the exact path
+  if (threadIdx.x == 0) p.tau[row] = rank > 0 ? keyv(kk) : -CUDART_INF_F;
+}
 
 // The outputs of one row from its candidates `src` and, on the streaming
 // path, the tail state (mT, T, B) of every element that is not a candidate
@@ -407,34 +506,20 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
     return;
   }
 
-  // the K-th largest value key: the largest key with at least K keys >= it
-  uint32_t pre = 0u;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t t = pre | (1u << bit);
-    int c = 0;
-    for (int i = tid; i < n; i += kFinThreads) c += (vkey(src.val(i)) >= t) ? 1 : 0;
-    if (block_sum(c, sc.i) >= K) pre = t;
-  }
-  int gt = 0, eq = 0;
-  for (int i = tid; i < n; i += kFinThreads) {
-    const uint32_t k = vkey(src.val(i));
-    gt += (k > pre) ? 1 : 0;
-    eq += (k == pre) ? 1 : 0;
-  }
-  gt = block_sum(gt, sc.i);
-  eq = block_sum(eq, sc.i);
-  const int need = K - gt;  // 1 .. eq values tied at the boundary join, lowest ids first
+  // the K-th largest value, and which of the values tied with it join
+  // (the lowest ids first): pre, then ids up to id_cut among the ties
+  int eq = 0, need = 0;
+  const uint32_t pre = rth_largest(n, K, [&](int i, uint32_t& k) {
+    k = vkey(src.val(i));
+    return true;
+  }, sc, eq, need);
   uint32_t id_cut = 0xffffffffu;
   if (need < eq) {
-    uint32_t lo = 0u;  // ends as the need-th smallest tied id
-    for (int bit = 22; bit >= 0; --bit) {
-      const uint32_t t = lo | (1u << bit);
-      int c = 0;
-      for (int i = tid; i < n; i += kFinThreads)
-        c += (vkey(src.val(i)) == pre && (uint32_t)src.idx(i) < t) ? 1 : 0;
-      if (block_sum(c, sc.i) < need) lo = t;
-    }
-    id_cut = lo;
+    int eq2 = 0, r2 = 0;
+    id_cut = ~rth_largest(n, need, [&](int i, uint32_t& k) {
+      k = ~(uint32_t)src.idx(i);
+      return vkey(src.val(i)) == pre;
+    }, sc, eq2, r2);
   }
 
   // gather the K selected as descending-sortable keys (value key, ~id)
@@ -496,6 +581,7 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
     while ((1 << lg) < n + 1) ++lg;
     const double unit = ldexp(1.0, 62 - lg);                    // n * unit < 2^62
     const double bw = (dK <= -1.0) ? wK * -dK : exp(-1.0);    // max of w |d| over d <= dK
+    const double to_w = unit / wK, to_b = unit / bw;
     long long aw = 0, ab = 0;
     for (int i = tid; i < n; i += kFinThreads) {
       const float v = src.val(i);
@@ -505,8 +591,8 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
       const double d = (double)v - md;
       const double w = exp(d);
       if (w > 0.0) {
-        aw += __double2ll_rn(w / wK * unit);
-        ab += __double2ll_rn(w * -d / bw * unit);
+        aw += __double2ll_rn(w * to_w);
+        ab += __double2ll_rn(w * -d * to_b);
       }
     }
     aw = block_sum(aw, sc.ll);
@@ -661,10 +747,9 @@ cudaError_t launch_sparse_capture(const SparseCaptureArgs& a, cudaStream_t strea
   p.dev_status = a.dev_status;
   p.force_exact = a.force_exact;
 
-  const unsigned sgrid = (unsigned)((a.n_rows + kWarpsPerCta - 1) / kWarpsPerCta);
   cudaError_t e;
-  if (a.bf16) e = launch_dependent(cap_sample_kernel<true>, dim3(sgrid), dim3(kThreads), stream, p);
-  else e = launch_dependent(cap_sample_kernel<false>, dim3(sgrid), dim3(kThreads), stream, p);
+  if (a.bf16) e = launch_dependent(cap_sample_kernel<true>, dim3((unsigned)a.n_rows), dim3(kFinThreads), stream, p);
+  else e = launch_dependent(cap_sample_kernel<false>, dim3((unsigned)a.n_rows), dim3(kFinThreads), stream, p);
   if (e != cudaSuccess) return e;
   if (p.total > 0) {
     const unsigned grid = (unsigned)((p.nwarps + kWarpsPerCta - 1) / kWarpsPerCta);
