@@ -50,7 +50,8 @@ constexpr int kMaxStreamWarps = 148 * kStreamCtasPerSm * kWarpsPerCta;
 constexpr int kSampleElems = 4096;
 constexpr int kSampleRank = 25;
 constexpr int kCap = KLD_CAPTURE_CANDIDATES;  // candidates kept per row
-constexpr int kFinThreads = 256;
+constexpr int kFinThreads = 128;     // finish: one CTA per row, 8 rows per SM
+constexpr int kSampleThreads = 256;  // sample: 16 sampled values per thread
 constexpr int kMaxK = KLD_SPARSE_MAX_K;
 
 // Tail state of one warp over one row piece (16 bytes): running maximum m
@@ -292,7 +293,7 @@ __device__ T block_sum(T v, T* sh) {
   if (lane == 0) sh[w] = v;
   __syncthreads();
   T t = sh[0];
-  for (int i = 1; i < kFinThreads / 32; ++i) t += sh[i];
+  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) t += sh[i];
   return t;
 }
 
@@ -303,7 +304,7 @@ __device__ float block_max(float v, float* sh) {
   if (lane == 0) sh[w] = v;
   __syncthreads();
   float t = sh[0];
-  for (int i = 1; i < kFinThreads / 32; ++i) t = fmaxf(t, sh[i]);
+  for (int i = 1; i < (int)(blockDim.x >> 5); ++i) t = fmaxf(t, sh[i]);
   return t;
 }
 
@@ -331,13 +332,18 @@ __device__ __forceinline__ CapPiece piece_merge(const CapPiece& a, const CapPiec
   return CapPiece{M, T, B, 0};
 }
 
-// Candidates held in shared memory.
-struct SmemCands {
-  const float* v;
-  const int* id;
+// Candidates: the row's streamed ones in its global buffer (read through
+// L1 on every pass), then the few of the row's ragged end, in shared memory.
+struct BufCands {
+  const int2* cand;
+  int ns;
+  const float* rv;
+  const int* ri;
   int n;
-  __device__ __forceinline__ float val(int i) const { return v[i]; }
-  __device__ __forceinline__ int idx(int i) const { return id[i]; }
+  __device__ __forceinline__ float val(int i) const {
+    return i < ns ? __int_as_float(__ldg(&cand[i].x)) : rv[i - ns];
+  }
+  __device__ __forceinline__ int idx(int i) const { return i < ns ? __ldg(&cand[i].y) : ri[i - ns]; }
 };
 
 // Every element of a row, read from global memory (the exact path).
@@ -349,11 +355,11 @@ struct RowCands {
   __device__ __forceinline__ int idx(int i) const { return i; }
 };
 
-struct FinScratch {
-  double d[kFinThreads / 32];
-  long long ll[kFinThreads / 32];
-  int i[kFinThreads / 32];
-  float f[kFinThreads / 32];
+struct FinScratch {  // block-reduction slots for up to 8 warps
+  double d[8];
+  long long ll[8];
+  int i[8];
+  float f[8];
   int n_sel;
   unsigned hist[256];
   unsigned digit, rank, eq;
@@ -371,9 +377,9 @@ __device__ uint32_t rth_largest(int n, int r, KeyFn key, FinScratch& sc, int& eq
   const int lane = threadIdx.x & 31;
   uint32_t prefix = 0u, pmask = 0u;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < 256; b += kFinThreads) sc.hist[b] = 0u;
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) sc.hist[b] = 0u;
     __syncthreads();
-    for (int i0 = threadIdx.x & ~31; i0 < n; i0 += kFinThreads) {  // warp-uniform trip count
+    for (int i0 = threadIdx.x & ~31; i0 < n; i0 += blockDim.x) {  // warp-uniform trip count
       const int i = i0 + lane;
       uint32_t k = 0u;
       const bool ok = i < n && key(i, k) && (k & pmask) == prefix;
@@ -431,15 +437,82 @@ __device__ uint32_t rth_largest(int n, int r, KeyFn key, FinScratch& sc, int& eq
   return prefix;
 }
 
+// Sort P = 128 R keys of sel[] descending with the finish CTA's 128
+// threads: a bitonic network on registers.  Thread t holds elements
+// t R .. t R + R - 1; partners closer than R are in the same thread, up to
+// 32 R apart in the same warp (shuffles), farther in another warp (shared
+// memory, the only stages with a barrier).
+// One stage of partners J < R apart inside a thread (J fixed at compile
+// time so the registers are addressed statically).
+template <int R, int J>
+__device__ __forceinline__ void local_stage(unsigned long long (&a)[R], int t, int kk) {
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if ((r ^ J) > r) {
+      const bool desc = ((t * R + r) & kk) == 0;
+      const unsigned long long x = a[r], y = a[r ^ J];
+      const bool sw = desc ? (x < y) : (x > y);
+      a[r] = sw ? y : x;
+      a[r ^ J] = sw ? x : y;
+    }
+  }
+}
+
+template <int R>
+__device__ void sort_desc(unsigned long long* sel) {
+  const int t = threadIdx.x;
+  unsigned long long a[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) a[r] = sel[t * R + r];
+  constexpr int P = kFinThreads * R;
+  for (int kk = 2; kk <= P; kk <<= 1) {
+    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+      if (jj < R) {
+        if (jj == 1) local_stage<R, 1>(a, t, kk);
+        else if (jj == 2) local_stage<R, (R > 2 ? 2 : 1)>(a, t, kk);
+        else local_stage<R, (R > 4 ? 4 : 1)>(a, t, kk);
+      } else if (jj / R < 32) {
+        const int tm = jj / R;
+        const bool lower = (t & tm) == 0;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, a[r], tm);
+          const bool desc = ((t * R + r) & kk) == 0;
+          const unsigned long long hi = a[r] > o ? a[r] : o, lo = a[r] > o ? o : a[r];
+          a[r] = (lower == desc) ? hi : lo;
+        }
+      } else {
+        const int tm = jj / R;
+        const bool lower = (t & tm) == 0;
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < R; ++r) sel[t * R + r] = a[r];
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const unsigned long long o = sel[(t ^ tm) * R + r];
+          const bool desc = ((t * R + r) & kk) == 0;
+          const unsigned long long hi = a[r] > o ? a[r] : o, lo = a[r] > o ? o : a[r];
+          a[r] = (lower == desc) ? hi : lo;
+        }
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < R; ++r) sel[t * R + r] = a[r];
+  __syncthreads();
+}
+
 // 1. one CTA per row: tau = the kSampleRank-th largest of kSampleElems
 // evenly spaced elements (counted with multiplicity); also clears the row's
 // candidate count.
 template <bool kBF16>
-__global__ void __launch_bounds__(kFinThreads) cap_sample_kernel(const CapParams p) {
+__global__ void __launch_bounds__(kSampleThreads) cap_sample_kernel(const CapParams p) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
   constexpr int kSampleVecs = kSampleElems / E;  // 512 (bf16) or 1024 (f32)
-  __shared__ float tmax[kFinThreads];
+  __shared__ float tmax[kSampleThreads];
   __shared__ FinScratch sc;
   wait_prior_grid();
   const int row = blockIdx.x;
@@ -453,14 +526,14 @@ __global__ void __launch_bounds__(kFinThreads) cap_sample_kernel(const CapParams
   // largest of those maxima is at most the sample's own kSampleRank-th
   // largest (a subset's), so tau only errs low: more candidates, never fewer
   float mx = -CUDART_INF_F;
-  for (int s = threadIdx.x; s < kSampleVecs; s += kFinThreads) {
+  for (int s = threadIdx.x; s < kSampleVecs; s += kSampleThreads) {
     const int64_t vec = ((int64_t)s * p.nvec) / kSampleVecs;
     mx = fmaxf(mx, El::vmax(*reinterpret_cast<const uint4*>(xrow + vec * 16)));
   }
   tmax[threadIdx.x] = mx;
   __syncthreads();
   int eq = 0, rank = 0;
-  const uint32_t kk = rth_largest(kFinThreads, kSampleRank, [&](int i, uint32_t& k) {
+  const uint32_t kk = rth_largest(kSampleThreads, kSampleRank, [&](int i, uint32_t& k) {
     const float v = tmax[i];
     k = vkey(v);
     return v == v;  // NaN (an invalid row) takes no part
@@ -524,7 +597,7 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
 
   // gather the K selected as descending-sortable keys (value key, ~id)
   if (tid == 0) sc.n_sel = 0;
-  int P = 1;
+  int P = kFinThreads;
   while (P < K) P <<= 1;
   for (int j = K + tid; j < P; j += kFinThreads) sel[j] = 0ull;
   __syncthreads();
@@ -537,33 +610,22 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
     }
   }
   __syncthreads();
-  // bitonic sort, descending
-  for (int kk = 2; kk <= P; kk <<= 1) {
-    for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-      for (int i = tid; i < P; i += kFinThreads) {
-        const int ixj = i ^ jj;
-        if (ixj > i) {
-          const unsigned long long a = sel[i], b = sel[ixj];
-          const bool desc = (i & kk) == 0;
-          if (desc ? (a < b) : (a > b)) {
-            sel[i] = b;
-            sel[ixj] = a;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
+  // sort, descending: P = 128 R >= K slots (the padding keys are 0)
+  if (P <= kFinThreads) sort_desc<1>(sel);
+  else if (P <= 2 * kFinThreads) sort_desc<2>(sel);
+  else if (P <= 4 * kFinThreads) sort_desc<4>(sel);
+  else sort_desc<8>(sel);
 
   // listed terms in sorted order (a fixed share per thread): the largest
-  // has weight exactly 1 and is left out of s1 so that log S = log1p(S - 1)
+  // has weight exactly 1 and is left out of s1 so that log S = log1p(S - 1).
+  // Weights are ex2 on the MUFU unit (relative error ~1e-7), sums f64.
   const double md = (double)m;
   double s1 = 0.0, b1 = 0.0;
   for (int j = tid; j < K; j += kFinThreads) {
-    const double v = (double)keyv((uint32_t)(sel[j] >> 32));
-    const double w = exp(v - md);
-    if (j > 0) s1 += w;
-    if (w > 0.0) b1 += w * (v - md);
+    const float d = keyv((uint32_t)(sel[j] >> 32)) - m;
+    const float w = ex2(d * kLog2e);
+    if (j > 0) s1 += (double)w;
+    if (w > 0.f) b1 += (double)w * (double)d;
   }
   s1 = block_sum(s1, sc.d);
   b1 = block_sum(b1, sc.d);
@@ -573,8 +635,9 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
   // (exact integer sums: the order candidates arrived in does not matter)
   const unsigned long long kth = sel[K - 1];
   const uint32_t kkey = (uint32_t)(kth >> 32), kid = ~(uint32_t)kth;
-  const double dK = (double)keyv(kkey) - md;
-  const double wK = exp(dK);
+  const float dKf = keyv(kkey) - m;
+  const double dK = (double)dKf;
+  const double wK = (double)ex2(dKf * kLog2e);
   double s_ns = 0.0, b_ns = 0.0;
   if (wK > 0.0 && n > K) {
     int lg = 0;
@@ -588,11 +651,12 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
       const uint32_t k = vkey(v);
       const uint32_t id = (uint32_t)src.idx(i);
       if (k > kkey || (k == kkey && id <= kid)) continue;       // listed
-      const double d = (double)v - md;
-      const double w = exp(d);
-      if (w > 0.0) {
+      const float df = v - m;
+      const float wf = ex2(df * kLog2e);
+      if (wf > 0.f) {
+        const double w = (double)wf;
         aw += __double2ll_rn(w * to_w);
-        ab += __double2ll_rn(w * -d * to_b);
+        ab += __double2ll_rn(w * -(double)df * to_b);
       }
     }
     aw = block_sum(aw, sc.ll);
@@ -633,21 +697,16 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
   }
 }
 
-constexpr size_t kFinSmem = sizeof(float) * (kCap + 8) + sizeof(int) * (kCap + 8) +
-                            sizeof(unsigned long long) * kMaxK;
-
 // 3. one CTA per row.
 template <bool kBF16>
-__global__ void __launch_bounds__(kFinThreads) cap_finalize_kernel(const CapParams p) {
+__global__ void __launch_bounds__(kFinThreads, 8) cap_finalize_kernel(const CapParams p) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
-  extern __shared__ __align__(16) unsigned char smem[];
-  float* cv = reinterpret_cast<float*>(smem);
-  int* ci = reinterpret_cast<int*>(cv + kCap + 8);
-  unsigned long long* sel = reinterpret_cast<unsigned long long*>(ci + kCap + 8);
+  __shared__ unsigned long long sel[kMaxK];
   __shared__ FinScratch sc;
   __shared__ CapPiece merged;
-  __shared__ int sh_n;
+  __shared__ float rv[8];
+  __shared__ int ri[8];
   wait_prior_grid();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
@@ -679,31 +738,25 @@ __global__ void __launch_bounds__(kFinThreads) cap_finalize_kernel(const CapPara
   // candidates: the streamed ones, then the ragged end of the row
   const int cnt = p.count[row];
   const int ns = min(cnt, kCap);
-  const int2* cand = p.cand + (int64_t)row * kCap;
-  for (int i = tid; i < ns; i += kFinThreads) {
-    const int2 c = cand[i];
-    cv[i] = __int_as_float(c.x);
-    ci[i] = c.y;
-  }
   const int ragged = p.vocab - p.nvec * E;
   const float tau = p.tau[row];
   int ge = 0;
   if (tid < ragged) {
     const int id = p.nvec * E + tid;
     const float v = El::load1(xrow, id);
-    cv[ns + tid] = v;
-    ci[ns + tid] = id;
+    rv[tid] = v;
+    ri[tid] = id;
     ge = v >= tau ? 1 : 0;
   }
   ge = __syncthreads_count(ge);
   const bool exact = p.force_exact || cnt > kCap || ns + ge < p.K;
   if (!exact) {
-    capture_finish<kBF16>(p, row, SmemCands{cv, ci, ns + ragged}, merged.m, merged.T, merged.B, sel, sc);
+    capture_finish<kBF16>(p, row, BufCands{p.cand + (int64_t)row * kCap, ns, rv, ri, ns + ragged}, merged.m,
+                          merged.T, merged.B, sel, sc);
   } else {
     // every element of the row is a candidate; nothing was left to the tail
     capture_finish<kBF16>(p, row, RowCands<kBF16>{xrow, p.vocab}, -CUDART_INF_F, 0.f, 0.f, sel, sc);
   }
-  (void)sh_n;
 }
 
 int stream_warps(int64_t total) {
@@ -748,8 +801,8 @@ cudaError_t launch_sparse_capture(const SparseCaptureArgs& a, cudaStream_t strea
   p.force_exact = a.force_exact;
 
   cudaError_t e;
-  if (a.bf16) e = launch_dependent(cap_sample_kernel<true>, dim3((unsigned)a.n_rows), dim3(kFinThreads), stream, p);
-  else e = launch_dependent(cap_sample_kernel<false>, dim3((unsigned)a.n_rows), dim3(kFinThreads), stream, p);
+  if (a.bf16) e = launch_dependent(cap_sample_kernel<true>, dim3((unsigned)a.n_rows), dim3(kSampleThreads), stream, p);
+  else e = launch_dependent(cap_sample_kernel<false>, dim3((unsigned)a.n_rows), dim3(kSampleThreads), stream, p);
   if (e != cudaSuccess) return e;
   if (p.total > 0) {
     const unsigned grid = (unsigned)((p.nwarps + kWarpsPerCta - 1) / kWarpsPerCta);
@@ -757,20 +810,8 @@ cudaError_t launch_sparse_capture(const SparseCaptureArgs& a, cudaStream_t strea
     else e = launch_dependent(cap_stream_kernel<false>, dim3(grid), dim3(kThreads), stream, p);
     if (e != cudaSuccess) return e;
   }
-  auto fin = a.bf16 ? cap_finalize_kernel<true> : cap_finalize_kernel<false>;
-  e = cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinSmem);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)a.n_rows);
-  cfg.blockDim = dim3(kFinThreads);
-  cfg.dynamicSmemBytes = kFinSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fin, p);
+  if (a.bf16) return launch_dependent(cap_finalize_kernel<true>, dim3((unsigned)a.n_rows), dim3(kFinThreads), stream, p);
+  return launch_dependent(cap_finalize_kernel<false>, dim3((unsigned)a.n_rows), dim3(kFinThreads), stream, p);
 }
 
 }  // namespace kld
