@@ -346,6 +346,7 @@ def run_ours(args) -> int:
         if not args.no_extra:
             line["extra_paths"] = {"topk_tail": measure_topk(args, kq, dev),
                                    "sparse_ref": measure_sparse_ref(args, kq, dev),
+                                   "sparse_capture": measure_sparse_capture(args, kq, dev),
                                    "shared_head": measure_shared_head(args, kq, dev)}
         if world == 1 and not args.no_cpu_baseline:
             rows = list(range(0, n, max(1, n // args.cpu_rows)))[:args.cpu_rows]
@@ -469,6 +470,48 @@ def measure_sparse_ref(args, kq, dev, n_rows=N_ROWS, k=512, steps=None) -> dict:
                          "frac": alg / (k_ms / 1e3) / 1e9 / peak,
                          "kernel": "kld::sparse_stream_kernel<bf16> + kld::sparse_merge_kernel<bf16>",
                          "kernel_ms": k_ms}}
+
+
+def measure_sparse_capture(args, kq, dev, n_rows=N_ROWS, k=512, steps=None) -> dict:
+    """The sparse reference record of one window: full logits (2047 x
+    248,320 bf16) -> top-512 ids and log-probs, NLL, entropy, tail mass;
+    kld_sparse_capture, inputs resident, larger than L2."""
+    import torch
+    from synth import workloads as W
+    d = W.window_full_vocab(seed=W.seed_for(2), device=dev, n_rows=n_rows)
+    x, tg = d["ref"], d["targets"]
+    n = x.shape[0]
+    top = torch.empty((n, k, 2), dtype=torch.int32, device=dev)
+    rows = torch.empty((n, 3), dtype=torch.float32, device=dev)
+    ws = torch.empty(kq.kld_sparse_capture_workspace_size(n, k), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kq.kld_sparse_capture(x, k, tg, top=top, rows=rows, workspace=ws, dev_status=status, stream=stream)
+
+    steps = steps or max(1, min(args.steps, 200))
+    for _ in range(max(3, args.warmup)):
+        step()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item()}"
+    ms = start.elapsed_time(stop) / steps
+    # logits and targets in; k (id, lp) entries and the 3-float row out
+    alg = n * (VOCAB * 2 + 4 + k * 8 + 12)
+    peak, _ = measured_peaks()
+    return {"workload": f"sparse capture: {n} positions x 248,320 bf16 logits -> top-{k} + (NLL, entropy, tail)",
+            "value": n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "step": "kld_sparse_capture (sample + stream + finish)", "gpu_launches_per_step": 3,
+            "roofline": {"bound": "hbm", "achieved": alg / (ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": alg / (ms / 1e3) / 1e9 / peak,
+                         "kernel": "kld::cap_sample_kernel + cap_stream_kernel + cap_finalize_kernel (bf16)",
+                         "kernel_ms": ms}}
 
 
 def measured_tensor_peak():
@@ -615,6 +658,8 @@ def main(argv=None) -> int:
                     help="only time the top-64 + tail path on WINDOWS windows (for profiling)")
     ap.add_argument("--profile-sparse", type=int, metavar="ROWS",
                     help="only time the sparse-reference score on ROWS positions (for profiling)")
+    ap.add_argument("--profile-capture", type=int, metavar="ROWS",
+                    help="only time the sparse capture on ROWS positions (for profiling)")
     ap.add_argument("--profile-head", nargs=2, type=int, metavar=("ROWS", "VOCAB"),
                     help="only time the shared-head path at a reduced size (for profiling)")
     ap.add_argument("--rows", type=int, default=N_ROWS,
@@ -637,6 +682,13 @@ def main(argv=None) -> int:
         kq.load_library()
         print(json.dumps(measure_sparse_ref(args, kq, torch.device("cuda:0"), n_rows=args.profile_sparse,
                                             steps=args.steps)), flush=True)
+        return 0
+    if args.profile_capture:
+        import torch
+        import quantization_fidelity_scoring_b200 as kq
+        kq.load_library()
+        print(json.dumps(measure_sparse_capture(args, kq, torch.device("cuda:0"), n_rows=args.profile_capture,
+                                                steps=args.steps)), flush=True)
         return 0
     if args.profile_head:
         import torch

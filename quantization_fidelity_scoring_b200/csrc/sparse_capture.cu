@@ -7,8 +7,8 @@
 // id first.
 //
 // Three kernels:
-//  1. sample (one CTA per row): 4096 evenly spaced elements of the row, 16
-//     per thread; the threshold tau is the 25th largest of the 256 thread
+//  1. sample (one CTA per row): 4096 elements of the row in evenly spaced
+//     runs of four 16-byte vectors (whole DRAM bursts), 16 per thread; the threshold tau is the 25th largest of the 256 thread
 //     maxima, at most the sample's own 25th largest, so about 25 / 4096 of
 //     the row is at or above it (~1,500 ids at V = 248,320) while the row's
 //     top 512 are all above it unless the sample holds 25 of them (mean 8.4
@@ -526,8 +526,12 @@ __global__ void __launch_bounds__(kSampleThreads) cap_sample_kernel(const CapPar
   // largest of those maxima is at most the sample's own kSampleRank-th
   // largest (a subset's), so tau only errs low: more candidates, never fewer
   float mx = -CUDART_INF_F;
+  // the sample is kSampleVecs / 4 runs of 4 vectors (64 bytes, 64-byte
+  // aligned), evenly spaced: whole DRAM bursts rather than 16 bytes of each
+  constexpr int kRuns = kSampleVecs / 4;
   for (int s = threadIdx.x; s < kSampleVecs; s += kSampleThreads) {
-    const int64_t vec = ((int64_t)s * p.nvec) / kSampleVecs;
+    const int64_t run0 = (((int64_t)(s >> 2) * p.nvec) / kRuns) & ~int64_t(3);
+    const int64_t vec = run0 + (s & 3);
     mx = fmaxf(mx, El::vmax(*reinterpret_cast<const uint4*>(xrow + vec * 16)));
   }
   tmax[threadIdx.x] = mx;
