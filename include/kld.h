@@ -320,7 +320,7 @@ kld_status kld_from_hidden_shared_head(const void* h_ref, const void* h_cand, co
 
 /*
  * Result of kld_reduce_stats, written to DEVICE memory.  Plain C layout:
- * 8-byte fields first, then 4-byte fields; sizeof = 360 on LP64.
+ * 8-byte fields first, then 4-byte fields; sizeof = 280 on LP64.
  */
 #define KLD_MAX_QUANTILES 8
 #define KLD_MAX_THRESHOLDS 8
@@ -377,6 +377,48 @@ kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const in
                             const double* quantiles, int32_t nq, const float* thresholds,
                             int32_t nt, kld_stats* out, void* workspace, size_t workspace_bytes,
                             int32_t* dev_status, void* stream);
+
+/*
+ * kld_reduce_shard_step - the statistics of kld_reduce_stats over the
+ * positions of several shards (ranks, or chunks scored apart), exchanging
+ * only a fixed-size block per shard and step.
+ *
+ * Defines the same quantities as kld_reduce_stats over the union of every
+ * shard's positions (the per-shard tail reports of "Qwen3.8-27B fidelity
+ * suite v5", "What is in here", are percentiles and exact exceedance counts
+ * over two shards' positions).  Order statistics and counts are exact; each
+ * shard sums its own positions in a fixed order and the shards' sums are
+ * added in shard order, so every shard gets identical statistics.
+ *
+ * Protocol: every shard calls steps 0 .. KLD_SHARD_STEPS - 1 in order, with
+ * its own arrays and workspace and the same n_shards, quantiles and
+ * thresholds.  Steps 0 .. KLD_SHARD_STEPS - 2 write this shard's block
+ * (kld_reduce_shard_block_bytes() bytes) to block_out.  Before step s + 1
+ * the caller gathers the step-s blocks of all shards, in shard order, into
+ * `gathered` (n_shards blocks back to back), e.g. with an all-gather.  The
+ * last step writes the statistics to `out`.
+ *
+ * Arguments: as kld_reduce_stats, plus
+ *   step         0 .. KLD_SHARD_STEPS - 1.
+ *   n_shards     1 .. 65536.
+ *   gathered     DEVICE, the previous step's blocks; required for step > 0; 16-byte aligned.
+ *   block_out    DEVICE, kld_reduce_shard_block_bytes(); required before the last step; 16-byte aligned.
+ *   out          DEVICE kld_stats; required at the last step only.
+ *   workspace    DEVICE, >= kld_reduce_shard_workspace_size(n) bytes, 256-byte
+ *                aligned; carries the shard's state from step to step.
+ * Which inputs are given (non-NULL) must be the same on every shard: a shard
+ * with n = 0 passes any non-NULL pointer for an input the others give (it is
+ * never read).
+ */
+#define KLD_SHARD_STEPS 5
+size_t kld_reduce_shard_block_bytes(void);
+size_t kld_reduce_shard_workspace_size(int64_t n);
+kld_status kld_reduce_shard_step(int32_t step, int32_t n_shards, const void* gathered, void* block_out,
+                                 const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
+                                 const uint8_t* top1, const float* ref_target_lp, const float* cand_target_lp,
+                                 const uint8_t* mask, int64_t n, const double* quantiles, int32_t nq,
+                                 const float* thresholds, int32_t nt, kld_stats* out, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

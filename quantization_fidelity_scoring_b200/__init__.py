@@ -7,11 +7,13 @@ from . import _lib
 from .api import (KldError, kld_from_hidden_shared_head, kld_full_vocab, kld_full_vocab_workspace_size,
                   kld_reduce_stats, kld_reduce_workspace_size, kld_shared_head_workspace_size,
                   kld_sparse_capture, kld_sparse_capture_workspace_size, kld_sparse_ref_score,
-                  kld_sparse_ref_workspace_size, kld_topk_tail, stats_to_dict)
+                  kld_sparse_ref_workspace_size, kld_topk_tail, stats_to_dict, kld_reduce_shard_step,
+                  kld_reduce_shard_block_bytes, kld_reduce_shard_workspace_size, stats_from_device)
 
 __all__ = ["KldError", "kld_from_hidden_shared_head", "kld_shared_head_workspace_size", "kld_full_vocab", "kld_full_vocab_workspace_size", "kld_topk_tail", "kld_reduce_stats",
            "kld_sparse_ref_score", "kld_sparse_ref_workspace_size", "kld_sparse_capture",
-           "kld_sparse_capture_workspace_size",
+           "kld_sparse_capture_workspace_size", "kld_reduce_shard_step", "kld_reduce_shard_block_bytes",
+           "kld_reduce_shard_workspace_size", "stats_from_device",
            "kld_reduce_workspace_size", "stats_to_dict", "load_library"]
 
 

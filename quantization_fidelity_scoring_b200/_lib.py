@@ -56,6 +56,7 @@ assert ctypes.sizeof(KldStats) == 280
 
 KLD_SPARSE_MAX_K = 1024
 KLD_CAPTURE_CANDIDATES = 8192
+KLD_SHARD_STEPS = 5
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -81,6 +82,10 @@ PROTOTYPES = {
     "kld_from_hidden_shared_head": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P,
                                                    _SZ, _P, _P]),
     "kld_reduce_workspace_size": (_SZ, [_I64]),
+    "kld_reduce_shard_block_bytes": (_SZ, []),
+    "kld_reduce_shard_workspace_size": (_SZ, [_I64]),
+    "kld_reduce_shard_step": (ctypes.c_int, [_I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _I32,
+                                             _P, _P, _SZ, _P, _P]),
     "kld_reduce_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _I32, _P, _P,
                                         _SZ, _P, _P]),
 }

@@ -296,3 +296,53 @@ def kld_reduce_stats(kl, ref_argmax=None, cand_argmax=None, top1=None, ref_targe
     host = out.cpu()
     raw = _lib.KldStats.from_buffer_copy(bytes(host.numpy().tobytes()))
     return stats_to_dict(raw)
+
+
+def kld_reduce_shard_block_bytes() -> int:
+    return int(_lib.load().kld_reduce_shard_block_bytes())
+
+
+def kld_reduce_shard_workspace_size(n: int) -> int:
+    return int(_lib.load().kld_reduce_shard_workspace_size(n))
+
+
+def kld_reduce_shard_step(step: int, n_shards: int, gathered, block_out, kl, ref_argmax=None, cand_argmax=None,
+                          top1=None, ref_target_lp=None, cand_target_lp=None, mask=None,
+                          quantiles=(0.5, 0.99, 0.999), thresholds=(), *, out=None, workspace, dev_status=None,
+                          stream=None) -> None:
+    """One step of the sharded statistics (see kld_reduce_shard_step in
+    include/kld.h).  gathered / block_out / out / workspace are device byte
+    tensors; every array argument is as in kld_reduce_stats."""
+    _need_cuda("kl", kl, torch.float32, 1)
+    n = kl.shape[0]
+    for name, t, dt in (("ref_argmax", ref_argmax, torch.int32), ("cand_argmax", cand_argmax, torch.int32),
+                        ("top1", top1, torch.uint8), ("ref_target_lp", ref_target_lp, torch.float32),
+                        ("cand_target_lp", cand_target_lp, torch.float32), ("mask", mask, torch.uint8)):
+        _need_cuda(name, t, dt, 1)
+        if t is not None and t.shape[0] != n:
+            raise ValueError(f"{name} length differs from kl")
+    qs = (ctypes.c_double * max(len(quantiles), 1))(*quantiles)
+    ts = (ctypes.c_float * max(len(thresholds), 1))(*thresholds)
+
+    def present(t):
+        # an input that is given but empty (a shard with no positions) must
+        # still read as present, like the same input on the other shards;
+        # with n == 0 the library never dereferences it
+        if t is None:
+            return None
+        return _ptr(t) if t.numel() else ctypes.c_void_p(workspace.data_ptr())
+
+    st = _lib.load().kld_reduce_shard_step(step, n_shards, _ptr(gathered), _ptr(block_out), present(kl),
+                                           present(ref_argmax), present(cand_argmax), present(top1),
+                                           present(ref_target_lp), present(cand_target_lp), present(mask), n,
+                                           ctypes.cast(qs, ctypes.c_void_p),
+                                           len(quantiles), ctypes.cast(ts, ctypes.c_void_p), len(thresholds),
+                                           _ptr(out), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                           _stream_handle(stream))
+    _check(st, "kld_reduce_shard_step")
+
+
+def stats_from_device(out) -> dict:
+    """The kld_stats struct in a device byte tensor, as a dict (synchronises)."""
+    raw = _lib.KldStats.from_buffer_copy(bytes(out.cpu().numpy().tobytes()))
+    return stats_to_dict(raw)

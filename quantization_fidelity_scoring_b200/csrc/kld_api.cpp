@@ -378,6 +378,54 @@ kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const in
   return cuda_status(kld::launch_reduce(a, static_cast<cudaStream_t>(stream)));
 }
 
+size_t kld_reduce_shard_block_bytes(void) { return kld::reduce_shard_block_bytes(); }
+
+size_t kld_reduce_shard_workspace_size(int64_t n) { return n < 0 ? 0 : kld::reduce_shard_workspace_bytes(n); }
+
+kld_status kld_reduce_shard_step(int32_t step, int32_t n_shards, const void* gathered, void* block_out,
+                                 const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
+                                 const uint8_t* top1, const float* ref_target_lp, const float* cand_target_lp,
+                                 const uint8_t* mask, int64_t n, const double* quantiles, int32_t nq,
+                                 const float* thresholds, int32_t nt, kld_stats* out, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (step < 0 || step >= KLD_SHARD_STEPS || n_shards < 1 || n_shards > 65536) return KLD_ERR_INVALID_ARG;
+  if (n < 0 || n > INT32_MAX) return KLD_ERR_INVALID_ARG;
+  if (nq < 0 || nq > KLD_MAX_QUANTILES || nt < 0 || nt > KLD_MAX_THRESHOLDS) return KLD_ERR_INVALID_ARG;
+  if ((nq > 0 && !quantiles) || (nt > 0 && !thresholds)) return KLD_ERR_INVALID_ARG;
+  if ((ref_argmax == nullptr) != (cand_argmax == nullptr)) return KLD_ERR_INVALID_ARG;
+  if (n > 0 && !kl) return KLD_ERR_INVALID_ARG;
+  if (step > 0 && !gathered) return KLD_ERR_INVALID_ARG;
+  if (step < KLD_SHARD_STEPS - 1 && !block_out) return KLD_ERR_INVALID_ARG;
+  if (step == KLD_SHARD_STEPS - 1 && !out) return KLD_ERR_INVALID_ARG;
+  for (int i = 0; i < nq; ++i)
+    if (!(quantiles[i] >= 0.0 && quantiles[i] <= 1.0)) return KLD_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < kld::reduce_shard_workspace_bytes(n)) return KLD_ERR_WORKSPACE;
+  if (!aligned(out, 8) || !aligned(workspace, 256) || !aligned(gathered, 16) || !aligned(block_out, 16) ||
+      !aligned(kl, 4) || !aligned(ref_argmax, 4) || !aligned(cand_argmax, 4) || !aligned(ref_target_lp, 4) ||
+      !aligned(cand_target_lp, 4) || !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+  kld::ReduceArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.kl = kl;
+  a.ref_argmax = ref_argmax;
+  a.cand_argmax = cand_argmax;
+  a.top1 = top1;
+  a.ref_lp = ref_target_lp;
+  a.cand_lp = cand_target_lp;
+  a.mask = mask;
+  a.n = n;
+  a.nq = nq;
+  a.nt = nt;
+  for (int i = 0; i < nq; ++i) a.quantiles[i] = quantiles[i];
+  for (int i = 0; i < nt; ++i) a.thresholds[i] = thresholds[i];
+  a.out = out;
+  a.workspace = workspace;
+  a.dev_status = dev_status;
+  return cuda_status(kld::launch_reduce_shard_step(a, step, n_shards, gathered, block_out,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 
+static_assert(KLD_SHARD_STEPS == kld::kShardSteps, "shard step count");
 static_assert(sizeof(kld_stats) == 280, "kld_stats layout changed: update the Python mirror");

@@ -123,5 +123,14 @@ struct ReduceArgs {
 };
 size_t reduce_workspace_bytes(int64_t n);
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream);
+// Statistics over several shards' positions, one step of a shard (see
+// kld_reduce_shard_step): steps 0 .. 3 add this shard's pass histogram (and
+// at step 0 its sums) to block_out; steps 1 .. 4 first add up the gathered
+// blocks of the previous step; step 4 writes the statistics.
+size_t reduce_shard_block_bytes();
+size_t reduce_shard_workspace_bytes(int64_t n);
+constexpr int kShardSteps = 5;
+cudaError_t launch_reduce_shard_step(const ReduceArgs& a, int step, int n_shards, const void* gathered,
+                                     void* block_out, cudaStream_t stream);
 
 }  // namespace kld

@@ -49,9 +49,10 @@ struct ReduceParams {
   double q[KLD_MAX_QUANTILES];
   float thr[KLD_MAX_THRESHOLDS];
   kld_stats* out;
-  unsigned* hist;     // [kPasses][kMaxTargets][kBins]
+  unsigned* hist;     // [kPasses][kMaxTargets][kBins]: the histograms of all positions
   Partial* partials;  // [gridDim of pass 0]
   int32_t* dev_status;
+  unsigned* hist_out; // where a pass adds its histogram (null: hist's own slot for the pass)
 };
 
 __device__ __forceinline__ uint32_t f2key(float f) {
@@ -414,7 +415,7 @@ __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReducePa
     if (threadIdx.x == 0) p.partials[blockIdx.x] = acc;
   }
   __syncthreads();
-  unsigned* g = p.hist + pass * kMaxTargets * kBins;
+  unsigned* g = p.hist_out ? p.hist_out : p.hist + pass * kMaxTargets * kBins;
   const int used = (pass == 0) ? kBins : sel.nu * kBins;
   for (int i = threadIdx.x; i < used; i += blockDim.x)
     if (sh[i]) atomicAdd(&g[i], sh[i]);
@@ -428,6 +429,60 @@ __global__ void __launch_bounds__(kBigThreads) reduce_final_kernel(const ReduceP
   Partial tot = p.partials[0];
   for (int b = 1; b < n_partials; ++b) partial_add(tot, p.partials[b]);
   write_stats(p, tot, sel);
+}
+
+// ---------------------------------------------------------------- shards
+//
+// Statistics over positions held by several shards: every shard runs the
+// passes of the grid path on its own positions, and between passes the
+// shards exchange fixed-size blocks (their pass histogram; at the first
+// pass also their sums).  Each shard adds the gathered blocks up in shard
+// order, so every shard holds the same totals and derives the same select
+// state and statistics.
+
+struct ShardBlock {
+  Partial partial;
+  unsigned hist[kMaxTargets * kBins];
+};
+
+// this shard's block: histogram cleared (before a pass adds into it)
+__global__ void shard_clear_kernel(ShardBlock* blk) {
+  wait_prior_grid();
+  for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) blk->hist[i] = 0u;
+}
+
+// this shard's sums of the first pass: its CTAs' partials in CTA order
+__global__ void shard_fold_kernel(const ReduceParams p, int n_partials, ShardBlock* blk) {
+  wait_prior_grid();
+  if (threadIdx.x != 0) return;
+  Partial tot = p.partials[0];
+  for (int b = 1; b < n_partials; ++b) partial_add(tot, p.partials[b]);
+  blk->partial = tot;
+}
+
+// all shards' blocks of pass `pass`: histograms into the totals, in shard
+// order (integers: exact); after the first pass also the sums (shard order)
+__global__ void shard_gather_kernel(const ReduceParams p, int pass, const ShardBlock* gathered, int n_shards,
+                                    Partial* total) {
+  wait_prior_grid();
+  unsigned* h = p.hist + pass * kMaxTargets * kBins;
+  for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) {
+    unsigned c = 0u;
+    for (int s = 0; s < n_shards; ++s) c += gathered[s].hist[i];
+    h[i] = c;
+  }
+  if (pass == 0 && threadIdx.x == 0) {
+    Partial t = gathered[0].partial;
+    for (int s = 1; s < n_shards; ++s) partial_add(t, gathered[s].partial);
+    *total = t;
+  }
+}
+
+__global__ void __launch_bounds__(kBigThreads) shard_final_kernel(const ReduceParams p, const Partial* total) {
+  wait_prior_grid();
+  __shared__ Select sel;
+  select_replay(sel, p, kPasses);
+  if (threadIdx.x == 0) write_stats(p, *total, sel);
 }
 
 int big_grid(long long n) {
@@ -445,6 +500,11 @@ size_t reduce_workspace_bytes(int64_t n) {
   (void)n;
   return kHistBytes + sizeof(Partial) * kMaxBigBlocks;
 }
+
+size_t reduce_shard_block_bytes() { return sizeof(ShardBlock); }
+
+// the shard workspace: the grid path's, then the all-shard sums
+size_t reduce_shard_workspace_bytes(int64_t n) { return reduce_workspace_bytes(n) + sizeof(Partial); }
 
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
   ReduceParams p;
@@ -464,6 +524,7 @@ cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
   p.hist = reinterpret_cast<unsigned*>(a.workspace);
   p.partials = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes);
   p.dev_status = a.dev_status;
+  p.hist_out = nullptr;
 
   if (a.n <= kSmallN) return launch_dependent(reduce_small_kernel, dim3(1), dim3(kSmallThreads), stream, p);
   const int grid = big_grid(a.n);
@@ -472,6 +533,45 @@ cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
     e = launch_dependent(reduce_pass_kernel, dim3(grid), dim3(kBigThreads), stream, p, pass);
   if (e != cudaSuccess) return e;
   return launch_dependent(reduce_final_kernel, dim3(1), dim3(kBigThreads), stream, p, grid);
+}
+
+cudaError_t launch_reduce_shard_step(const ReduceArgs& a, int step, int n_shards, const void* gathered,
+                                     void* block_out, cudaStream_t stream) {
+  ReduceParams p;
+  p.kl = a.kl;
+  p.ra = a.ref_argmax;
+  p.ca = a.cand_argmax;
+  p.top1 = a.top1;
+  p.lpr = a.ref_lp;
+  p.lpc = a.cand_lp;
+  p.mask = a.mask;
+  p.n = a.n;
+  p.nq = a.nq;
+  p.nt = a.nt;
+  for (int i = 0; i < KLD_MAX_QUANTILES; ++i) p.q[i] = a.quantiles[i];
+  for (int i = 0; i < KLD_MAX_THRESHOLDS; ++i) p.thr[i] = a.thresholds[i];
+  p.out = a.out;
+  p.hist = reinterpret_cast<unsigned*>(a.workspace);
+  p.partials = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes);
+  p.dev_status = a.dev_status;
+  Partial* total = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes +
+                                              sizeof(Partial) * kMaxBigBlocks);
+  ShardBlock* blk = reinterpret_cast<ShardBlock*>(block_out);
+  const ShardBlock* all = reinterpret_cast<const ShardBlock*>(gathered);
+  const int grid = big_grid(a.n);
+  cudaError_t e = cudaSuccess;
+  if (step > 0) {  // the previous pass, all shards
+    e = launch_dependent(shard_gather_kernel, dim3(1), dim3(1024), stream, p, step - 1, all, n_shards, total);
+    if (e != cudaSuccess) return e;
+  }
+  if (step == kPasses) return launch_dependent(shard_final_kernel, dim3(1), dim3(kBigThreads), stream, p,
+                                               (const Partial*)total);
+  e = launch_dependent(shard_clear_kernel, dim3(1), dim3(1024), stream, blk);
+  if (e != cudaSuccess) return e;
+  p.hist_out = blk->hist;
+  e = launch_dependent(reduce_pass_kernel, dim3(grid), dim3(kBigThreads), stream, p, step);
+  if (e != cudaSuccess || step != 0) return e;
+  return launch_dependent(shard_fold_kernel, dim3(1), dim3(32), stream, p, grid, blk);
 }
 
 }  // namespace kld

@@ -189,3 +189,34 @@ def test_sparse_capture_validation(lib):
     assert cp(lib, ws=A16 + 32) == _lib.KLD_ERR_ALIGNMENT
     assert cp(lib, n=0) == _lib.KLD_OK
     assert lib.kld_sparse_capture_workspace_size(2, 64) > _lib.KLD_CAPTURE_CANDIDATES * 8
+
+
+def sh(lib, **kw):
+    a = dict(step=1, ns=2, g=A16, b=A16 + 65536, kl=A16 + 131072, n=100, q=(0.5,), out=None,
+             ws=A16 + (1 << 19), wsb=None)
+    a.update(kw)
+    qs = (ctypes.c_double * max(8, len(a["q"])))(*a["q"])
+    ts = (ctypes.c_float * 8)()
+    wsb = lib.kld_reduce_shard_workspace_size(max(a["n"], 0)) if a["wsb"] is None else a["wsb"]
+    return lib.kld_reduce_shard_step(a["step"], a["ns"], a["g"], a["b"], a["kl"], None, None, None, None, None,
+                                     None, a["n"], ctypes.cast(qs, ctypes.c_void_p), len(a["q"]),
+                                     ctypes.cast(ts, ctypes.c_void_p), 0, a["out"], a["ws"], wsb, None, None)
+
+
+def test_reduce_shard_validation(lib):
+    last = _lib.KLD_SHARD_STEPS - 1
+    assert sh(lib, step=-1) == _lib.KLD_ERR_INVALID_ARG
+    assert sh(lib, step=last + 1) == _lib.KLD_ERR_INVALID_ARG
+    assert sh(lib, ns=0) == _lib.KLD_ERR_INVALID_ARG
+    assert sh(lib, g=None) == _lib.KLD_ERR_INVALID_ARG                 # the previous blocks are needed
+    assert sh(lib, b=None) == _lib.KLD_ERR_INVALID_ARG                 # this shard's block is needed
+    assert sh(lib, step=last, b=None, out=None) == _lib.KLD_ERR_INVALID_ARG
+    assert sh(lib, q=(2.0,)) == _lib.KLD_ERR_INVALID_ARG
+    assert sh(lib, kl=None) == _lib.KLD_ERR_INVALID_ARG
+    assert sh(lib, ws=None) == _lib.KLD_ERR_WORKSPACE
+    assert sh(lib, wsb=8) == _lib.KLD_ERR_WORKSPACE
+    assert sh(lib, g=A16 + 8) == _lib.KLD_ERR_ALIGNMENT
+    assert sh(lib, ws=A16 + 64) == _lib.KLD_ERR_ALIGNMENT
+    assert sh(lib, step=last, b=None, out=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
+    assert lib.kld_reduce_shard_block_bytes() >= 16 * 256 * 4
+    assert lib.kld_reduce_shard_workspace_size(10) > lib.kld_reduce_workspace_size(10)

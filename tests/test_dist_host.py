@@ -78,3 +78,50 @@ def test_reference_arm_under_torchrun_prints_once(tmp_path):
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["value"] > 0 and line["higher_is_better"] is True
+
+
+class _StampStep:
+    """Stands in for the library's shard step on CPU: writes (rank, step)
+    into this rank's block and checks the blocks gathered from the previous
+    step came from every rank, in rank order."""
+    block_bytes = 64
+
+    def __init__(self, rank, world):
+        self.rank, self.world, self.seen = rank, world, []
+
+    def __call__(self, step, n_shards, gathered, block_out, *arrays, out=None, workspace=None, **kw):
+        assert n_shards == self.world
+        if step > 0:
+            g = gathered.view(self.world, self.block_bytes)
+            for r in range(self.world):
+                assert g[r, 0].item() == r and g[r, 1].item() == step - 1, (step, r, g[r, :2])
+            self.seen.append(step)
+        if block_out is not None:
+            block_out.zero_()
+            block_out[0], block_out[1] = self.rank, step
+        else:
+            out.fill_(7)
+
+
+def _shard_main(rank, world, port, out_dir):
+    from quantization_fidelity_scoring_b200 import shards
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        fake = _StampStep(rank, world)
+        kl = torch.zeros(5 + rank)
+        out = shards.reduce_stats_across_ranks(kl, step_fn=fake)
+        with open(os.path.join(out_dir, f"shard{rank}.json"), "w") as f:
+            json.dump({"seen": fake.seen, "out": int(out[0].item())}, f)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_shard_exchange_two_gloo_ranks(tmp_path):
+    """The sharded statistics' exchange: after every step each rank holds
+    every rank's block, in rank order, and the last step runs everywhere."""
+    world, port = 2, free_port()
+    mp.start_processes(_shard_main, args=(world, port, str(tmp_path)), nprocs=world, start_method="spawn")
+    for r in range(world):
+        res = json.load(open(tmp_path / f"shard{r}.json"))
+        assert res["seen"] == [1, 2, 3, 4] and res["out"] == 7
