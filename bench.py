@@ -6,9 +6,11 @@ One step scores one window of full-vocabulary logits (2047 positions x
 248,320 vocabulary ids, bf16, seeded synthetic Zipf/Gumbel rows) with
 kld_full_vocab and reduces it with kld_reduce_stats (mean, median, p99,
 p99.9, top-1, perplexity).  Inputs are resident in HBM and larger than L2
-(2.03 GB per step).  With N GPUs (torchrun) every rank scores its own window:
-weak scaling, no collective on the data path; the timing is the max over
-ranks.  Rank 0 prints one JSON line.
+(2.03 GB per step).  With N GPUs (torchrun) every rank scores its own window
+(weak scaling) and the step's statistics cover every rank's positions: the
+reduction runs as shard steps with an all-gather of one small block per rank
+between them, the only collective on the data path; the timing is the max
+over ranks.  Rank 0 prints one JSON line.
 
 --impl reference times the f64 CPU oracle on the same workload instead.
 """
@@ -234,13 +236,15 @@ def run_reference(args) -> int:
     return 0
 
 
-def config_dict(rows: int = N_ROWS) -> dict:
+def config_dict(rows: int = N_ROWS, world: int = 1) -> dict:
     workload = WORKLOAD if rows == N_ROWS else WORKLOAD.replace("2047 positions", f"{rows} positions") + \
         " (reduced profiling case)"
     return {"workload": workload, "n_rows": rows, "vocab": VOCAB, "input_dtype": "bf16",
             "step": "kld_full_vocab + kld_reduce_stats (mean, p50, p99, p99.9, top-1, ppl)",
             "l2": f"inputs larger than L2: {2 * rows * VOCAB * 2 / 1e9:.2f} GB of logits per step",
-            "parallelism": "dp (each rank scores its own window)"}
+            "parallelism": "dp (each rank scores its own window)" if world == 1 else
+            f"dp{world}: each rank scores its own window; the statistics cover all ranks' positions "
+            "(shard steps with an all-gather of one 16.5 KB block per rank and step)"}
 
 
 def run_ours(args) -> int:
@@ -272,6 +276,10 @@ def run_ours(args) -> int:
     fws = torch.empty(kq.kld_full_vocab_workspace_size(n), dtype=torch.uint8, device=dev)
     stats_buf = torch.empty(280, dtype=torch.uint8, device=dev)
 
+    if world > 1:
+        from quantization_fidelity_scoring_b200 import shards
+        sws = torch.empty(kq.kld_reduce_shard_workspace_size(n), dtype=torch.uint8, device=dev)
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
@@ -279,8 +287,14 @@ def run_ours(args) -> int:
                           cand_target_lp=lpc, workspace=fws, dev_status=status, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf,
-                            workspace=ws, dev_status=status, stream=stream, to_host=False)
+        if world > 1:
+            # the statistics of every rank's positions: shard steps with an
+            # all-gather of each step's 16.5 KB block
+            shards.reduce_stats_across_ranks(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf,
+                                             workspace=sws, dev_status=status, to_host=False)
+        else:
+            kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf,
+                                workspace=ws, dev_status=status, stream=stream, to_host=False)
 
     sampler = ClockSampler(local).start()
     # warm-up: at least W steps and about a second of load so the clocks settle
@@ -339,8 +353,8 @@ def run_ours(args) -> int:
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded Zipf/Gumbel logits; no corpus or model)",
-            "config": config_dict(args.rows), "roofline": roofline,
-            "clocks": sampler.summary(t0, t1), "gpu_launches": launches_per_step(n) * args.steps,
+            "config": config_dict(args.rows, world), "roofline": roofline,
+            "clocks": sampler.summary(t0, t1), "gpu_launches": launches_per_step(n, world) * args.steps,
             "e2e": e2e,
         }
         if not args.no_extra:
@@ -360,9 +374,12 @@ def run_ours(args) -> int:
     return 0
 
 
-def launches_per_step(n: int) -> int:
+def launches_per_step(n: int, world: int = 1) -> int:
     """Library kernels per step: streaming pass + piece merge + reduction
-    (one CTA up to 65,536 positions, else zero + 4 passes + final)."""
+    (one CTA up to 65,536 positions, else zero + 4 passes + final; across
+    ranks the five shard steps: 3 + 3 x 3 + 2 kernels)."""
+    if world > 1:
+        return 2 + 14
     return 2 + (1 if n <= 65536 else 6)
 
 
@@ -603,6 +620,9 @@ def measure_e2e(args, kq, d, dev, world) -> dict:
     h_stats = torch.empty(280, dtype=torch.uint8).pin_memory()
     comp = torch.cuda.current_stream()
     copy = torch.cuda.Stream(device=dev)
+    if world > 1:
+        from quantization_fidelity_scoring_b200 import shards
+        sws = torch.empty(kq.kld_reduce_shard_workspace_size(n), dtype=torch.uint8, device=dev)
     chunks = [(a, min(n, a + chunk)) for a in range(0, n, chunk)]
 
     def step():
@@ -620,8 +640,12 @@ def measure_e2e(args, kq, d, dev, world) -> dict:
             kq.kld_full_vocab(d_ref[a:b], d_cand[a:b], d_t[a:b], kl=kl[a:b], ref_argmax=ra[a:b],
                               cand_argmax=ca[a:b], ref_target_lp=lpr[a:b], cand_target_lp=lpc[a:b],
                               workspace=fws, stream=comp)
-        kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf, workspace=ws,
-                            stream=comp, to_host=False)
+        if world > 1:
+            shards.reduce_stats_across_ranks(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf,
+                                             workspace=sws, to_host=False)
+        else:
+            kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf, workspace=ws,
+                                stream=comp, to_host=False)
         h_stats.copy_(stats_buf, non_blocking=True)
         comp.synchronize()
 
