@@ -11,12 +11,15 @@
 // advances two positions.  Lane l of a half holds list slots 4l .. 4l+3
 // (vector loads when k is a multiple of 4; element loads otherwise).
 // Matching: the candidate's ids go into a 256-slot open-addressed table in
-// shared memory whose 64-bit entries hold (id, slot, fp16 log-prob); the
-// load factor is at most 1/4, so almost every insert and lookup finishes at
-// its first probe and lanes rarely diverge, and the two halves' tables are
-// offset by 16 banks.  A repeated candidate id keeps its lowest slot
-// (atomicMin on the packed entry).  Results do not depend on the order of
-// insertion, so they are deterministic.  The three masses that feed 1 - sum
+// shared memory of 32-bit entries (id << 6 | list slot), and their fp16
+// log-probs into a per-position array by list slot; the load factor is at
+// most 1/4, so almost every insert and lookup finishes at its first probe,
+// and the two halves' tables are offset by 16 banks.  The inserts are
+// shared-memory compare-and-swaps, which the hardware serialises per lane,
+// and with the table traffic they bound this kernel; 64-bit entries that
+// carried the log-prob cost 10 % more.  A repeated candidate id keeps its
+// lowest slot (atomicMin on the entry).  Results do not depend on the order
+// of insertion, so they are deterministic.  The three masses that feed 1 - sum
 // (candidate list, reference list, matched candidate cells) are exp on the
 // MUFU unit accumulated in f64, in fixed lane order; the KL terms are f32
 // and the tail term takes one logarithm of the f64 ratio p_tail / q_tail.
@@ -36,8 +39,8 @@ constexpr int kPerWarp = 32 / kGroup;        // positions per warp
 constexpr int kPer = 64 / kGroup;            // list slots per lane
 constexpr int kPositions = kWarps * kPerWarp;
 constexpr int kSlots = 256;                  // >= 4 * 64: short probe chains that always end
-constexpr int kTableStride = kSlots + 8;     // 64-bit words; next table starts 16 banks over
-constexpr unsigned long long kEmpty = ~0ull;
+constexpr int kTableStride = kSlots + 64 + 16;  // 32-bit words: table, then 64 fp16 log-probs (32 words)
+constexpr uint32_t kEmpty = ~0u;
 constexpr double kQFloor = 1e-12;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -55,12 +58,10 @@ __device__ __forceinline__ float fast_log(float x) {
   return r * kLn2;
 }
 
-// Entry: id in bits 22..46, list slot in 16..21, fp16 log-prob bits in 0..15.
-// For equal ids the lower slot is the smaller entry.
-__device__ __forceinline__ unsigned long long pack(uint32_t id, int slot, uint16_t lp) {
-  return ((unsigned long long)id << 22) | ((unsigned long long)slot << 16) | lp;
-}
-__device__ __forceinline__ uint32_t entry_id(unsigned long long e) { return (uint32_t)(e >> 22); }
+// Entry: id in bits 6..31, list slot in 0..5.  For equal ids the lower slot
+// is the smaller entry.
+__device__ __forceinline__ uint32_t pack(uint32_t id, int slot) { return (id << 6) | (uint32_t)slot; }
+__device__ __forceinline__ uint32_t entry_id(uint32_t e) { return e >> 6; }
 
 // Butterfly sums inside a 16-lane group (offsets 8, 4, 2, 1 stay in the group).
 template <typename T>
@@ -116,7 +117,7 @@ __device__ __forceinline__ void load_list(const TopkParams& p, const int32_t* id
 }
 
 __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p) {
-  __shared__ __align__(16) unsigned long long table[kPositions * kTableStride];
+  __shared__ __align__(16) uint32_t table[kPositions * kTableStride];
 
   wait_prior_grid();
   const int lane = threadIdx.x & 31;
@@ -126,7 +127,8 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
   const unsigned gmask = 0xffffu << (grp * kGroup);
   const int k = p.k;
   const uint32_t V = (uint32_t)p.vocab;
-  unsigned long long* tab = table + gslot * kTableStride;
+  uint32_t* tab = table + gslot * kTableStride;
+  uint16_t* clp = reinterpret_cast<uint16_t*>(tab + kSlots);
 
   const int64_t n_iter = (p.n_rows + kPerWarp - 1) / kPerWarp;
   for (int64_t it = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); it < n_iter;
@@ -149,10 +151,11 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
 
     // clear this group's table: 16 lanes x 8 stores of 16 bytes
     {
-      ulonglong2* t2 = reinterpret_cast<ulonglong2*>(tab);
-      const ulonglong2 e2 = make_ulonglong2(kEmpty, kEmpty);
+      uint4* t4 = reinterpret_cast<uint4*>(tab);
 #pragma unroll
-      for (int s = gl; s < kSlots / 2; s += kGroup) t2[s] = e2;
+      for (int s = gl; s < kSlots / 4; s += kGroup) t4[s] = make_uint4(kEmpty, kEmpty, kEmpty, kEmpty);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) clp[gl * kPer + i] = cb[i];
     }
     __syncwarp();
     if (!bad) {
@@ -160,10 +163,10 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
       for (int i = 0; i < kPer; ++i) {
         if (!valid[i]) continue;
         const uint32_t id = (uint32_t)c[i];
-        const unsigned long long entry = pack(id, gl * kPer + i, cb[i]);
+        const uint32_t entry = pack(id, gl * kPer + i);
         uint32_t s = slot_of(id);
         for (int probe = 0; probe < kSlots; ++probe) {
-          const unsigned long long old = atomicCAS(&tab[s], kEmpty, entry);
+          const uint32_t old = atomicCAS(&tab[s], kEmpty, entry);
           if (old == kEmpty) break;
           if (entry_id(old) == id) {
             atomicMin(&tab[s], entry);
@@ -188,13 +191,13 @@ __global__ void __launch_bounds__(kThreads) topk_tail_kernel(const TopkParams p)
         p_sum += (double)pj;
         const uint32_t id = (uint32_t)r[i];
         uint32_t s = slot_of(id);
-        unsigned long long e = tab[s];
+        uint32_t e = tab[s];
         for (int probe = 1; probe < kSlots && e != kEmpty && entry_id(e) != id; ++probe) {
           s = (s + 1) & (kSlots - 1);  // rare at load factor 1/4
           e = tab[s];
         }
         if (e != kEmpty && entry_id(e) == id) {
-          const float bm = h2f((uint16_t)(e & 0xffffu));
+          const float bm = h2f(clp[e & 63u]);
           qm_sum += (double)mass(bm);
           klm += pj * (a - bm);
           ++matched;
