@@ -531,6 +531,52 @@ def measure_sparse_capture(args, kq, dev, n_rows=N_ROWS, k=512, steps=None) -> d
                          "kernel_ms": ms}}
 
 
+def measure_reduce(args, kq, dev, n=N_ROWS, steps=None) -> dict:
+    """Only the statistics (kld_reduce_stats: mean, p50/p99/p99.9, top-1,
+    perplexities) of n positions' results, resident on the device."""
+    from synth import workloads as W
+    import torch
+    d = W.position_results(seed=window_seed(0) + 7, device=dev, n=n)
+    out = torch.empty(280, dtype=torch.uint8, device=dev)
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(s=stream):
+        kq.kld_reduce_stats(d["kl"], d["ra"], d["ca"], None, d["lpr"], d["lpc"], None, QUANTILES, (), out=out,
+                            workspace=ws, dev_status=status, stream=s, to_host=False)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    k = steps or args.steps
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(k):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    host_ms = a.elapsed_time(b) / k
+    # the same calls replayed from a CUDA graph: device time without the
+    # host's per-call cost
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for _ in range(k):
+            step(side)
+    graph.replay()
+    torch.cuda.synchronize()
+    a.record(stream)
+    graph.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ms = a.elapsed_time(b) / k
+    return {"path": "kld_reduce_stats", "positions": n, "ms": ms, "us": ms * 1e3, "us_host_loop": host_ms * 1e3,
+            "launches_per_step": launches_per_step(n) - 2}
+
+
 def measured_tensor_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -684,6 +730,8 @@ def main(argv=None) -> int:
                     help="only time the sparse-reference score on ROWS positions (for profiling)")
     ap.add_argument("--profile-capture", type=int, metavar="ROWS",
                     help="only time the sparse capture on ROWS positions (for profiling)")
+    ap.add_argument("--profile-reduce", type=int, metavar="POSITIONS",
+                    help="only time the statistics of POSITIONS per-position results (for profiling)")
     ap.add_argument("--profile-head", nargs=2, type=int, metavar=("ROWS", "VOCAB"),
                     help="only time the shared-head path at a reduced size (for profiling)")
     ap.add_argument("--rows", type=int, default=N_ROWS,
@@ -713,6 +761,12 @@ def main(argv=None) -> int:
         kq.load_library()
         print(json.dumps(measure_sparse_capture(args, kq, torch.device("cuda:0"), n_rows=args.profile_capture,
                                                 steps=args.steps)), flush=True)
+        return 0
+    if args.profile_reduce:
+        import torch
+        import quantization_fidelity_scoring_b200 as kq
+        kq.load_library()
+        print(json.dumps(measure_reduce(args, kq, torch.device("cuda:0"), n=args.profile_reduce)), flush=True)
         return 0
     if args.profile_head:
         import torch

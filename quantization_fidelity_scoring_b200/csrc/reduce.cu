@@ -8,13 +8,23 @@
 //
 // Order statistics are exact: the f32 KL bit patterns are mapped to
 // order-preserving 32-bit keys and each requested rank is found by an
-// MSB-first radix select, 8 bits per pass (4 passes), with integer
-// histograms.  Sums are f64 in fixed orders (per-thread strided, then fixed
-// trees), so every output is bitwise reproducible.
+// MSB-first radix select over integer histograms.  kld_reduce_stats takes
+// the key in three digits of 12, 10 and 10 bits; each pass histograms only
+// the keys whose leading digits match a target's prefix so far.  Sums are
+// f64 (counts 32-bit integers) in fixed orders: per-thread strided, then
+// fixed shuffle trees, then CTA partials in CTA order, so every output is
+// bitwise reproducible.
 //
-// Small inputs (n <= kSmallN) run in one CTA with shared-memory histograms;
-// larger inputs use a grid of CTAs per pass with global integer histograms.
+// Up to kSmallN positions run in one CTA that keeps the keys in shared
+// memory.  Larger inputs take one grid launch per pass after a zeroing
+// launch; within a pass every CTA adds its shared-memory histogram to a
+// global one and the last CTA to finish (a ticket counter) chooses the next
+// digits, so no separate selection launch is needed.  The shard protocol
+// (kld_reduce_shard_step) keeps four 8-bit passes, whose 16 KB histograms are
+// what the shards exchange.
 #include <math_constants.h>
+
+#include <mutex>
 
 #include "kld_common.cuh"
 #include "launch.h"
@@ -23,14 +33,31 @@ namespace kld {
 namespace {
 
 constexpr int kMaxTargets = 2 * KLD_MAX_QUANTILES;
+constexpr int kBatch = 8;                // positions a thread loads before using any
+
+// kld_reduce_stats: digits of 12, 10, 10 bits
+constexpr int kTopBits = 12;
+constexpr int kTopBins = 1 << kTopBits;  // first-pass histogram (no prefix yet)
+constexpr int kLowBits = 10;
+constexpr int kLowBins = 1 << kLowBits;  // later passes: one row per distinct prefix
+constexpr int kLowHistWords = kMaxTargets * kLowBins;
+constexpr int64_t kSmallN = 8192;
+
+// shard protocol: four 8-bit passes
 constexpr int kBins = 256;
 constexpr int kPasses = 4;
-constexpr int64_t kSmallN = 65536;
 constexpr int kBigThreads = 256;
 constexpr int kMaxBigBlocks = 1024;
-constexpr int kSmallThreads = 512;
 
-struct Partial {  // per-CTA sums of the first pass
+// Sums of a set of positions.  Counts fit 32 bits: n <= INT32_MAX.
+struct Sums {
+  double kl, nll_r, nll_c;
+  unsigned n, n_nan, agree;
+  unsigned exceed[KLD_MAX_THRESHOLDS];
+};
+
+// The shard block's sums: 64-bit counts, as shards' counts add up.
+struct Partial {
   double kl, nll_r, nll_c;
   long long n, n_nan, agree;
   long long exceed[KLD_MAX_THRESHOLDS];
@@ -49,10 +76,10 @@ struct ReduceParams {
   double q[KLD_MAX_QUANTILES];
   float thr[KLD_MAX_THRESHOLDS];
   kld_stats* out;
-  unsigned* hist;     // [kPasses][kMaxTargets][kBins]: the histograms of all positions
-  Partial* partials;  // [gridDim of pass 0]
+  unsigned* hist;     // shard protocol: [kPasses][kMaxTargets][kBins], the histograms of all positions
+  Partial* partials;  // shard protocol: [gridDim of pass 0]
   int32_t* dev_status;
-  unsigned* hist_out; // where a pass adds its histogram (null: hist's own slot for the pass)
+  unsigned* hist_out; // shard protocol: where a pass adds its histogram
 };
 
 __device__ __forceinline__ uint32_t f2key(float f) {
@@ -65,23 +92,21 @@ __device__ __forceinline__ float key2f(uint32_t k) {
   const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
   return __uint_as_float(u);
 }
+// Key 0 is never the key of a non-NaN value (the least, -inf, maps to
+// 0x007fffff), so 0 marks "not scored" wherever keys are stored.
 
-// Per-target radix-select state, identical in every thread that derives it.
+// ------------------------------------------------------------ radix select
+
+// Per-target radix-select state, identical in every thread that reads it.
 struct Select {
   int nt;                      // number of target ranks
+  int nu;                      // number of distinct prefixes
   long long n;                 // scored count
   uint32_t prefix[kMaxTargets];
   long long rem[kMaxTargets];  // rank within the current prefix group
-  int uslot[kMaxTargets];      // index of the target's prefix among the unique ones
+  int uslot[kMaxTargets];      // index of the target's prefix among the distinct ones
   uint32_t uprefix[kMaxTargets];
-  int nu;
 };
-
-__device__ __forceinline__ bool scored(const ReduceParams& p, long long i, float& v) {
-  if (p.mask && !p.mask[i]) return false;
-  v = p.kl[i];
-  return !(v != v);
-}
 
 // Targets from the scored count: for every quantile, the lower and upper
 // order statistic ranks of linear interpolation at h = (n - 1) q.  Thread 0.
@@ -100,7 +125,7 @@ __device__ void select_init(Select& s, const ReduceParams& p, long long n) {
   for (int t = 0; t < s.nt; ++t) s.prefix[t] = 0u;
 }
 
-// Group targets by prefix (warp 0): uslot[t] indexes uprefix[] of unique
+// Group targets by prefix (warp 0): uslot[t] indexes uprefix[] of distinct
 // prefixes, numbered in order of their first target.  Call from every thread.
 __device__ void select_unique(Select& s) {
   if (threadIdx.x < 32) {
@@ -120,38 +145,89 @@ __device__ void select_unique(Select& s) {
   __syncthreads();
 }
 
-// Advance every target by one 8-bit digit using histogram h[u][bin]: warp w
-// takes targets w, w + warps, ...  Lane l holds bins 8l .. 8l+7; a warp scan
-// of the lane totals finds the bin holding the target rank.  Call from every
-// thread; regroups the prefixes afterwards.
-__device__ void select_step(Select& s, const unsigned* h) {
+__device__ __forceinline__ unsigned warp_exclusive_scan(unsigned x, int lane) {
+  unsigned inc = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned o = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += o;
+  }
+  return inc - x;
+}
+
+// Advance every target by one digit of kDigitBits bits from histogram rows
+// h[u * row_stride + bin] (u: the target's prefix slot).  Warp w takes
+// targets w, w + warps, ...  Lane l sums a run of consecutive bins and a
+// warp scan of the run totals finds the run holding the target rank; for
+// digits wider than 8 bits a second scan over that run's 32 sub-runs
+// narrows it to at most 4 bins.  The last bins are walked in registers.
+// Call from every thread; regroups the prefixes.
+template <int kDigitBits>
+__device__ void select_step(Select& s, const unsigned* h, int row_stride) {
+  constexpr int kPer = (1 << kDigitBits) / 32;      // bins per lane, first level
+  constexpr bool kTwoLevel = kPer > 8;
+  constexpr int kSub = kTwoLevel ? kPer / 32 : kPer;  // bins a lane walks
+  static_assert(kPer % 4 == 0 && (kSub == 1 || kSub % 4 == 0), "bins are read as 16-byte vectors");
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int t = w; t < s.nt; t += nw) {
-    const unsigned* row = h + s.uslot[t] * kBins + lane * 8;
-    unsigned c[8];
+    const unsigned* row = h + s.uslot[t] * row_stride;
+    const unsigned rem = (unsigned)s.rem[t];
+    unsigned c[kSub];
     unsigned run = 0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      run += row[k];
-      c[k] = run;  // inclusive prefix within the lane
+    for (int k = 0; k < kPer; k += 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(row + lane * kPer + k);
+      if constexpr (!kTwoLevel) {
+        c[k] = v.x;
+        c[k + 1] = v.y;
+        c[k + 2] = v.z;
+        c[k + 3] = v.w;
+      }
+      run += v.x + v.y + v.z + v.w;
     }
-    unsigned base = run;  // inclusive warp scan of lane totals
+    const unsigned excl = warp_exclusive_scan(run, lane);
+    int L = __ffs(__ballot_sync(0xffffffffu, excl + run > rem)) - 1;
+    if (L < 0) L = 31;
+    unsigned before = __shfl_sync(0xffffffffu, excl, L);
+    int first = L * kPer;  // first bin of the run holding the target
+    if constexpr (kTwoLevel) {
+      const unsigned* sub = row + first + lane * kSub;
+      unsigned r2 = 0;
+      if constexpr (kSub == 1) {
+        c[0] = sub[0];
+        r2 = c[0];
+      } else {
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const unsigned o = __shfl_up_sync(0xffffffffu, base, off);
-      if (lane >= off) base += o;
+        for (int k = 0; k < kSub; k += 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sub + k);
+          c[k] = v.x;
+          c[k + 1] = v.y;
+          c[k + 2] = v.z;
+          c[k + 3] = v.w;
+          r2 += v.x + v.y + v.z + v.w;
+        }
+      }
+      const unsigned e2 = warp_exclusive_scan(r2, lane);
+      L = __ffs(__ballot_sync(0xffffffffu, before + e2 + r2 > rem)) - 1;
+      if (L < 0) L = 31;
+      before += __shfl_sync(0xffffffffu, e2, L);
+      first += L * kSub;
     }
-    base -= run;  // exclusive
-    const unsigned long long rem = (unsigned long long)s.rem[t];
-    const unsigned hit = __ballot_sync(0xffffffffu, (unsigned long long)base + run > rem);
-    const int L = hit ? __ffs(hit) - 1 : 31;
-    if (lane == L) {
-      int k = 7;
-      for (int j = 7; j >= 0; --j)
-        if ((unsigned long long)base + c[j] > rem) k = j;
-      const unsigned before = base + (k ? c[k - 1] : 0u);
-      s.rem[t] = (long long)(rem - before);
-      s.prefix[t] = (s.prefix[t] << 8) | (uint32_t)(8 * L + k);
+    // lane L holds the final bins: walk them
+    unsigned acc = before;
+    int k = 0;
+#pragma unroll
+    for (int j = 0; j < kSub - 1; ++j) {
+      if (k == j && acc + c[j] <= rem) {
+        acc += c[j];
+        k = j + 1;
+      }
+    }
+    k = __shfl_sync(0xffffffffu, k, L);
+    acc = __shfl_sync(0xffffffffu, acc, L);
+    if (lane == 0) {
+      s.rem[t] = (long long)(rem - acc);
+      s.prefix[t] = (s.prefix[t] << kDigitBits) | (uint32_t)(first + k);
     }
     __syncwarp();
   }
@@ -159,48 +235,47 @@ __device__ void select_step(Select& s, const unsigned* h) {
   select_unique(s);
 }
 
-// One histogram pass over [begin, end) with stride `stride`, adding into the
-// shared-memory histogram sh[u][bin] for elements whose key matches a unique
-// prefix of this pass.  Pass 0 histograms every scored element.
-__device__ __forceinline__ void hist_pass(const ReduceParams& p, const Select& s, int pass,
-                                          long long begin, long long stride, unsigned* sh) {
-  const int shift = 24 - 8 * pass;
-  for (long long i = begin; i < p.n; i += stride) {
-    float v;
-    if (!scored(p, i, v)) continue;
-    const uint32_t key = f2key(v);
-    const uint32_t digit = (key >> shift) & 0xffu;
-    if (pass == 0) {
-      atomicAdd(&sh[digit], 1u);
-    } else {
-      const uint32_t pre = key >> (shift + 8);
-      for (int u = 0; u < s.nu; ++u) {
-        if (s.uprefix[u] == pre) {
-          atomicAdd(&sh[u * kBins + digit], 1u);
-          break;
-        }
-      }
-    }
-  }
+// A pass's distinct prefixes in registers; unused slots hold a value no
+// prefix takes (prefixes have at most 24 bits).
+struct Prefixes {
+  uint32_t v[kMaxTargets];
+};
+
+__device__ __forceinline__ Prefixes load_prefixes(const Select& s) {
+  Prefixes r;
+#pragma unroll
+  for (int u = 0; u < kMaxTargets; ++u) r.v[u] = (u < s.nu) ? s.uprefix[u] : 0xffffffffu;
+  return r;
 }
 
-// Pass-0 sums of one thread (fixed stride order).  Positions are taken four
-// at a time with every load issued before any is used, so one memory latency
-// covers the batch.
-__device__ __forceinline__ void thread_sums(const ReduceParams& p, long long begin, long long stride,
-                                            Partial& acc) {
-  constexpr int B = 4;
-  acc.kl = acc.nll_r = acc.nll_c = 0.0;
-  acc.n = acc.n_nan = acc.agree = 0;
-  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) acc.exceed[j] = 0;
-  for (long long i0 = begin; i0 < p.n; i0 += B * stride) {
-    float v[B], lr[B], lc[B];
-    int ra[B], ca[B];
-    bool in[B];
+// The slot of the distinct prefix `pre` is, or -1.
+__device__ __forceinline__ int prefix_slot(const Prefixes& P, uint32_t pre) {
+  int u = -1;
 #pragma unroll
-    for (int b = 0; b < B; ++b) {
+  for (int j = kMaxTargets - 1; j >= 0; --j)
+    if (P.v[j] == pre) u = j;
+  return u;
+}
+
+// ---------------------------------------------------------------- sums
+
+__device__ __forceinline__ bool has_agreement(const ReduceParams& p) { return p.ra != nullptr || p.top1 != nullptr; }
+
+// Positions first, first + stride, ... below end, kBatch at a time with
+// every load of a batch issued before any is used.  Adds scored positions
+// to `acc` and hands every position's index and key (0: not scored) to
+// on_pos.
+template <class F>
+__device__ __forceinline__ void scan_positions(const ReduceParams& p, long long first, long long stride,
+                                               long long end, Sums& acc, F&& on_pos) {
+  for (long long i0 = first; i0 < end; i0 += kBatch * stride) {
+    float v[kBatch], lr[kBatch], lc[kBatch];
+    int ra[kBatch], ca[kBatch];
+    bool in[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
       const long long i = i0 + b * stride;
-      in[b] = i < p.n && (!p.mask || p.mask[i]);
+      in[b] = i < end && (!p.mask || p.mask[i]);
       v[b] = in[b] ? p.kl[i] : 0.f;
       lr[b] = (in[b] && p.lpr) ? p.lpr[i] : 0.f;
       lc[b] = (in[b] && p.lpc) ? p.lpc[i] : 0.f;
@@ -209,89 +284,113 @@ __device__ __forceinline__ void thread_sums(const ReduceParams& p, long long beg
       if (in[b] && !p.ra && p.top1) ra[b] = ca[b] = p.top1[i] ? 0 : -1;
     }
 #pragma unroll
-    for (int b = 0; b < B; ++b) {
-      if (!in[b]) continue;
-      if (v[b] != v[b]) {
-        ++acc.n_nan;
-        continue;
+    for (int b = 0; b < kBatch; ++b) {
+      const long long i = i0 + b * stride;
+      if (i >= end) break;
+      uint32_t key = 0u;
+      if (in[b]) {
+        if (v[b] != v[b]) {
+          ++acc.n_nan;
+        } else {
+          ++acc.n;
+          acc.kl += (double)v[b];
+          acc.nll_r -= (double)lr[b];
+          acc.nll_c -= (double)lc[b];
+          acc.agree += (ra[b] >= 0 && ra[b] == ca[b]) ? 1u : 0u;
+#pragma unroll
+          for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j)
+            if (j < p.nt) acc.exceed[j] += (v[b] > p.thr[j]) ? 1u : 0u;
+          key = f2key(v[b]);
+        }
       }
-      ++acc.n;
-      acc.kl += (double)v[b];
-      acc.nll_r -= (double)lr[b];
-      acc.nll_c -= (double)lc[b];
-      acc.agree += (ra[b] >= 0 && ra[b] == ca[b]) ? 1 : 0;
-      for (int j = 0; j < p.nt; ++j) acc.exceed[j] += (v[b] > p.thr[j]) ? 1 : 0;
+      on_pos(i, key);
     }
   }
 }
 
-__device__ __forceinline__ void partial_add(Partial& a, const Partial& b) {
+// Keys only (kBatch at a time), for passes after the first: on_key(key)
+// for the scored positions among first, first + stride, ... below end.
+template <class F>
+__device__ __forceinline__ void scan_keys(const ReduceParams& p, long long first, long long stride, long long end,
+                                          F&& on_key) {
+  for (long long i0 = first; i0 < end; i0 += kBatch * stride) {
+    float v[kBatch];
+    bool in[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const long long i = i0 + b * stride;
+      in[b] = i < end && (!p.mask || p.mask[i]);
+      v[b] = in[b] ? p.kl[i] : 0.f;
+    }
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      if (in[b] && !(v[b] != v[b])) on_key(f2key(v[b]));
+  }
+}
+
+__device__ __forceinline__ void sums_add(Sums& a, const Sums& b, int nt) {
   a.kl += b.kl;
   a.nll_r += b.nll_r;
   a.nll_c += b.nll_c;
   a.n += b.n;
   a.n_nan += b.n_nan;
   a.agree += b.agree;
-  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) a.exceed[j] += b.exceed[j];
-}
-
-__device__ __forceinline__ Partial shfl_down_partial(const Partial& a, int off, int nt) {
-  Partial o;
-  o.kl = __shfl_down_sync(0xffffffffu, a.kl, off);
-  o.nll_r = __shfl_down_sync(0xffffffffu, a.nll_r, off);
-  o.nll_c = __shfl_down_sync(0xffffffffu, a.nll_c, off);
-  o.n = __shfl_down_sync(0xffffffffu, a.n, off);
-  o.n_nan = __shfl_down_sync(0xffffffffu, a.n_nan, off);
-  o.agree = __shfl_down_sync(0xffffffffu, a.agree, off);
+#pragma unroll
   for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j)
-    o.exceed[j] = (j < nt) ? __shfl_down_sync(0xffffffffu, a.exceed[j], off) : 0;
-  return o;
+    if (j < nt) a.exceed[j] += b.exceed[j];
 }
 
-// Fixed-order CTA reduction of per-thread partials: a butterfly in every
-// warp, then warp 0 does the same over the warp totals.  Result valid in
-// thread 0.  Call from every thread.
-__device__ void block_sum(Partial& acc, Partial* sh_warp, int nt) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+// Fixed-order warp sum: f64 by a shuffle tree (result in lane 0), counts
+// by redux (exact, in every lane).
+__device__ __forceinline__ void warp_sums(Sums& a, int nt) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
-    const Partial o = shfl_down_partial(acc, off, nt);
-    if (lane < off) partial_add(acc, o);
+    a.kl += __shfl_down_sync(0xffffffffu, a.kl, off);
+    a.nll_r += __shfl_down_sync(0xffffffffu, a.nll_r, off);
+    a.nll_c += __shfl_down_sync(0xffffffffu, a.nll_c, off);
   }
-  if (lane == 0) sh_warp[w] = acc;
-  __syncthreads();
-  if (w == 0) {
-    Partial t;
-    if (lane < nw) {
-      t = sh_warp[lane];
-    } else {
-      t.kl = t.nll_r = t.nll_c = 0.0;
-      t.n = t.n_nan = t.agree = 0;
-      for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) t.exceed[j] = 0;
-    }
+  a.n = __reduce_add_sync(0xffffffffu, a.n);
+  a.n_nan = __reduce_add_sync(0xffffffffu, a.n_nan);
+  a.agree = __reduce_add_sync(0xffffffffu, a.agree);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const Partial o = shfl_down_partial(t, off, nt);
-      if (lane < off) partial_add(t, o);
-    }
-    if (lane == 0) acc = t;
-  }
-  __syncthreads();
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j)
+    if (j < nt) a.exceed[j] = __reduce_add_sync(0xffffffffu, a.exceed[j]);
 }
 
-__device__ void write_stats(const ReduceParams& p, const Partial& tot, const Select& s) {
+// Sum of every thread's `a` in a fixed order (warps, then the warp totals
+// in warp order), returned to every thread.  sh holds 32 entries.  Call
+// from every thread.
+__device__ Sums block_sums(Sums a, Sums* sh, int nt) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  warp_sums(a, nt);
+  if (lane == 0) sh[w] = a;
+  __syncthreads();
+  if (w == 0) {
+    Sums t{};
+    if (lane < nw) t = sh[lane];
+    warp_sums(t, nt);
+    __syncwarp();
+    if (lane == 0) sh[0] = t;
+  }
+  __syncthreads();
+  const Sums r = sh[0];
+  __syncthreads();
+  return r;
+}
+
+__device__ void write_stats(const ReduceParams& p, long long n, long long n_nan, long long agree, double kl,
+                            double nll_r, double nll_c, const long long* exceed, const Select& s) {
   kld_stats st;
-  const long long n = tot.n;
   const double nan = CUDART_NAN;
   st.n = n;
-  st.n_nan = tot.n_nan;
-  const bool have_agree = p.ra != nullptr || p.top1 != nullptr;
-  st.top1_agree = have_agree ? tot.agree : -1;
-  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) st.exceed[j] = (j < p.nt) ? tot.exceed[j] : 0;
-  st.mean_kl = n ? tot.kl / (double)n : nan;
-  st.top1_rate = (have_agree && n) ? (double)tot.agree / (double)n : nan;
-  st.ref_mean_nll = (p.lpr && n) ? tot.nll_r / (double)n : nan;
-  st.cand_mean_nll = (p.lpc && n) ? tot.nll_c / (double)n : nan;
+  st.n_nan = n_nan;
+  const bool have_agree = has_agreement(p);
+  st.top1_agree = have_agree ? agree : -1;
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) st.exceed[j] = (j < p.nt) ? exceed[j] : 0;
+  st.mean_kl = n ? kl / (double)n : nan;
+  st.top1_rate = (have_agree && n) ? (double)agree / (double)n : nan;
+  st.ref_mean_nll = (p.lpr && n) ? nll_r / (double)n : nan;
+  st.cand_mean_nll = (p.lpc && n) ? nll_c / (double)n : nan;
   st.ref_ppl = exp(st.ref_mean_nll);
   st.cand_ppl = exp(st.cand_mean_nll);
   st.ppl_ratio = st.cand_ppl / st.ref_ppl;
@@ -313,72 +412,363 @@ __device__ void write_stats(const ReduceParams& p, const Partial& tot, const Sel
   *p.out = st;
 }
 
-// ---------------------------------------------------------------- one CTA
+// ---------------------------------------------------------------- targets
 
-// Up to kCacheN scored keys stay in shared memory across the passes; key 0
-// marks a position that is not scored (only NaN bit patterns map to 0).
-constexpr int kCacheN = 6144;
-
-__global__ void __launch_bounds__(kSmallThreads) reduce_small_kernel(const ReduceParams p) {
-  __shared__ unsigned sh[kMaxTargets * kBins];
-  __shared__ uint32_t keys[kCacheN];
-  __shared__ Partial sh_warp[kSmallThreads / 32];
-  __shared__ Select sel;
-
-  wait_prior_grid();
-  const bool cached = p.n <= kCacheN;
-  Partial acc;
-  thread_sums(p, threadIdx.x, blockDim.x, acc);
-  if (cached) {
-    for (int i = threadIdx.x; i < (int)p.n; i += blockDim.x) {
-      float v;
-      keys[i] = scored(p, i, v) ? f2key(v) : 0u;
+// The statistics from the totals (doubles valid in lane 0, counts in every
+// lane) and the targets' order statistics as keys; warp 0, fields written
+// by several lanes side by side.
+__device__ void write_stats_warp(const ReduceParams& p, const Sums& t, const uint32_t* target_key, int lane) {
+  kld_stats* o = p.out;
+  const double kl = __shfl_sync(0xffffffffu, t.kl, 0);
+  const double nll_r = __shfl_sync(0xffffffffu, t.nll_r, 0);
+  const double nll_c = __shfl_sync(0xffffffffu, t.nll_c, 0);
+  const long long n = t.n;
+  const double nan = CUDART_NAN;
+  const double ref_nll = (p.lpr && n) ? nll_r / (double)n : nan;
+  const double cand_nll = (p.lpc && n) ? nll_c / (double)n : nan;
+  double ppl = nan;
+  if (lane == 1) ppl = exp(ref_nll);
+  if (lane == 2) ppl = exp(cand_nll);
+  const double ref_ppl = __shfl_sync(0xffffffffu, ppl, 1);
+  const double cand_ppl = __shfl_sync(0xffffffffu, ppl, 2);
+  if (lane == 0) {
+    const bool have_agree = has_agreement(p);
+    o->n = n;
+    o->n_nan = t.n_nan;
+    o->top1_agree = have_agree ? (long long)t.agree : -1;
+    for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) o->exceed[j] = (j < p.nt) ? (long long)t.exceed[j] : 0;
+    o->mean_kl = n ? kl / (double)n : nan;
+    o->top1_rate = (have_agree && n) ? (double)t.agree / (double)n : nan;
+    o->ref_mean_nll = ref_nll;
+    o->cand_mean_nll = cand_nll;
+    o->nq = p.nq;
+    o->nt = p.nt;
+  } else if (lane == 1) {
+    o->ref_ppl = ref_ppl;
+  } else if (lane == 2) {
+    o->cand_ppl = cand_ppl;
+  } else if (lane == 3) {
+    o->ppl_ratio = cand_ppl / ref_ppl;
+  } else if (lane >= 8 && lane < 8 + KLD_MAX_QUANTILES) {
+    const int i = lane - 8;
+    if (i < p.nq && n > 0) {
+      const float lo = key2f(target_key[2 * i]);
+      const float hi = key2f(target_key[2 * i + 1]);
+      const double h = __dmul_rn((double)(n - 1), p.q[i]);
+      const double frac = __dsub_rn(h, floor(h));
+      o->q_lo[i] = lo;
+      o->q_hi[i] = hi;
+      o->q_value[i] = __dadd_rn((double)lo, __dmul_rn(__dsub_rn((double)hi, (double)lo), frac));
+    } else {
+      o->q_lo[i] = o->q_hi[i] = CUDART_NAN_F;
+      o->q_value[i] = nan;
     }
   }
-  block_sum(acc, sh_warp, p.nt);
-  if (threadIdx.x == 0) select_init(sel, p, acc.n);
+}
+
+// ---------------------------------------------------------------- one CTA
+
+// Histogram of one select pass over keys[0 .. m) in shared memory (0 = not
+// scored): the digit at `shift` of every key (kTop), or of every key whose
+// bits above the digit extend a target prefix, in the row of that prefix.
+// Keys are loaded four at a time before any is counted.
+template <int kDigitBits, bool kTop>
+__device__ __forceinline__ void hist_keys(const uint32_t* keys, int m, const Select& sel, int shift, unsigned* hist) {
+  constexpr int B = 4;
+  Prefixes P;
+  if constexpr (!kTop) P = load_prefixes(sel);
+  for (int i0 = threadIdx.x; i0 < m; i0 += B * blockDim.x) {
+    uint32_t k[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int i = i0 + b * blockDim.x;
+      k[b] = (i < m) ? keys[i] : 0u;
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      if (!k[b]) continue;
+      int u = 0;
+      if constexpr (!kTop) u = prefix_slot(P, k[b] >> (shift + kDigitBits));
+      if (u >= 0) atomicAdd(&hist[(u << kDigitBits) | ((k[b] >> shift) & ((1u << kDigitBits) - 1u))], 1u);
+    }
+  }
+}
+
+constexpr int kSmallThreads = 512;
+
+// All of kld_reduce_stats for n <= kSmallN in one CTA: every thread sums
+// its positions and keeps their keys in shared memory; four 8-bit select
+// passes follow, each one histogram over all targets' prefixes; warp 0
+// writes the statistics.
+__global__ void __launch_bounds__(kSmallThreads) reduce_small_kernel(const ReduceParams p) {
+  extern __shared__ __align__(16) uint32_t keys[];  // p.n
+  __shared__ __align__(16) unsigned hist[kMaxTargets * kBins];
+  __shared__ Sums sh[32];
+  __shared__ Select sel;
+  static_assert(kSmallThreads / 32 <= kMaxTargets, "one first-pass histogram row per warp");
+  for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) hist[i] = 0u;
+  wait_prior_grid();
+  Sums acc{};
+  scan_positions(p, threadIdx.x, blockDim.x, p.n, acc, [&](long long i, uint32_t key) { keys[i] = key; });
+  const Sums tot = block_sums(acc, sh, p.nt);  // its barriers publish keys[] and the cleared histogram
+  if (threadIdx.x == 0) select_init(sel, p, tot.n);
   __syncthreads();
   select_unique(sel);
-  for (int pass = 0; pass < kPasses; ++pass) {
-    for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) sh[i] = 0u;
+  const int m = (int)p.n;
+  if (sel.nt > 0) {
+    // first pass: every warp counts into its own row (the top bytes of KL
+    // values fall in a handful of bins), then the rows are added up
+    unsigned* row = hist + (threadIdx.x >> 5) * kBins;
+    for (int i0 = threadIdx.x; i0 < m; i0 += 4 * blockDim.x) {
+      uint32_t k[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) k[b] = (i0 + b * (int)blockDim.x < m) ? keys[i0 + b * blockDim.x] : 0u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        if (k[b]) atomicAdd(&row[k[b] >> 24], 1u);
+    }
+    __syncthreads();
+    unsigned c = 0u;
+    if (threadIdx.x < kBins)
+      for (int r = 0; r < (int)(blockDim.x >> 5); ++r) c += hist[r * kBins + threadIdx.x];
+    __syncthreads();
+    if (threadIdx.x < kBins) hist[threadIdx.x] = c;
+  }
+  __syncthreads();
+  select_step<8>(sel, hist, kBins);
+  for (int pass = 1; pass < kPasses; ++pass) {
+    for (int i = threadIdx.x; i < sel.nu * kBins; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();
+    if (sel.nt > 0) hist_keys<8, false>(keys, m, sel, 24 - 8 * pass, hist);
+    __syncthreads();
+    select_step<8>(sel, hist, kBins);
+  }
+  if (threadIdx.x < 32) write_stats_warp(p, tot, sel.prefix, threadIdx.x);
+}
+
+constexpr size_t kSmallSmemMax = sizeof(uint32_t) * kSmallN;
+
+// ---------------------------------------------------------------- grid
+
+// kld_reduce_stats for n > kSmallN: one cooperative launch (every CTA
+// resident at once) over contiguous chunks of positions, one CTA per SM.
+// Pass 0 sums the chunk, keeps its keys in shared memory (when the chunk
+// fits) and histograms their top 12 bits; passes 1 and 2 histogram the
+// next 10 bits of the keys that extend a target's prefix.  After passes 0
+// and 1 every CTA adds its histogram into global memory and meets the
+// others at a grid barrier (a counter polled with a bounded wait); then
+// each CTA reads the whole histogram and takes the next digits itself, so
+// no CTA waits for another to publish them.  After pass 2 the last CTA to
+// arrive (a ticket) takes the final digits and writes the statistics.
+
+constexpr int kCoopThreads = 512;
+constexpr int kCoopKeys = 32768;  // keys a CTA keeps in shared memory (128 KB)
+constexpr int kMaxCoopGrid = 1024;
+constexpr long long kSpinLimit = 1ll << 21;  // polls before a wait gives up (about a second)
+constexpr size_t kCoopSmem = sizeof(unsigned) * (kLowHistWords + kCoopKeys);
+
+struct CoopWs {
+  unsigned arrive[4];
+  alignas(16) unsigned hist0[kTopBins];
+  alignas(16) unsigned hist1[kLowHistWords];
+  alignas(16) unsigned hist2[kLowHistWords];
+  Sums partials[kMaxCoopGrid];
+};
+
+// Cleared before every cooperative launch: its counters and the first
+// pass's histogram (the later passes' are cleared inside it).
+__global__ void __launch_bounds__(1024) reduce_zero_kernel(CoopWs* g) {
+  wait_prior_grid();
+  if (threadIdx.x < 4) g->arrive[threadIdx.x] = 0u;
+  uint4* h = reinterpret_cast<uint4*>(g->hist0);
+  for (int i = threadIdx.x; i < kTopBins / 4; i += blockDim.x) h[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ Sums load_sums_cg(const Sums* s, int nt) {
+  Sums r{};
+  r.kl = __ldcg(&s->kl);
+  r.nll_r = __ldcg(&s->nll_r);
+  r.nll_c = __ldcg(&s->nll_c);
+  r.n = __ldcg(&s->n);
+  r.n_nan = __ldcg(&s->n_nan);
+  r.agree = __ldcg(&s->agree);
+#pragma unroll
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j)
+    if (j < nt) r.exceed[j] = __ldcg(&s->exceed[j]);
+  return r;
+}
+
+// Adds this CTA's histogram (`words` bins) to gh and counts the CTA in at
+// `counter`, every thread's global writes fenced first.  Call from every
+// thread; returns the counter's value before this CTA's arrival (thread 0).
+__device__ unsigned flush_and_arrive(const unsigned* sh_hist, unsigned* gh, int words, unsigned* counter,
+                                     unsigned* sh_ticket) {
+  for (int i = threadIdx.x; i < words; i += blockDim.x) {
+    const unsigned c = sh_hist[i];
+    if (c) atomicAdd(&gh[i], c);
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) *sh_ticket = atomicAdd(counter, 1u);
+  __syncthreads();
+  return *sh_ticket;
+}
+
+// Grid barrier after flush_and_arrive: thread 0 polls the counter until
+// every CTA has arrived (bounded; a timeout is recorded as
+// KLD_DEV_TIMEOUT and returns false).  Call from every thread.
+__device__ bool grid_wait(const unsigned* counter, int32_t* dev_status, int* sh_ok) {
+  if (threadIdx.x == 0) {
+    int ok = 0;
+    for (long long it = 0; it < kSpinLimit; ++it) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+      if (v >= gridDim.x) {
+        ok = 1;
+        break;
+      }
+      __nanosleep(32);
+    }
+    if (!ok) set_dev_status(dev_status, 0x4 /* KLD_DEV_TIMEOUT */);
+    *sh_ok = ok;
+  }
+  __syncthreads();
+  return *sh_ok != 0;
+}
+
+__global__ void __launch_bounds__(kCoopThreads, 1) reduce_coop_kernel(const ReduceParams p, CoopWs* g) {
+  extern __shared__ __align__(16) unsigned dsm[];
+  unsigned* hist = dsm;                  // kTopBins, later nu rows of kLowBins
+  uint32_t* keys = dsm + kLowHistWords;  // this CTA's chunk, when it fits
+  __shared__ Sums sh[32];
+  __shared__ Select sel;
+  __shared__ unsigned ticket;
+  __shared__ int ok;
+  __shared__ unsigned n_scored;
+
+  const long long chunk = (p.n + gridDim.x - 1) / gridDim.x;
+  const long long begin = (long long)blockIdx.x * chunk;
+  const long long end = (begin + chunk < p.n) ? begin + chunk : p.n;
+  const int m = (end > begin) ? (int)(end - begin) : 0;
+  const bool cached = chunk <= kCoopKeys;
+
+  for (int i = threadIdx.x; i < kTopBins; i += blockDim.x) hist[i] = 0u;
+  if (threadIdx.x == 0) n_scored = 0u;
+  {  // the later passes' global histograms, cleared across the grid
+    const int vecs = 2 * kLowHistWords / 4;
+    uint4* h12 = reinterpret_cast<uint4*>(g->hist1);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < vecs; i += gridDim.x * blockDim.x)
+      h12[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+
+  // pass 0: sums, keys, top-12-bit histogram
+  Sums acc{};
+  scan_positions(p, begin + threadIdx.x, blockDim.x, end, acc, [&](long long i, uint32_t key) {
+    if (cached) keys[i - begin] = key;
+    else if (key) atomicAdd(&hist[key >> (32 - kTopBits)], 1u);
+  });
+  const Sums cta = block_sums(acc, sh, p.nt);  // its barriers publish keys[] (or complete the histogram)
+  if (threadIdx.x == 0) g->partials[blockIdx.x] = cta;
+  if (cached) {
+    hist_keys<kTopBits, true>(keys, m, sel, 32 - kTopBits, hist);
+    __syncthreads();
+  }
+  flush_and_arrive(hist, g->hist0, kTopBins, &g->arrive[0], &ticket);
+  if (!grid_wait(&g->arrive[0], p.dev_status, &ok)) return;
+  {  // every CTA: the whole first-pass histogram, the scored count, the first digits
+    unsigned c = 0u;
+    for (int i = threadIdx.x; i < kTopBins; i += blockDim.x) {
+      const unsigned v = __ldcg(g->hist0 + i);
+      hist[i] = v;
+      c += v;
+    }
+    c = __reduce_add_sync(0xffffffffu, c);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&n_scored, c);
+    __syncthreads();
+    if (threadIdx.x == 0) select_init(sel, p, (long long)n_scored);
+    __syncthreads();
+    select_unique(sel);
+    select_step<kTopBits>(sel, hist, kTopBins);
+  }
+
+  // passes 1 and 2
+  for (int pass = 1; pass <= 2; ++pass) {
+    const int shift = (pass == 1) ? kLowBits : 0;  // this pass's digit: key bits [shift, shift + 10)
+    const int words = sel.nu * kLowBins;          // nu = 0 when there is no target
+    for (int i = threadIdx.x; i < words; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
     if (sel.nt > 0) {
       if (cached) {
-        const int shift = 24 - 8 * pass;
-        for (int i = threadIdx.x; i < (int)p.n; i += blockDim.x) {
-          const uint32_t key = keys[i];
-          if (key == 0u) continue;
-          const uint32_t digit = (key >> shift) & 0xffu;
-          if (pass == 0) {
-            atomicAdd(&sh[digit], 1u);
-          } else {
-            const uint32_t pre = key >> (shift + 8);
-            for (int u = 0; u < sel.nu; ++u)
-              if (sel.uprefix[u] == pre) {
-                atomicAdd(&sh[u * kBins + digit], 1u);
-                break;
-              }
-          }
-        }
+        hist_keys<kLowBits, false>(keys, m, sel, shift, hist);
       } else {
-        hist_pass(p, sel, pass, threadIdx.x, blockDim.x, sh);
+        const Prefixes P = load_prefixes(sel);
+        scan_keys(p, begin + threadIdx.x, blockDim.x, end, [&](uint32_t k) {
+          const int u = prefix_slot(P, k >> (shift + kLowBits));
+          if (u >= 0) atomicAdd(&hist[u * kLowBins + ((k >> shift) & (kLowBins - 1))], 1u);
+        });
       }
     }
     __syncthreads();
-    select_step(sel, sh);
+    unsigned* gh = (pass == 1) ? g->hist1 : g->hist2;
+    const unsigned before = flush_and_arrive(hist, gh, words, &g->arrive[pass], &ticket);
+    if (pass == 1) {
+      if (!grid_wait(&g->arrive[1], p.dev_status, &ok)) return;
+    } else if (before != gridDim.x - 1) {
+      return;  // not the last CTA of the final pass
+    } else {
+      __threadfence();
+    }
+    for (int i = threadIdx.x; i < words; i += blockDim.x) hist[i] = __ldcg(gh + i);
+    __syncthreads();
+    select_step<kLowBits>(sel, hist, kLowBins);
   }
-  if (threadIdx.x == 0) write_stats(p, acc, sel);
+
+  // the last CTA: all sums in CTA order, then the statistics
+  Sums s{};
+  for (int b = threadIdx.x; b < (int)gridDim.x; b += blockDim.x) sums_add(s, load_sums_cg(&g->partials[b], p.nt), p.nt);
+  const Sums tot = block_sums(s, sh, p.nt);
+  if (threadIdx.x < 32) write_stats_warp(p, tot, sel.prefix, threadIdx.x);
 }
 
-// ---------------------------------------------------------------- many CTAs
+// ---------------------------------------------------------------- shards
+//
+// Statistics over positions held by several shards: every shard runs four
+// 8-bit passes over its own positions, and between passes the shards
+// exchange fixed-size blocks (their pass histogram; at the first pass also
+// their sums).  Each shard adds the gathered blocks up in shard order, so
+// every shard holds the same totals and derives the same select state and
+// statistics.
 
-__global__ void reduce_zero_kernel(unsigned* hist) {
-  wait_prior_grid();
-  for (int i = threadIdx.x; i < kPasses * kMaxTargets * kBins; i += blockDim.x) hist[i] = 0u;
+struct ShardBlock {
+  Partial partial;
+  unsigned hist[kMaxTargets * kBins];
+};
+
+__device__ __forceinline__ Partial to_partial(const Sums& s) {
+  Partial r;
+  r.kl = s.kl;
+  r.nll_r = s.nll_r;
+  r.nll_c = s.nll_c;
+  r.n = s.n;
+  r.n_nan = s.n_nan;
+  r.agree = s.agree;
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) r.exceed[j] = s.exceed[j];
+  return r;
 }
 
-// Rebuild the select state from the histograms of passes < pass.  Call
-// from every thread of the block.
+__device__ __forceinline__ void partial_add(Partial& a, const Partial& b) {
+  a.kl += b.kl;
+  a.nll_r += b.nll_r;
+  a.nll_c += b.nll_c;
+  a.n += b.n;
+  a.n_nan += b.n_nan;
+  a.agree += b.agree;
+  for (int j = 0; j < KLD_MAX_THRESHOLDS; ++j) a.exceed[j] += b.exceed[j];
+}
+
+// Rebuild the select state from the all-shard histograms of passes < pass.
+// Call from every thread of the block.
 __device__ void select_replay(Select& s, const ReduceParams& p, int pass) {
   if (threadIdx.x == 0) {
     long long n = 0;
@@ -387,63 +777,43 @@ __device__ void select_replay(Select& s, const ReduceParams& p, int pass) {
   }
   __syncthreads();
   select_unique(s);
-  for (int q = 0; q < pass; ++q) select_step(s, p.hist + q * kMaxTargets * kBins);
+  for (int q = 0; q < pass; ++q) select_step<8>(s, p.hist + q * kMaxTargets * kBins, kBins);
 }
 
+// One 8-bit pass over this shard's positions, adding its histogram to
+// p.hist_out; pass 0 histograms every scored key and writes the CTA's sums.
 __global__ void __launch_bounds__(kBigThreads) reduce_pass_kernel(const ReduceParams p, int pass) {
-  wait_prior_grid();
-  __shared__ unsigned sh[kMaxTargets * kBins];
+  __shared__ __align__(16) unsigned sh[kMaxTargets * kBins];
   __shared__ Select sel;
-  __shared__ Partial sh_warp[kBigThreads / 32];
+  __shared__ Sums sh_w[32];
   for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) sh[i] = 0u;
-  if (pass == 0) {
-    if (threadIdx.x == 0) {
-      sel.nt = 1;  // histogram every scored element
-      sel.nu = 0;
-    }
-    __syncthreads();
-  } else {
-    select_replay(sel, p, pass);
-  }
+  wait_prior_grid();
+  if (pass > 0) select_replay(sel, p, pass);  // starts with a barrier
+  __syncthreads();
   const long long begin = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long stride = (long long)gridDim.x * blockDim.x;
-  if (sel.nt > 0) hist_pass(p, sel, pass, begin, stride, sh);
+  int used = kBins;
   if (pass == 0) {
-    Partial acc;
-    thread_sums(p, begin, stride, acc);
-    block_sum(acc, sh_warp, p.nt);
-    if (threadIdx.x == 0) p.partials[blockIdx.x] = acc;
+    Sums acc{};
+    scan_positions(p, begin, stride, p.n, acc, [&](long long, uint32_t key) {
+      if (key) atomicAdd(&sh[key >> 24], 1u);
+    });
+    const Sums cta = block_sums(acc, sh_w, p.nt);
+    if (threadIdx.x == 0) p.partials[blockIdx.x] = to_partial(cta);
+  } else {
+    used = sel.nu * kBins;
+    const int shift = 24 - 8 * pass;
+    const Prefixes P = load_prefixes(sel);
+    if (sel.nt > 0)
+      scan_keys(p, begin, stride, p.n, [&](uint32_t key) {
+        const int u = prefix_slot(P, key >> (shift + 8));
+        if (u >= 0) atomicAdd(&sh[u * kBins + ((key >> shift) & 0xffu)], 1u);
+      });
   }
   __syncthreads();
-  unsigned* g = p.hist_out ? p.hist_out : p.hist + pass * kMaxTargets * kBins;
-  const int used = (pass == 0) ? kBins : sel.nu * kBins;
   for (int i = threadIdx.x; i < used; i += blockDim.x)
-    if (sh[i]) atomicAdd(&g[i], sh[i]);
+    if (sh[i]) atomicAdd(&p.hist_out[i], sh[i]);
 }
-
-__global__ void __launch_bounds__(kBigThreads) reduce_final_kernel(const ReduceParams p, int n_partials) {
-  wait_prior_grid();
-  __shared__ Select sel;
-  select_replay(sel, p, kPasses);
-  if (threadIdx.x != 0) return;
-  Partial tot = p.partials[0];
-  for (int b = 1; b < n_partials; ++b) partial_add(tot, p.partials[b]);
-  write_stats(p, tot, sel);
-}
-
-// ---------------------------------------------------------------- shards
-//
-// Statistics over positions held by several shards: every shard runs the
-// passes of the grid path on its own positions, and between passes the
-// shards exchange fixed-size blocks (their pass histogram; at the first
-// pass also their sums).  Each shard adds the gathered blocks up in shard
-// order, so every shard holds the same totals and derives the same select
-// state and statistics.
-
-struct ShardBlock {
-  Partial partial;
-  unsigned hist[kMaxTargets * kBins];
-};
 
 // this shard's block: histogram cleared (before a pass adds into it)
 __global__ void shard_clear_kernel(ShardBlock* blk) {
@@ -451,13 +821,21 @@ __global__ void shard_clear_kernel(ShardBlock* blk) {
   for (int i = threadIdx.x; i < kMaxTargets * kBins; i += blockDim.x) blk->hist[i] = 0u;
 }
 
-// this shard's sums of the first pass: its CTAs' partials in CTA order
-__global__ void shard_fold_kernel(const ReduceParams p, int n_partials, ShardBlock* blk) {
+// this shard's sums of the first pass: its CTAs' partials, each thread
+// adding a strided set in CTA order, then a fixed tree over the threads
+__global__ void __launch_bounds__(kBigThreads) shard_fold_kernel(const ReduceParams p, int n_partials,
+                                                                 ShardBlock* blk) {
+  __shared__ Partial sh[kBigThreads];
   wait_prior_grid();
-  if (threadIdx.x != 0) return;
-  Partial tot = p.partials[0];
-  for (int b = 1; b < n_partials; ++b) partial_add(tot, p.partials[b]);
-  blk->partial = tot;
+  Partial t{};
+  for (int b = threadIdx.x; b < n_partials; b += blockDim.x) partial_add(t, p.partials[b]);
+  sh[threadIdx.x] = t;
+  __syncthreads();
+  for (int half = blockDim.x / 2; half > 0; half >>= 1) {
+    if ((int)threadIdx.x < half) partial_add(sh[threadIdx.x], sh[threadIdx.x + half]);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) blk->partial = sh[0];
 }
 
 // all shards' blocks of pass `pass`: histograms into the totals, in shard
@@ -482,7 +860,10 @@ __global__ void __launch_bounds__(kBigThreads) shard_final_kernel(const ReducePa
   wait_prior_grid();
   __shared__ Select sel;
   select_replay(sel, p, kPasses);
-  if (threadIdx.x == 0) write_stats(p, *total, sel);
+  if (threadIdx.x == 0) {
+    const Partial& t = *total;
+    write_stats(p, t.n, t.n_nan, t.agree, t.kl, t.nll_r, t.nll_c, t.exceed, sel);
+  }
 }
 
 int big_grid(long long n) {
@@ -492,70 +873,119 @@ int big_grid(long long n) {
   return (int)g;
 }
 
-constexpr size_t kHistBytes = sizeof(unsigned) * kPasses * kMaxTargets * kBins;
+constexpr size_t kShardHistBytes = sizeof(unsigned) * kPasses * kMaxTargets * kBins;
+
+ReduceParams make_params(const ReduceArgs& a) {
+  ReduceParams p;
+  p.kl = a.kl;
+  p.ra = a.ref_argmax;
+  p.ca = a.cand_argmax;
+  p.top1 = a.top1;
+  p.lpr = a.ref_lp;
+  p.lpc = a.cand_lp;
+  p.mask = a.mask;
+  p.n = a.n;
+  p.nq = a.nq;
+  p.nt = a.nt;
+  for (int i = 0; i < KLD_MAX_QUANTILES; ++i) p.q[i] = a.quantiles[i];
+  for (int i = 0; i < KLD_MAX_THRESHOLDS; ++i) p.thr[i] = a.thresholds[i];
+  p.out = a.out;
+  p.hist = nullptr;
+  p.partials = nullptr;
+  p.dev_status = a.dev_status;
+  p.hist_out = nullptr;
+  return p;
+}
+
+// Kernels that take more than 48 KB of dynamic shared memory must say so,
+// once per device.
+template <typename Kernel>
+cudaError_t allow_smem(Kernel kernel, size_t bytes, unsigned long long* done_mask) {
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && ((*done_mask >> dev) & 1ull)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev < 64) *done_mask |= 1ull << dev;
+  return e;
+}
+
+// Cooperative grid for n positions: about eight positions per thread, at
+// most as many CTAs as can be resident at once.
+cudaError_t coop_grid(long long n, int* grid) {
+  int dev = 0, sms = 0, occ = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, reduce_coop_kernel, kCoopThreads, kCoopSmem);
+  if (e != cudaSuccess) return e;
+  long long g = (n + kCoopThreads * kBatch - 1) / (kCoopThreads * kBatch);
+  long long cap = (long long)sms * occ;
+  if (cap > kMaxCoopGrid) cap = kMaxCoopGrid;
+  if (cap < 1) return cudaErrorCooperativeLaunchTooLarge;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  *grid = (int)g;
+  return cudaSuccess;
+}
+
+cudaError_t launch_coop(const ReduceParams& p, CoopWs* g, int grid, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kCoopThreads);
+  cfg.dynamicSmemBytes = kCoopSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, reduce_coop_kernel, p, g);
+}
 
 }  // namespace
 
 size_t reduce_workspace_bytes(int64_t n) {
   (void)n;
-  return kHistBytes + sizeof(Partial) * kMaxBigBlocks;
+  return sizeof(CoopWs);
 }
 
 size_t reduce_shard_block_bytes() { return sizeof(ShardBlock); }
 
-// the shard workspace: the grid path's, then the all-shard sums
-size_t reduce_shard_workspace_bytes(int64_t n) { return reduce_workspace_bytes(n) + sizeof(Partial); }
+// the shard workspace: pass histograms, CTA sums, the all-shard sums
+size_t reduce_shard_workspace_bytes(int64_t n) {
+  (void)n;
+  return kShardHistBytes + sizeof(Partial) * (kMaxBigBlocks + 1);
+}
 
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
-  ReduceParams p;
-  p.kl = a.kl;
-  p.ra = a.ref_argmax;
-  p.ca = a.cand_argmax;
-  p.top1 = a.top1;
-  p.lpr = a.ref_lp;
-  p.lpc = a.cand_lp;
-  p.mask = a.mask;
-  p.n = a.n;
-  p.nq = a.nq;
-  p.nt = a.nt;
-  for (int i = 0; i < KLD_MAX_QUANTILES; ++i) p.q[i] = a.quantiles[i];
-  for (int i = 0; i < KLD_MAX_THRESHOLDS; ++i) p.thr[i] = a.thresholds[i];
-  p.out = a.out;
-  p.hist = reinterpret_cast<unsigned*>(a.workspace);
-  p.partials = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes);
-  p.dev_status = a.dev_status;
-  p.hist_out = nullptr;
-
-  if (a.n <= kSmallN) return launch_dependent(reduce_small_kernel, dim3(1), dim3(kSmallThreads), stream, p);
-  const int grid = big_grid(a.n);
-  cudaError_t e = launch_dependent(reduce_zero_kernel, dim3(1), dim3(1024), stream, p.hist);
-  for (int pass = 0; pass < kPasses && e == cudaSuccess; ++pass)
-    e = launch_dependent(reduce_pass_kernel, dim3(grid), dim3(kBigThreads), stream, p, pass);
+  const ReduceParams p = make_params(a);
+  if (a.n <= kSmallN) {
+    static unsigned long long small_ok = 0;
+    cudaError_t e = allow_smem(reduce_small_kernel, kSmallSmemMax, &small_ok);
+    if (e != cudaSuccess) return e;
+    return launch_dependent_smem(reduce_small_kernel, dim3(1), dim3(kSmallThreads), sizeof(uint32_t) * (size_t)a.n,
+                                 stream, p);
+  }
+  static unsigned long long coop_ok = 0;
+  cudaError_t e = allow_smem(reduce_coop_kernel, kCoopSmem, &coop_ok);
+  int grid = 0;
+  if (e == cudaSuccess) e = coop_grid(a.n, &grid);
   if (e != cudaSuccess) return e;
-  return launch_dependent(reduce_final_kernel, dim3(1), dim3(kBigThreads), stream, p, grid);
+  CoopWs* g = reinterpret_cast<CoopWs*>(a.workspace);
+  e = launch_dependent(reduce_zero_kernel, dim3(1), dim3(1024), stream, g);
+  if (e != cudaSuccess) return e;
+  return launch_coop(p, g, grid, stream);
 }
 
 cudaError_t launch_reduce_shard_step(const ReduceArgs& a, int step, int n_shards, const void* gathered,
                                      void* block_out, cudaStream_t stream) {
-  ReduceParams p;
-  p.kl = a.kl;
-  p.ra = a.ref_argmax;
-  p.ca = a.cand_argmax;
-  p.top1 = a.top1;
-  p.lpr = a.ref_lp;
-  p.lpc = a.cand_lp;
-  p.mask = a.mask;
-  p.n = a.n;
-  p.nq = a.nq;
-  p.nt = a.nt;
-  for (int i = 0; i < KLD_MAX_QUANTILES; ++i) p.q[i] = a.quantiles[i];
-  for (int i = 0; i < KLD_MAX_THRESHOLDS; ++i) p.thr[i] = a.thresholds[i];
-  p.out = a.out;
+  ReduceParams p = make_params(a);
   p.hist = reinterpret_cast<unsigned*>(a.workspace);
-  p.partials = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes);
-  p.dev_status = a.dev_status;
-  Partial* total = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kHistBytes +
-                                              sizeof(Partial) * kMaxBigBlocks);
+  p.partials = reinterpret_cast<Partial*>(reinterpret_cast<char*>(a.workspace) + kShardHistBytes);
+  Partial* total = p.partials + kMaxBigBlocks;
   ShardBlock* blk = reinterpret_cast<ShardBlock*>(block_out);
   const ShardBlock* all = reinterpret_cast<const ShardBlock*>(gathered);
   const int grid = big_grid(a.n);
@@ -571,7 +1001,7 @@ cudaError_t launch_reduce_shard_step(const ReduceArgs& a, int step, int n_shards
   p.hist_out = blk->hist;
   e = launch_dependent(reduce_pass_kernel, dim3(grid), dim3(kBigThreads), stream, p, step);
   if (e != cudaSuccess || step != 0) return e;
-  return launch_dependent(shard_fold_kernel, dim3(1), dim3(32), stream, p, grid, blk);
+  return launch_dependent(shard_fold_kernel, dim3(1), dim3(kBigThreads), stream, p, grid, blk);
 }
 
 }  // namespace kld

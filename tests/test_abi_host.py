@@ -219,4 +219,4 @@ def test_reduce_shard_validation(lib):
     assert sh(lib, ws=A16 + 64) == _lib.KLD_ERR_ALIGNMENT
     assert sh(lib, step=last, b=None, out=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
     assert lib.kld_reduce_shard_block_bytes() >= 16 * 256 * 4
-    assert lib.kld_reduce_shard_workspace_size(10) > lib.kld_reduce_workspace_size(10)
+    assert lib.kld_reduce_shard_workspace_size(10) >= 4 * 16 * 256 * 4   # the four passes' all-shard histograms
