@@ -521,3 +521,84 @@ def reduce_stats(kl, ref_argmax=None, cand_argmax=None, top1=None,
         out["ppl_ratio"] = out["cand_ppl"] / out["ref_ppl"]
     out["exceed"] = [int(np.sum(valid & (kl > np.float32(t)))) for t in thresholds]
     return out
+
+
+# ---------------------------------------------------------------------------
+# paired comparison of two candidates (per-context differences, cluster
+# bootstrap)
+# ---------------------------------------------------------------------------
+
+def paired_compare(kl_a, kl_b, ctx_len: int, cluster, resample, quantiles=(0.025, 0.975), mask=None) -> dict:
+    """Paired per-context comparison of two candidates scored against one
+    reference, with a source-cluster bootstrap interval.
+
+    "Qwen3.8-27B fidelity suite v5": the suite's contexts are grouped into
+    source clusters ("What is in here"); two candidates are compared "paired
+    per context" and the difference is reported with a 95 % source-cluster
+    bootstrap interval, together with how many contexts each side wins and
+    the ties (the sibling-rebuild paragraph and the "compare against a
+    published candidate" step).
+
+    Readings (the page gives no formulas):
+    * kl_a, kl_b hold n_ctx contexts of ctx_len positions each, context-major.
+      A position counts when mask is set (all when None) and neither KL is
+      NaN; a context counts when it has at least one such position.
+    * Per counted context c: mean_a(c), mean_b(c) are exact means of its
+      counted positions and d_c = mean_a(c) - mean_b(c).
+    * The reported difference is the mean of d_c over counted contexts;
+      mean_a / mean_b likewise.  a_lower / b_lower / ties count the contexts
+      with d_c < 0 / d_c > 0 / d_c == 0.
+    * Bootstrap replicate r draws the clusters resample[r, 0..C-1] (with
+      repetition; C = number of clusters) and takes every counted context of
+      each drawn cluster: stat_r = sum_j D[j] / sum_j N[j] over the draws,
+      with D[k] = sum of d_c and N[k] = number of counted contexts in cluster
+      k.  A replicate whose draws hold no counted context is NaN and left
+      out.  The interval ends are the linear-interpolation percentiles of the
+      replicates (the convention of reduce_stats).
+    The random draws are an input: the page does not say how they are made.
+    """
+    a = np.asarray(kl_a, dtype=np.float32).reshape(-1, ctx_len)
+    b = np.asarray(kl_b, dtype=np.float32).reshape(-1, ctx_len)
+    n_ctx = a.shape[0]
+    use = ~(np.isnan(a) | np.isnan(b))
+    if mask is not None:
+        use &= np.asarray(mask).astype(bool).reshape(-1, ctx_len)
+    cluster = np.asarray(cluster, dtype=np.int64)
+    n_clusters = int(np.asarray(resample).shape[1]) if np.asarray(resample).ndim == 2 else 0
+    ctx_a, ctx_b, ctx_n = [], [], []
+    for c in range(n_ctx):
+        va = a[c][use[c]].astype(np.float64)
+        vb = b[c][use[c]].astype(np.float64)
+        ctx_n.append(int(va.shape[0]))
+        ctx_a.append(exact_mean(va))
+        ctx_b.append(exact_mean(vb))
+    counted = [c for c in range(n_ctx) if ctx_n[c] > 0]
+    d = {c: ctx_a[c] - ctx_b[c] for c in counted}
+    out = dict(n_ctx=len(counted), n_pos=int(sum(ctx_n)))
+    out["mean_a"] = exact_mean(np.array([ctx_a[c] for c in counted]))
+    out["mean_b"] = exact_mean(np.array([ctx_b[c] for c in counted]))
+    out["diff"] = exact_mean(np.array([d[c] for c in counted]))
+    out["a_lower"] = sum(1 for c in counted if d[c] < 0)
+    out["b_lower"] = sum(1 for c in counted if d[c] > 0)
+    out["ties"] = sum(1 for c in counted if d[c] == 0)
+    D = [[] for _ in range(n_clusters)]
+    N = [0] * n_clusters
+    for c in counted:
+        D[cluster[c]].append(d[c])
+        N[cluster[c]] += 1
+    stats = []
+    for draws in np.asarray(resample, dtype=np.int64):
+        terms, cnt = [], 0
+        for k in draws:
+            terms.extend(D[k])
+            cnt += N[k]
+        stats.append(math.fsum(terms) / cnt if cnt else math.nan)
+    stats = np.array(stats, dtype=np.float64)
+    out["boot"] = stats
+    ok = np.sort(stats[~np.isnan(stats)])
+    out["n_boot"] = int(ok.shape[0])
+    out["ci"] = [quantile_linear(ok, q)[0] for q in quantiles]
+    out["ctx_mean_a"] = np.array(ctx_a)
+    out["ctx_mean_b"] = np.array(ctx_b)
+    out["ctx_n"] = np.array(ctx_n)
+    return out

@@ -521,6 +521,104 @@ def pin_shared_head_matmul(O):
         assert _close(res2["kl"][i], O.full_vocab_row(H[i] @ W.T, (H[i] + 0.1) @ W.T)["kl"], rtol=1e-12)
 
 
+# ---------------------------------------------------------------------------
+# paired comparison
+# ---------------------------------------------------------------------------
+
+def _paired_case(seed, n_ctx=5, L=4, C=3, nan=True):
+    rng = np.random.default_rng(seed)
+    a = rng.lognormal(-6, 1.5, (n_ctx, L)).astype(np.float32)
+    b = (a * rng.uniform(0.7, 1.4, (n_ctx, L))).astype(np.float32)
+    if nan:
+        a[0, 1] = np.nan
+        b[2, 3] = np.nan
+    mask = np.ones((n_ctx, L), dtype=np.uint8)
+    mask[1, 0] = 0
+    cluster = np.array([k % C for k in range(n_ctx)])
+    return a, b, mask, cluster
+
+
+def pin_paired_brute_force(O):
+    # every draw of 3 clusters out of 3 (27 replicates), replicate statistics
+    # from cluster multiplicities in exact rationals
+    a, b, mask, cluster = _paired_case(20)
+    n_ctx, L = a.shape
+    C = 3
+    draws = np.array([[i, j, k] for i in range(C) for j in range(C) for k in range(C)])
+    r = O.paired_compare(a, b, L, cluster, draws, quantiles=(0.1, 0.5, 0.9), mask=mask)
+    d = {}
+    for c in range(n_ctx):
+        keep = [i for i in range(L) if mask[c, i] and not (math.isnan(a[c, i]) or math.isnan(b[c, i]))]
+        if keep:
+            ma = sum(Fraction(float(a[c, i])) for i in keep) / len(keep)
+            mb = sum(Fraction(float(b[c, i])) for i in keep) / len(keep)
+            d[c] = ma - mb
+    assert r["n_ctx"] == len(d)
+    assert _close(r["diff"], float(sum(d.values()) / len(d)), rtol=1e-14, atol=0)
+    assert r["a_lower"] == sum(1 for v in d.values() if v < 0)
+    assert r["b_lower"] == sum(1 for v in d.values() if v > 0)
+    for row, got in zip(draws, r["boot"]):
+        mult = np.bincount(row, minlength=C)
+        num = sum(mult[cluster[c]] * d[c] for c in d)
+        den = sum(mult[cluster[c]] for c in d)
+        assert _close(got, float(num / den), rtol=1e-13, atol=0)
+    want = np.quantile(r["boot"], (0.1, 0.5, 0.9), method="linear")
+    for got, w in zip(r["ci"], want):
+        assert _close(got, float(w), rtol=1e-14, atol=1e-300)
+
+
+def pin_paired_identical(O):
+    a, _, mask, cluster = _paired_case(21, n_ctx=9, L=6)
+    rs = np.random.default_rng(22).integers(0, 3, (40, 3))
+    r = O.paired_compare(a, a.copy(), 6, cluster, rs, mask=mask)
+    assert r["diff"] == 0.0 and r["ties"] == r["n_ctx"] and r["a_lower"] == r["b_lower"] == 0
+    assert r["ci"] == [0.0, 0.0] and r["mean_a"] == r["mean_b"]
+
+
+def pin_paired_constant_shift(O):
+    # values on a 2^-10 grid: every mean and difference is exact
+    rng = np.random.default_rng(23)
+    b = (rng.integers(1, 1000, (8, 8)) / 1024.0).astype(np.float32)
+    a = b + np.float32(2.0 ** -8)
+    rs = rng.integers(0, 4, (30, 4))
+    r = O.paired_compare(a, b, 8, np.arange(8) % 4, rs)
+    assert r["diff"] == 2.0 ** -8 and r["a_lower"] == 0 and r["b_lower"] == 8
+    assert all(v == 2.0 ** -8 for v in r["boot"]) and r["ci"] == [2.0 ** -8, 2.0 ** -8]
+
+
+def pin_paired_each_cluster_once(O):
+    # a replicate that draws every cluster once is the full sample
+    a, b, mask, cluster = _paired_case(24, n_ctx=12, L=5, C=4)
+    rs = np.array([np.random.default_rng(s).permutation(4) for s in range(10)])
+    r = O.paired_compare(a, b, 5, cluster, rs, mask=mask)
+    for v in r["boot"]:
+        assert _close(v, r["diff"], rtol=1e-14, atol=0)
+
+
+def pin_paired_swap(O):
+    # B against A: the difference and the interval change sign, wins swap
+    a, b, mask, cluster = _paired_case(25, n_ctx=10, L=7, C=4)
+    rs = np.random.default_rng(26).integers(0, 4, (101, 4))
+    r = O.paired_compare(a, b, 7, cluster, rs, quantiles=(0.025, 0.975), mask=mask)
+    s2 = O.paired_compare(b, a, 7, cluster, rs, quantiles=(0.025, 0.975), mask=mask)
+    assert s2["diff"] == -r["diff"] and s2["a_lower"] == r["b_lower"] and s2["b_lower"] == r["a_lower"]
+    assert _close(s2["ci"][0], -r["ci"][1], rtol=1e-12, atol=1e-18)
+    assert _close(s2["ci"][1], -r["ci"][0], rtol=1e-12, atol=1e-18)
+
+
+def pin_paired_context_bootstrap(O):
+    # one context per cluster and no dropped positions: an ordinary bootstrap
+    # of the per-context differences
+    rng = np.random.default_rng(27)
+    a = rng.lognormal(-6, 1, (20, 9)).astype(np.float32)
+    b = rng.lognormal(-6, 1, (20, 9)).astype(np.float32)
+    rs = rng.integers(0, 20, (50, 20))
+    r = O.paired_compare(a, b, 9, np.arange(20), rs)
+    d = a.astype(np.float64).mean(axis=1) - b.astype(np.float64).mean(axis=1)
+    for row, got in zip(rs, r["boot"]):
+        assert _close(got, float(np.mean(d[row])), rtol=1e-12, atol=0)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -585,6 +683,13 @@ MUTANTS = [
     ("capture ties keep the higher id", "order = np.lexsort((np.arange(V), -lp))",
      "order = np.lexsort((-np.arange(V), -lp))"),
     ("capture NLL sign", "out[\"nll\"] = -float(lp[int(target)])", "out[\"nll\"] = float(lp[int(target)])"),
+    ("paired difference reversed", "d = {c: ctx_a[c] - ctx_b[c] for c in counted}",
+     "d = {c: ctx_b[c] - ctx_a[c] for c in counted}"),
+    ("replicate divides by clusters drawn", "stats.append(math.fsum(terms) / cnt if cnt else math.nan)",
+     "stats.append(math.fsum(terms) / len(draws) if cnt else math.nan)"),
+    ("paired positions keep B's NaNs", "use = ~(np.isnan(a) | np.isnan(b))", "use = ~np.isnan(a)"),
+    ("ties counted for A", "out[\"a_lower\"] = sum(1 for c in counted if d[c] < 0)",
+     "out[\"a_lower\"] = sum(1 for c in counted if d[c] <= 0)"),
     ("transposed head", "return np.asarray(H, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T",
      "return (np.asarray(W, dtype=np.float64) @ np.asarray(H, dtype=np.float64).T).T[:, ::-1]"),
 ]
