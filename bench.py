@@ -361,7 +361,8 @@ def run_ours(args) -> int:
             line["extra_paths"] = {"topk_tail": measure_topk(args, kq, dev),
                                    "sparse_ref": measure_sparse_ref(args, kq, dev),
                                    "sparse_capture": measure_sparse_capture(args, kq, dev),
-                                   "shared_head": measure_shared_head(args, kq, dev)}
+                                   "shared_head": measure_shared_head(args, kq, dev),
+                                   "paired": measure_paired(args, kq, dev)}
         if world == 1 and not args.no_cpu_baseline:
             rows = list(range(0, n, max(1, n // args.cpu_rows)))[:args.cpu_rows]
             dt = oracle_rows(ref, cand, targets, rows)
@@ -577,6 +578,54 @@ def measure_reduce(args, kq, dev, n=N_ROWS, steps=None) -> dict:
             "launches_per_step": launches_per_step(n) - 2}
 
 
+def measure_paired(args, kq, dev, steps=None) -> dict:
+    """Two candidates compared paired per context over one whole suite
+    (5,120 contexts x 2,047 positions, 842 source clusters) with a
+    10,000-replicate cluster bootstrap: kld_paired_compare.  Inputs are
+    resident; L2 is flushed before every timed call (the inputs are about
+    L2's size)."""
+    import torch
+    from synth import workloads as W
+    d = W.paired_candidates(seed=W.seed_for(8), device=dev)
+    a, b, cl, rs = d["kl_a"], d["kl_b"], d["cluster"], d["resample"]
+    n_ctx, L = a.shape
+    B, C = rs.shape
+    out = torch.empty(144, dtype=torch.uint8, device=dev)
+    boot = torch.empty(B, dtype=torch.float64, device=dev)
+    ws = torch.empty(kq.kld_paired_workspace_size(n_ctx, C, B), dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kq.kld_paired_compare(a, b, cl, rs, (0.025, 0.975), None, boot_stats=boot, out=out, workspace=ws,
+                              dev_status=status, stream=stream, to_host=False)
+
+    steps = steps or max(1, min(args.steps, 100))
+    for _ in range(max(3, args.warmup)):
+        step()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        kev[i][0].record(stream)
+        step()
+        kev[i][1].record(stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item()}"
+    ms = statistics.mean(x.elapsed_time(y) for x, y in kev)
+    # both candidates' KL, the cluster ids and the draws in; replicate statistics out
+    alg = 2 * n_ctx * L * 4 + n_ctx * 4 + B * C * 4 + B * 8
+    peak, _ = measured_peaks()
+    return {"workload": f"paired comparison: {n_ctx} contexts x {L} positions, two candidates, {C} source "
+                        f"clusters, {B}-replicate cluster bootstrap",
+            "value": n_ctx * L / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "step": "kld_paired_compare", "gpu_launches_per_step": 6, "l2": "flushed before every call",
+            "roofline": {"bound": "hbm", "achieved": alg / (ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": alg / (ms / 1e3) / 1e9 / peak,
+                         "kernel": "kld::paired_{ctx,cluster,boot,rank,finish}_kernel", "kernel_ms": ms}}
+
+
 def measured_tensor_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -730,6 +779,8 @@ def main(argv=None) -> int:
                     help="only time the sparse-reference score on ROWS positions (for profiling)")
     ap.add_argument("--profile-capture", type=int, metavar="ROWS",
                     help="only time the sparse capture on ROWS positions (for profiling)")
+    ap.add_argument("--profile-paired", action="store_true",
+                    help="only time the paired comparison of two candidates over one suite (for profiling)")
     ap.add_argument("--profile-reduce", type=int, metavar="POSITIONS",
                     help="only time the statistics of POSITIONS per-position results (for profiling)")
     ap.add_argument("--profile-head", nargs=2, type=int, metavar=("ROWS", "VOCAB"),
@@ -761,6 +812,12 @@ def main(argv=None) -> int:
         kq.load_library()
         print(json.dumps(measure_sparse_capture(args, kq, torch.device("cuda:0"), n_rows=args.profile_capture,
                                                 steps=args.steps)), flush=True)
+        return 0
+    if args.profile_paired:
+        import torch
+        import quantization_fidelity_scoring_b200 as kq
+        kq.load_library()
+        print(json.dumps(measure_paired(args, kq, torch.device("cuda:0"), steps=args.steps)), flush=True)
         return 0
     if args.profile_reduce:
         import torch

@@ -65,7 +65,8 @@ typedef enum kld_status {
 
 /* Bits OR-ed into *dev_status by the kernels. */
 #define KLD_DEV_BAD_TARGET 0x1 /* a target id was outside [0, vocab): that row's target lps are NaN */
-#define KLD_DEV_BAD_ID 0x2     /* a top-k id was outside [0, vocab): that row's KL is NaN */
+#define KLD_DEV_BAD_ID 0x2     /* an id was outside its range: a top-k id (that row's KL is NaN),
+                                  a cluster id or a bootstrap draw (see kld_paired_compare) */
 #define KLD_DEV_TIMEOUT 0x4    /* a bounded wait inside a kernel gave up; outputs are invalid */
 
 typedef enum kld_dtype {
@@ -419,6 +420,78 @@ kld_status kld_reduce_shard_step(int32_t step, int32_t n_shards, const void* gat
                                  const uint8_t* mask, int64_t n, const double* quantiles, int32_t nq,
                                  const float* thresholds, int32_t nt, kld_stats* out, void* workspace,
                                  size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Result of kld_paired_compare, written to DEVICE memory (plain C layout,
+ * 8-byte fields first; sizeof = 144 on LP64).
+ */
+typedef struct kld_paired {
+  int64_t n_ctx;    /* contexts with at least one counted position */
+  int64_t n_pos;    /* counted positions over all contexts */
+  int64_t a_lower;  /* counted contexts whose mean KL is lower for candidate A */
+  int64_t b_lower;  /* ... lower for candidate B */
+  int64_t ties;     /* ... equal */
+  int64_t n_boot;   /* replicates whose draws hold a counted context */
+  double mean_a;    /* mean over counted contexts of A's per-context mean KL */
+  double mean_b;    /* the same for B */
+  double diff;      /* mean over counted contexts of (A's - B's per-context mean) */
+  double ci[KLD_MAX_QUANTILES]; /* bootstrap percentiles of diff, one per quantile */
+  int32_t nq;
+  int32_t pad;
+} kld_paired;
+
+/* Workspace bytes kld_paired_compare needs. */
+size_t kld_paired_workspace_size(int64_t n_ctx, int32_t n_clusters, int32_t n_boot);
+
+/*
+ * kld_paired_compare - two candidates scored against one reference, paired
+ * per context, with a source-cluster bootstrap interval.
+ *
+ * Defines ("Qwen3.8-27B fidelity suite v5": contexts grouped into source
+ * clusters, "What is in here"; the paired comparison of two candidates with
+ * a 95 % source-cluster bootstrap interval and per-context win / tie counts,
+ * in the sibling-rebuild paragraph and the "compare against a published
+ * candidate" step).  The page gives no formulas; this library reads them so:
+ * a position counts when mask[i] != 0 (all when mask is NULL) and neither
+ * KL is NaN; per counted context c, m_A(c) and m_B(c) are the means of its
+ * counted positions and d_c = m_A(c) - m_B(c); diff is the mean of d_c over
+ * counted contexts.  Bootstrap replicate r draws the clusters
+ * resample[r * n_clusters + j], j < n_clusters, and its statistic is
+ *     sum over draws of D[k]  /  sum over draws of N[k]
+ * with D[k] the sum of d_c and N[k] the number of counted contexts of
+ * cluster k (NaN, and left out, when the draws hold no counted context).
+ * ci[i] is the linear-interpolation percentile (h = (n_boot - 1) q, as in
+ * kld_reduce_stats) of the replicate statistics; both order statistics are
+ * exact.  Sums are f64 in a fixed order, so results are reproducible.
+ *
+ * Arguments (pointers DEVICE unless noted):
+ *   kl_a, kl_b     f32 [n_ctx, ctx_len], context-major, per-position KL of
+ *                  candidates A and B against the same reference; 16-byte aligned.
+ *   mask           u8 [n_ctx, ctx_len] or NULL.
+ *   n_ctx          >= 0 contexts; ctx_len >= 1 positions each (n_ctx * ctx_len < 2^40).
+ *   cluster        int32 [n_ctx], each context's cluster in [0, n_clusters);
+ *                  out-of-range ids set KLD_DEV_BAD_ID and drop the context.
+ *   n_clusters     >= 1.
+ *   resample       int32 [n_boot, n_clusters], the draws (the caller's random
+ *                  numbers); out-of-range draws set KLD_DEV_BAD_ID and are skipped.
+ *                  May be NULL when n_boot == 0.
+ *   n_boot         0 .. 2^20 replicates; n_boot * n_clusters < 2^31 (the percentiles
+ *                  compare every pair of replicates: O(n_boot^2) work).
+ *   quantiles      HOST double [nq] in [0, 1]; nq <= KLD_MAX_QUANTILES.
+ *   out            DEVICE kld_paired, 8-byte aligned.
+ *   boot_stats     DEVICE double [n_boot] for the replicate statistics, or NULL.
+ *   workspace      DEVICE, >= kld_paired_workspace_size(...) bytes, 256-byte aligned.
+ *   dev_status     DEVICE int32 or NULL: KLD_DEV_BAD_ID bits are OR-ed in.
+ *   stream         cudaStream_t or NULL.
+ * Ownership: the caller owns every buffer; nothing is kept after the call.
+ * Errors: KLD_ERR_INVALID_ARG for sizes or quantiles out of range or a
+ * missing pointer, KLD_ERR_ALIGNMENT, KLD_ERR_WORKSPACE, KLD_ERR_CUDA.
+ */
+kld_status kld_paired_compare(const float* kl_a, const float* kl_b, const uint8_t* mask, int64_t n_ctx,
+                              int32_t ctx_len, const int32_t* cluster, int32_t n_clusters,
+                              const int32_t* resample, int32_t n_boot, const double* quantiles, int32_t nq,
+                              kld_paired* out, double* boot_stats, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -54,6 +54,26 @@ class KldStats(ctypes.Structure):
 
 assert ctypes.sizeof(KldStats) == 280
 
+class KldPaired(ctypes.Structure):
+    """Mirror of struct kld_paired (include/kld.h)."""
+    _fields_ = [
+        ("n_ctx", ctypes.c_int64),
+        ("n_pos", ctypes.c_int64),
+        ("a_lower", ctypes.c_int64),
+        ("b_lower", ctypes.c_int64),
+        ("ties", ctypes.c_int64),
+        ("n_boot", ctypes.c_int64),
+        ("mean_a", ctypes.c_double),
+        ("mean_b", ctypes.c_double),
+        ("diff", ctypes.c_double),
+        ("ci", ctypes.c_double * KLD_MAX_QUANTILES),
+        ("nq", ctypes.c_int32),
+        ("pad", ctypes.c_int32),
+    ]
+
+
+assert ctypes.sizeof(KldPaired) == 144
+
 KLD_SPARSE_MAX_K = 1024
 KLD_CAPTURE_CANDIDATES = 8192
 KLD_SHARD_STEPS = 5
@@ -88,6 +108,9 @@ PROTOTYPES = {
                                              _P, _P, _SZ, _P, _P]),
     "kld_reduce_stats": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _I32, _P, _P,
                                         _SZ, _P, _P]),
+    "kld_paired_workspace_size": (_SZ, [_I64, _I32, _I32]),
+    "kld_paired_compare": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _P, _I32, _P, _I32, _P, _I32, _P, _P, _P, _SZ,
+                                          _P, _P]),
 }
 
 # exported for tests only (not part of the public header)

@@ -298,6 +298,60 @@ def kld_reduce_stats(kl, ref_argmax=None, cand_argmax=None, top1=None, ref_targe
     return stats_to_dict(raw)
 
 
+def kld_paired_workspace_size(n_ctx: int, n_clusters: int, n_boot: int) -> int:
+    return int(_lib.load().kld_paired_workspace_size(n_ctx, n_clusters, n_boot))
+
+
+def paired_from_device(buf) -> dict:
+    raw = _lib.KldPaired.from_buffer_copy(bytes(buf.cpu().numpy().tobytes()))
+    out = {k: getattr(raw, k) for k in ("n_ctx", "n_pos", "a_lower", "b_lower", "ties", "n_boot",
+                                        "mean_a", "mean_b", "diff", "nq")}
+    out["ci"] = list(raw.ci)[:raw.nq]
+    return out
+
+
+def kld_paired_compare(kl_a, kl_b, cluster, resample, quantiles=(0.025, 0.975), mask=None, *, boot_stats=None,
+                       out=None, workspace=None, dev_status=None, stream=None, to_host: bool = True):
+    """Paired per-context comparison of candidates A and B with a
+    source-cluster bootstrap interval (kld_paired_compare in include/kld.h).
+
+    kl_a, kl_b: f32 [n_ctx, ctx_len]; mask: u8 of the same shape or None;
+    cluster: int32 [n_ctx]; resample: int32 [n_boot, n_clusters], the
+    bootstrap draws.  Returns a dict when to_host, else the device buffer
+    holding the kld_paired struct."""
+    _need_cuda("kl_a", kl_a, torch.float32, 2)
+    _need_cuda("kl_b", kl_b, torch.float32, 2)
+    _need_cuda("mask", mask, torch.uint8, 2)
+    _need_cuda("cluster", cluster, torch.int32, 1)
+    _need_cuda("resample", resample, torch.int32, 2)
+    _need_cuda("boot_stats", boot_stats, torch.float64, 1)
+    n_ctx, ctx_len = kl_a.shape
+    if kl_b.shape != kl_a.shape or (mask is not None and mask.shape != kl_a.shape):
+        raise ValueError("kl_b and mask must have kl_a's shape")
+    if cluster.shape[0] != n_ctx:
+        raise ValueError("cluster needs one id per context")
+    n_boot, n_clusters = resample.shape
+    if boot_stats is not None and boot_stats.shape[0] != n_boot:
+        raise ValueError("boot_stats needs one entry per replicate")
+    for name, t in (("kl_a", kl_a), ("kl_b", kl_b), ("mask", mask), ("resample", resample)):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    lib = _lib.load()
+    dev = kl_a.device
+    if workspace is None:
+        workspace = torch.empty(lib.kld_paired_workspace_size(n_ctx, n_clusters, n_boot), dtype=torch.uint8,
+                                device=dev)
+    if out is None:
+        out = torch.empty(ctypes.sizeof(_lib.KldPaired), dtype=torch.uint8, device=dev)
+    qs = (ctypes.c_double * max(len(quantiles), 1))(*quantiles)
+    st = lib.kld_paired_compare(_ptr(kl_a), _ptr(kl_b), _ptr(mask), n_ctx, ctx_len, _ptr(cluster), n_clusters,
+                                _ptr(resample), n_boot, ctypes.cast(qs, ctypes.c_void_p), len(quantiles),
+                                _ptr(out), _ptr(boot_stats), _ptr(workspace), workspace.numel(),
+                                _ptr(dev_status), _stream_handle(stream))
+    _check(st, "kld_paired_compare")
+    return paired_from_device(out) if to_host else out
+
+
 def kld_reduce_shard_block_bytes() -> int:
     return int(_lib.load().kld_reduce_shard_block_bytes())
 

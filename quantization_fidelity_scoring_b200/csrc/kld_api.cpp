@@ -425,7 +425,49 @@ kld_status kld_reduce_shard_step(int32_t step, int32_t n_shards, const void* gat
                                                    static_cast<cudaStream_t>(stream)));
 }
 
+size_t kld_paired_workspace_size(int64_t n_ctx, int32_t n_clusters, int32_t n_boot) {
+  return kld::paired_workspace_bytes(n_ctx, n_clusters, n_boot);
+}
+
+kld_status kld_paired_compare(const float* kl_a, const float* kl_b, const uint8_t* mask, int64_t n_ctx,
+                              int32_t ctx_len, const int32_t* cluster, int32_t n_clusters,
+                              const int32_t* resample, int32_t n_boot, const double* quantiles, int32_t nq,
+                              kld_paired* out, double* boot_stats, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_status, void* stream) {
+  if (n_ctx < 0 || ctx_len < 1 || n_clusters < 1 || n_boot < 0) return KLD_ERR_INVALID_ARG;
+  if (n_ctx > ((int64_t)1 << 40) / ctx_len || n_ctx > INT32_MAX) return KLD_ERR_INVALID_ARG;
+  if ((int64_t)n_boot * n_clusters >= ((int64_t)1 << 31) || n_boot > (1 << 20)) return KLD_ERR_INVALID_ARG;
+  if (nq < 0 || nq > KLD_MAX_QUANTILES || (nq > 0 && !quantiles)) return KLD_ERR_INVALID_ARG;
+  for (int i = 0; i < nq; ++i)
+    if (!(quantiles[i] >= 0.0 && quantiles[i] <= 1.0)) return KLD_ERR_INVALID_ARG;
+  if (!out || (n_ctx > 0 && (!kl_a || !kl_b || !cluster)) || (n_boot > 0 && !resample)) return KLD_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < kld::paired_workspace_bytes(n_ctx, n_clusters, n_boot))
+    return KLD_ERR_WORKSPACE;
+  if (!aligned(workspace, 256) || !aligned(out, 8) || !aligned(boot_stats, 8) || !aligned(kl_a, 16) ||
+      !aligned(kl_b, 16) || !aligned(cluster, 4) || !aligned(resample, 4) || !aligned(dev_status, 4))
+    return KLD_ERR_ALIGNMENT;
+  kld::PairedArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.kl_a = kl_a;
+  a.kl_b = kl_b;
+  a.mask = mask;
+  a.n_ctx = n_ctx;
+  a.ctx_len = ctx_len;
+  a.cluster = cluster;
+  a.n_clusters = n_clusters;
+  a.resample = resample;
+  a.n_boot = n_boot;
+  a.nq = nq;
+  for (int i = 0; i < nq; ++i) a.quantiles[i] = quantiles[i];
+  a.out = out;
+  a.boot_stats = boot_stats;
+  a.workspace = workspace;
+  a.dev_status = dev_status;
+  return cuda_status(kld::launch_paired(a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 
 static_assert(KLD_SHARD_STEPS == kld::kShardSteps, "shard step count");
 static_assert(sizeof(kld_stats) == 280, "kld_stats layout changed: update the Python mirror");
+static_assert(sizeof(kld_paired) == 144, "kld_paired layout changed: update the Python mirror");

@@ -133,4 +133,24 @@ constexpr int kShardSteps = 5;
 cudaError_t launch_reduce_shard_step(const ReduceArgs& a, int step, int n_shards, const void* gathered,
                                      void* block_out, cudaStream_t stream);
 
+struct PairedArgs {
+  const float* kl_a;
+  const float* kl_b;
+  const uint8_t* mask;
+  int64_t n_ctx;
+  int ctx_len;
+  const int32_t* cluster;
+  int n_clusters;
+  const int32_t* resample;
+  int n_boot;
+  int nq;
+  double quantiles[KLD_MAX_QUANTILES];
+  kld_paired* out;
+  double* boot_stats;  // or null: replicate statistics kept in the workspace
+  void* workspace;     // >= paired_workspace_bytes(n_ctx, n_clusters, n_boot)
+  int32_t* dev_status;
+};
+size_t paired_workspace_bytes(int64_t n_ctx, int32_t n_clusters, int32_t n_boot);
+cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream);
+
 }  // namespace kld

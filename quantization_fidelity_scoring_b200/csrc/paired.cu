@@ -1,0 +1,495 @@
+// Paired comparison of two candidates scored against one reference:
+// per-context means, per-cluster sums, source-cluster bootstrap replicates
+// and exact percentiles of the replicates.
+//
+// "Qwen3.8-27B fidelity suite v5": the suite's contexts come from source
+// clusters ("What is in here"), and two candidates are compared paired per
+// context, reported as a difference with a 95 % source-cluster bootstrap
+// interval and the contexts each side wins (the sibling-rebuild paragraph
+// and the "compare against a published candidate" step).  The page gives
+// no formulas; kld.h states the reading implemented here.
+//
+// Six launches, all deterministic (f64 sums in fixed orders, integer
+// counts):
+//   ctx      one warp per context: sums of A's and B's counted KL (exact in
+//            f64 for ordinary spreads of f32 values), the count, the means
+//            and their difference d_c.
+//   cluster  one warp per cluster: D[k] and N[k] over the contexts in
+//            context order; more blocks sum chunks of 1024 contexts (means,
+//            win and tie counts) for the finish to add in order.
+//   boot     one warp per replicate: the draws' D and N gathered and summed.
+//   count    every replicate counts the replicates below and equal to it,
+//            one tile of 1024 replicates per block row;
+//   pick     the replicate whose rank range holds a target rank is that
+//            order statistic (exact, ties included).
+//   finish   one warp writes the result.
+#include <math_constants.h>
+
+#include "kld_common.cuh"
+#include "launch.h"
+
+namespace kld {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxTargets = 2 * KLD_MAX_QUANTILES;
+constexpr int kRankTile = 1024;  // replicates staged in shared memory at a time
+constexpr int kIdTile = 4096;    // cluster ids staged in shared memory at a time
+constexpr int kBootThreads = 1024;
+constexpr int kBootSmemClusters = 2048;  // clusters whose sums a boot CTA keeps in shared memory
+
+constexpr int kTotChunk = 1024;  // contexts per totals block
+
+// Sums over one chunk of counted contexts.
+struct PairedPart {
+  double sa, sb, sd;  // m_A, m_B, d
+  long long n_used, n_pos, a_lower, b_lower, ties;
+};
+
+struct PairedTotals {
+  unsigned n_valid;  // replicates whose draws hold a counted context
+  unsigned pad;
+  double ostat[kMaxTargets];
+};
+
+struct PairedParams {
+  const float* a;
+  const float* b;
+  const uint8_t* mask;
+  long long n_ctx;
+  int ctx_len;
+  const int32_t* cluster;
+  int n_clusters;
+  const int32_t* resample;
+  int n_boot;
+  int nq;
+  double q[KLD_MAX_QUANTILES];
+  kld_paired* out;
+  double* boot;  // [n_boot] replicate statistics
+  double* ctx_a;
+  double* ctx_b;
+  double* ctx_d;
+  int32_t* ctx_n;
+  double* Dk;
+  long long* Nk;
+  unsigned* less;  // [n_boot] replicates below each replicate
+  unsigned* eq;    // [n_boot] replicates equal to it (itself included)
+  PairedPart* parts;  // [ceil(n_ctx / kTotChunk)]
+  PairedTotals* tot;
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xffffffffu, x, off);
+  return x;  // lane 0
+}
+
+__device__ __forceinline__ long long warp_sum(long long x) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xffffffffu, x, off);
+  return x;  // lane 0
+}
+
+// Rank (0-based, ascending) of target t among n values: quantile t / 2,
+// lower (even t) or upper (odd t) order statistic of linear interpolation.
+__device__ __forceinline__ long long target_rank(const PairedParams& p, long long n, int t) {
+  const double h = __dmul_rn((double)(n - 1), p.q[t >> 1]);
+  long long lo = (long long)floor(h);
+  if (lo > n - 1) lo = n - 1;
+  if (lo < 0) lo = 0;
+  if (!(t & 1)) return lo;
+  return (lo + 1 < n) ? lo + 1 : n - 1;
+}
+
+__device__ __forceinline__ void add_pair(float va, float vb, bool in, double& sa, double& sb, unsigned& cnt) {
+  if (in && !(va != va) && !(vb != vb)) {
+    sa += (double)va;
+    sb += (double)vb;
+    ++cnt;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) paired_ctx_kernel(const PairedParams p) {
+  wait_prior_grid();
+  if (blockIdx.x == 0 && threadIdx.x == 0) p.tot->n_valid = 0u;
+  const int lane = threadIdx.x & 31;
+  const long long c = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (c >= p.n_ctx) return;
+  const long long base = c * p.ctx_len;
+  const float* a = p.a + base;
+  const float* b = p.b + base;
+  const uint8_t* m = p.mask ? p.mask + base : nullptr;
+  const int L = p.ctx_len;
+  double sa = 0.0, sb = 0.0;
+  unsigned cnt = 0;
+  // the row's head up to a 16-byte boundary (both rows share the offset),
+  // then 16-byte vectors, then the tail
+  const int head = (int)((4 - (base & 3)) & 3) < L ? (int)((4 - (base & 3)) & 3) : L;
+  if (lane < head) add_pair(a[lane], b[lane], !m || m[lane], sa, sb, cnt);
+  const int nvec = (L - head) >> 2;
+  const float4* a4 = reinterpret_cast<const float4*>(a + head);
+  const float4* b4 = reinterpret_cast<const float4*>(b + head);
+  constexpr int U = 2;  // vectors in flight per lane and row
+  for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
+    float4 va[U], vb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nvec) {
+        va[u] = __ldcs(a4 + v);
+        vb[u] = __ldcs(b4 + v);
+      } else {
+        va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      const bool live = v < nvec;
+      const int i = head + 4 * v;
+      add_pair(va[u].x, vb[u].x, live && (!m || m[i]), sa, sb, cnt);
+      add_pair(va[u].y, vb[u].y, live && (!m || m[i + 1]), sa, sb, cnt);
+      add_pair(va[u].z, vb[u].z, live && (!m || m[i + 2]), sa, sb, cnt);
+      add_pair(va[u].w, vb[u].w, live && (!m || m[i + 3]), sa, sb, cnt);
+    }
+  }
+  const int tail0 = head + 4 * nvec;
+  if (tail0 + lane < L) add_pair(a[tail0 + lane], b[tail0 + lane], !m || m[tail0 + lane], sa, sb, cnt);
+  sa = warp_sum(sa);
+  sb = warp_sum(sb);
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) {
+    const double ma = cnt ? sa / (double)cnt : 0.0;
+    const double mb = cnt ? sb / (double)cnt : 0.0;
+    p.ctx_n[c] = (int32_t)cnt;
+    p.ctx_a[c] = ma;
+    p.ctx_b[c] = mb;
+    p.ctx_d[c] = ma - mb;
+  }
+}
+
+// Blocks [0, cluster_blocks): one warp per cluster.  Block cluster_blocks:
+// the totals over all counted contexts.
+__global__ void __launch_bounds__(kThreads) paired_cluster_kernel(const PairedParams p, int cluster_blocks) {
+  wait_prior_grid();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if ((int)blockIdx.x < cluster_blocks) {
+    // the block's warps scan the cluster ids from shared memory, a tile at
+    // a time; lane l takes contexts l, l + 32, ... in order
+    __shared__ int32_t ids[kIdTile];
+    const int k = blockIdx.x * kWarps + w;
+    double D = 0.0;
+    long long N = 0;
+    for (long long c0 = 0; c0 < p.n_ctx; c0 += kIdTile) {
+      const int m = (p.n_ctx - c0 < kIdTile) ? (int)(p.n_ctx - c0) : kIdTile;
+      __syncthreads();
+      for (int i = threadIdx.x; i < m; i += blockDim.x) ids[i] = __ldg(p.cluster + c0 + i);
+      __syncthreads();
+      if (k < p.n_clusters) {
+        for (int i = lane; i < m; i += 32) {
+          if (ids[i] == k && p.ctx_n[c0 + i] > 0) {
+            D += p.ctx_d[c0 + i];
+            ++N;
+          }
+        }
+      }
+    }
+    D = warp_sum(D);
+    N = warp_sum(N);
+    if (lane == 0 && k < p.n_clusters) {
+      p.Dk[k] = D;
+      p.Nk[k] = N;
+    }
+    return;
+  }
+  // totals of one chunk of kTotChunk contexts: per-thread strided sums,
+  // then a fixed tree; the finish kernel adds the chunks in order
+  const int chunk = blockIdx.x - cluster_blocks;
+  const long long c0 = (long long)chunk * kTotChunk;
+  const long long c1 = (c0 + kTotChunk < p.n_ctx) ? c0 + kTotChunk : p.n_ctx;
+  double sa = 0.0, sb = 0.0, sd = 0.0;
+  long long used = 0, pos = 0, al = 0, bl = 0, ties = 0;
+  bool bad = false;
+  for (long long c = c0 + threadIdx.x; c < c1; c += blockDim.x) {
+    const int k = p.cluster[c];
+    if (k < 0 || k >= p.n_clusters) {
+      bad = true;
+      continue;
+    }
+    const int n = p.ctx_n[c];
+    if (n <= 0) continue;
+    const double d = p.ctx_d[c];
+    pos += n;
+    ++used;
+    sa += p.ctx_a[c];
+    sb += p.ctx_b[c];
+    sd += d;
+    al += d < 0.0;
+    bl += d > 0.0;
+    ties += d == 0.0;
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) set_dev_status(p.dev_status, 0x2 /* KLD_DEV_BAD_ID */);
+  __shared__ PairedPart sh[kWarps];
+  sa = warp_sum(sa);
+  sb = warp_sum(sb);
+  sd = warp_sum(sd);
+  used = warp_sum(used);
+  pos = warp_sum(pos);
+  al = warp_sum(al);
+  bl = warp_sum(bl);
+  ties = warp_sum(ties);
+  if (lane == 0) sh[w] = PairedPart{sa, sb, sd, used, pos, al, bl, ties};
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    PairedPart t = sh[0];
+    for (int j = 1; j < kWarps; ++j) {
+      t.sa += sh[j].sa;
+      t.sb += sh[j].sb;
+      t.sd += sh[j].sd;
+      t.n_used += sh[j].n_used;
+      t.n_pos += sh[j].n_pos;
+      t.a_lower += sh[j].a_lower;
+      t.b_lower += sh[j].b_lower;
+      t.ties += sh[j].ties;
+    }
+    p.parts[chunk] = t;
+  }
+}
+
+// One warp per replicate; the clusters' sums sit in shared memory when
+// there are at most kBootSmemClusters of them.  Draws are loaded four per
+// lane before their sums are gathered.
+__global__ void __launch_bounds__(kBootThreads) paired_boot_kernel(const PairedParams p) {
+  __shared__ double sD[kBootSmemClusters];
+  __shared__ int sN[kBootSmemClusters];  // counts of contexts, < 2^31
+  wait_prior_grid();
+  const bool staged = p.n_clusters <= kBootSmemClusters;
+  if (staged) {
+    for (int k = threadIdx.x; k < p.n_clusters; k += blockDim.x) {
+      sD[k] = p.Dk[k];
+      sN[k] = (int)p.Nk[k];
+    }
+  }
+  __syncthreads();
+  __shared__ unsigned cta_valid;
+  if (threadIdx.x == 0) cta_valid = 0u;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const long long r = (long long)blockIdx.x * (kBootThreads / 32) + (threadIdx.x >> 5);
+  const int32_t* draws = p.resample + r * p.n_clusters;
+  const int C = (r < p.n_boot) ? p.n_clusters : 0;  // warps past the last replicate idle
+  double D = 0.0;
+  long long N = 0;
+  bool bad = false;
+  constexpr int U = 4;
+  for (int j0 = lane; j0 < C; j0 += 32 * U) {
+    int k[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) k[u] = (j0 + 32 * u < C) ? __ldcs(draws + j0 + 32 * u) : 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (j0 + 32 * u >= C) continue;
+      if (k[u] < 0 || k[u] >= C) {
+        bad = true;
+        continue;
+      }
+      if (staged) {
+        D += sD[k[u]];
+        N += sN[k[u]];
+      } else {
+        D += __ldg(p.Dk + k[u]);
+        N += __ldg(p.Nk + k[u]);
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_dev_status(p.dev_status, 0x2 /* KLD_DEV_BAD_ID */);
+  D = warp_sum(D);
+  N = warp_sum(N);
+  if (lane == 0 && r < p.n_boot) {
+    p.boot[r] = N ? D / (double)N : CUDART_NAN;
+    p.less[r] = 0u;
+    p.eq[r] = 0u;
+    if (N) atomicAdd(&cta_valid, 1u);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && cta_valid) atomicAdd(&p.tot->n_valid, cta_valid);
+}
+
+// Block (x, y): replicates x*256 .. +255 against tile y of all replicates;
+// counts of the tile's values below and equal to each are added (integers,
+// so the order does not matter).
+__global__ void __launch_bounds__(kThreads) paired_count_kernel(const PairedParams p) {
+  __shared__ double tile[kRankTile];
+  wait_prior_grid();
+  const long long t0 = (long long)blockIdx.y * kRankTile;
+  for (int i = threadIdx.x; i < kRankTile; i += blockDim.x)
+    tile[i] = (t0 + i < p.n_boot) ? p.boot[t0 + i] : CUDART_NAN;
+  __syncthreads();
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= p.n_boot) return;
+  const double se = p.boot[e];
+  if (se != se) return;
+  unsigned lt = 0, et = 0;
+#pragma unroll 8
+  for (int j = 0; j < kRankTile; ++j) {
+    const double v = tile[j];
+    lt += v < se;
+    et += v == se;
+  }
+  if (lt) atomicAdd(p.less + e, lt);
+  if (et) atomicAdd(p.eq + e, et);
+}
+
+// The replicate whose rank range [less, less + eq) holds a target rank is
+// that order statistic (equal replicates write the same value).
+__global__ void __launch_bounds__(kThreads) paired_pick_kernel(const PairedParams p) {
+  wait_prior_grid();
+  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= p.n_boot) return;
+  const double se = p.boot[e];
+  const long long n = p.tot->n_valid;
+  if (se != se || n == 0) return;
+  const long long lo = p.less[e], hi = lo + p.eq[e];
+  for (int t = 0; t < 2 * p.nq; ++t) {
+    const long long r = target_rank(p, n, t);
+    if (lo <= r && r < hi) p.tot->ostat[t] = se;
+  }
+}
+
+// One warp: the chunks' sums (lane l adds chunks l, l + 32, ... in order,
+// then a fixed tree), the interval ends, the result.
+__global__ void paired_finish_kernel(const PairedParams p, int n_parts) {
+  wait_prior_grid();
+  const int lane = threadIdx.x;
+  const PairedTotals* t = p.tot;
+  kld_paired* o = p.out;
+  const double nan = CUDART_NAN;
+  double sa = 0.0, sb = 0.0, sd = 0.0;
+  long long used = 0, pos = 0, al = 0, bl = 0, ties = 0;
+  for (int j = lane; j < n_parts; j += 32) {
+    const PairedPart& q = p.parts[j];
+    sa += q.sa;
+    sb += q.sb;
+    sd += q.sd;
+    used += q.n_used;
+    pos += q.n_pos;
+    al += q.a_lower;
+    bl += q.b_lower;
+    ties += q.ties;
+  }
+  sa = warp_sum(sa);
+  sb = warp_sum(sb);
+  sd = warp_sum(sd);
+  used = __shfl_sync(0xffffffffu, warp_sum(used), 0);
+  pos = warp_sum(pos);
+  al = warp_sum(al);
+  bl = warp_sum(bl);
+  ties = warp_sum(ties);
+  const long long nb = t->n_valid;
+  if (lane == 0) {
+    o->n_ctx = used;
+    o->n_pos = pos;
+    o->a_lower = al;
+    o->b_lower = bl;
+    o->ties = ties;
+    o->n_boot = nb;
+    o->mean_a = used ? sa / (double)used : nan;
+    o->mean_b = used ? sb / (double)used : nan;
+    o->diff = used ? sd / (double)used : nan;
+    o->nq = p.nq;
+    o->pad = 0;
+  }
+  if (lane < KLD_MAX_QUANTILES) {
+    double v = nan;
+    if (lane < p.nq && nb > 0) {
+      const double lo = t->ostat[2 * lane], hi = t->ostat[2 * lane + 1];
+      const double h = __dmul_rn((double)(nb - 1), p.q[lane]);
+      const double frac = __dsub_rn(h, floor(h));
+      v = __dadd_rn(lo, __dmul_rn(__dsub_rn(hi, lo), frac));
+    }
+    o->ci[lane] = v;
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+size_t paired_workspace_bytes(int64_t n_ctx, int32_t n_clusters, int32_t n_boot) {
+  const size_t nc = n_ctx > 0 ? (size_t)n_ctx : 0;
+  const size_t k = n_clusters > 0 ? (size_t)n_clusters : 0;
+  const size_t b = n_boot > 0 ? (size_t)n_boot : 0;
+  const size_t parts = (nc + kTotChunk - 1) / kTotChunk + 1;
+  return align256(sizeof(PairedTotals)) + align256(sizeof(PairedPart) * parts) + 3 * align256(sizeof(double) * nc) +
+         align256(sizeof(int32_t) * nc) +
+         align256(sizeof(double) * k) + align256(sizeof(long long) * k) + 2 * align256(sizeof(unsigned) * b) +
+         align256(sizeof(double) * b);
+}
+
+cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
+  PairedParams p;
+  p.a = a.kl_a;
+  p.b = a.kl_b;
+  p.mask = a.mask;
+  p.n_ctx = a.n_ctx;
+  p.ctx_len = a.ctx_len;
+  p.cluster = a.cluster;
+  p.n_clusters = a.n_clusters;
+  p.resample = a.resample;
+  p.n_boot = a.n_boot;
+  p.nq = a.nq;
+  for (int i = 0; i < KLD_MAX_QUANTILES; ++i) p.q[i] = a.quantiles[i];
+  p.out = a.out;
+  p.dev_status = a.dev_status;
+  char* ws = reinterpret_cast<char*>(a.workspace);
+  const size_t nc = (size_t)a.n_ctx, k = (size_t)a.n_clusters, b = (size_t)a.n_boot;
+  const int n_parts = (int)((nc + kTotChunk - 1) / kTotChunk);
+  p.tot = reinterpret_cast<PairedTotals*>(ws);
+  ws += align256(sizeof(PairedTotals));
+  p.parts = reinterpret_cast<PairedPart*>(ws);
+  ws += align256(sizeof(PairedPart) * (size_t)(n_parts + 1));
+  p.ctx_a = reinterpret_cast<double*>(ws);
+  ws += align256(sizeof(double) * nc);
+  p.ctx_b = reinterpret_cast<double*>(ws);
+  ws += align256(sizeof(double) * nc);
+  p.ctx_d = reinterpret_cast<double*>(ws);
+  ws += align256(sizeof(double) * nc);
+  p.ctx_n = reinterpret_cast<int32_t*>(ws);
+  ws += align256(sizeof(int32_t) * nc);
+  p.Dk = reinterpret_cast<double*>(ws);
+  ws += align256(sizeof(double) * k);
+  p.Nk = reinterpret_cast<long long*>(ws);
+  ws += align256(sizeof(long long) * k);
+  p.less = reinterpret_cast<unsigned*>(ws);
+  ws += align256(sizeof(unsigned) * b);
+  p.eq = reinterpret_cast<unsigned*>(ws);
+  ws += align256(sizeof(unsigned) * b);
+  p.boot = a.boot_stats ? a.boot_stats : reinterpret_cast<double*>(ws);
+
+  cudaError_t e = cudaSuccess;
+  const unsigned ctx_grid = (unsigned)((nc + kWarps - 1) / kWarps);
+  if (ctx_grid > 0) e = launch_dependent(paired_ctx_kernel, dim3(ctx_grid), dim3(kThreads), stream, p);
+  else e = launch_dependent(paired_ctx_kernel, dim3(1), dim3(kThreads), stream, p);  // clears the counter
+  if (e != cudaSuccess) return e;
+  const int cluster_blocks = (int)((k + kWarps - 1) / kWarps);
+  e = launch_dependent(paired_cluster_kernel, dim3(cluster_blocks + n_parts), dim3(kThreads), stream, p,
+                       cluster_blocks);
+  if (e != cudaSuccess) return e;
+  if (b > 0) {
+    constexpr int kBootWarps = kBootThreads / 32;
+    e = launch_dependent(paired_boot_kernel, dim3((unsigned)((b + kBootWarps - 1) / kBootWarps)),
+                         dim3(kBootThreads), stream, p);
+    if (e != cudaSuccess) return e;
+    const unsigned gx = (unsigned)((b + kThreads - 1) / kThreads);
+    const unsigned gy = (unsigned)((b + kRankTile - 1) / kRankTile);
+    e = launch_dependent(paired_count_kernel, dim3(gx, gy), dim3(kThreads), stream, p);
+    if (e != cudaSuccess) return e;
+    e = launch_dependent(paired_pick_kernel, dim3(gx), dim3(kThreads), stream, p);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_dependent(paired_finish_kernel, dim3(1), dim3(32), stream, p, n_parts);
+}
+
+}  // namespace kld

@@ -342,3 +342,28 @@ def position_results(seed: int = seed_for(7), device="cpu", n: int = 2047) -> di
     lpr = 2.0 * torch.log1p(-torch.rand(n, generator=g, device=device))
     lpc = lpr + 0.05 * torch.log1p(-torch.rand(n, generator=g, device=device))
     return dict(kl=kl, ra=ra, ca=ca, lpr=lpr.float(), lpc=lpc.float())
+
+
+def paired_candidates(seed: int = seed_for(8), device="cpu", n_ctx: int = 5120, ctx_len: int = 2047,
+                      n_clusters: int = 842, n_boot: int = 10_000) -> dict:
+    """Two candidates' per-position KL over one suite, its source clusters
+    and bootstrap draws ("Qwen3.8-27B fidelity suite v5", "What is in
+    here": 5,120 contexts of 2,047 scored positions over 842 source
+    clusters).
+
+    kl_a: f32 [n_ctx, ctx_len], log-normal around e^-7.5 with a spread of
+    e^±2 (means near the pages' 5e-4), scaled per context by e^{N(0, 0.5^2)};
+    kl_b = kl_a * e^{N(0, 0.1^2)} per position.  Contexts go to clusters in
+    contiguous runs of uneven length (every cluster gets at least one).
+    resample: int32 [n_boot, n_clusters], uniform draws of cluster ids."""
+    g = _gen(seed, device)
+    base = -7.5 + 0.5 * torch.randn((n_ctx, 1), generator=g, device=device)
+    kl_a = torch.exp(base + 2.0 * torch.randn((n_ctx, ctx_len), generator=g, device=device)).float()
+    kl_b = (kl_a * torch.exp(0.1 * torch.randn((n_ctx, ctx_len), generator=g, device=device))).float()
+    cut = torch.randperm(max(n_ctx - 1, 1), generator=g, device=device)[:n_clusters - 1] + 1
+    starts = torch.zeros(n_ctx, dtype=torch.int32, device=device)
+    if n_ctx > 1 and n_clusters > 1:
+        starts[cut.clamp(max=n_ctx - 1)] = 1
+    cluster = (torch.cumsum(starts, 0) % max(n_clusters, 1)).to(torch.int32)
+    resample = torch.randint(0, n_clusters, (n_boot, n_clusters), generator=g, device=device, dtype=torch.int32)
+    return dict(kl_a=kl_a, kl_b=kl_b, cluster=cluster, resample=resample, n_clusters=n_clusters)

@@ -220,3 +220,44 @@ def test_reduce_shard_validation(lib):
     assert sh(lib, step=last, b=None, out=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
     assert lib.kld_reduce_shard_block_bytes() >= 16 * 256 * 4
     assert lib.kld_reduce_shard_workspace_size(10) >= 4 * 16 * 256 * 4   # the four passes' all-shard histograms
+
+
+def test_paired_struct_size_matches_header():
+    assert ctypes.sizeof(_lib.KldPaired) == 144
+
+
+def pc(lib, **kw):
+    a = dict(a=A16, b=A16 + 4096, mask=None, n=4, L=16, cl=A16 + 8192, C=3, rs=A16 + 12288, B=5,
+             q=(0.025, 0.975), out=A16 + 16384, boot=None, ws=A16 + 65536, wsb=None, st=None)
+    a.update(kw)
+    wsb = lib.kld_paired_workspace_size(max(a["n"], 0), max(a["C"], 0), max(a["B"], 0)) if a["wsb"] is None \
+        else a["wsb"]
+    qs = (ctypes.c_double * max(len(a["q"]), 1))(*a["q"])
+    return lib.kld_paired_compare(a["a"], a["b"], a["mask"], a["n"], a["L"], a["cl"], a["C"], a["rs"], a["B"],
+                                  ctypes.cast(qs, ctypes.c_void_p), len(a["q"]), a["out"], a["boot"], a["ws"],
+                                  wsb, a["st"], None)
+
+
+def test_paired_validation(lib):
+    assert pc(lib, n=-1) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, L=0) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, C=0) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, B=-1) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, B=1 << 19, C=1 << 12) == _lib.KLD_ERR_INVALID_ARG        # draws beyond 2^31
+    assert pc(lib, B=(1 << 20) + 1, C=1) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, q=(1.5,)) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, q=(0.5,) * 9) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, a=None) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, cl=None) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, rs=None) == _lib.KLD_ERR_INVALID_ARG                     # draws needed when B > 0
+    assert pc(lib, out=None) == _lib.KLD_ERR_INVALID_ARG
+    assert pc(lib, ws=None) == _lib.KLD_ERR_WORKSPACE
+    assert pc(lib, wsb=8) == _lib.KLD_ERR_WORKSPACE
+    assert pc(lib, ws=A16 + 64) == _lib.KLD_ERR_ALIGNMENT
+    assert pc(lib, out=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
+    assert pc(lib, a=MIS) == _lib.KLD_ERR_ALIGNMENT                          # rows are read as 16-byte vectors
+    assert pc(lib, b=A16 + 4104) == _lib.KLD_ERR_ALIGNMENT
+    assert pc(lib, boot=A16 + 4) == _lib.KLD_ERR_ALIGNMENT
+    small = lib.kld_paired_workspace_size(10, 3, 5)
+    assert lib.kld_paired_workspace_size(1000, 3, 5) > small
+    assert lib.kld_paired_workspace_size(10, 3, 5000) > small
