@@ -53,6 +53,7 @@ constexpr int kCap = KLD_CAPTURE_CANDIDATES;  // candidates kept per row
 constexpr int kFinThreads = 128;     // finish: one CTA per row, 8 rows per SM
 constexpr int kSampleThreads = 256;  // sample: 16 sampled values per thread
 constexpr int kMaxK = KLD_SPARSE_MAX_K;
+constexpr int kStage = 2048;  // candidates a finish CTA keeps in shared memory
 
 // Tail state of one warp over one row piece (16 bytes): running maximum m
 // over all elements, and over the non-candidates T = sum e^{x-m},
@@ -346,6 +347,16 @@ struct BufCands {
   __device__ __forceinline__ int idx(int i) const { return i < ns ? __ldg(&cand[i].y) : ri[i - ns]; }
 };
 
+// A row's candidates staged in shared memory (most rows: the finish
+// reads every candidate on each of its passes).
+struct SmemCands {
+  const float* v;
+  const int* id;
+  int n;
+  __device__ __forceinline__ float val(int i) const { return v[i]; }
+  __device__ __forceinline__ int idx(int i) const { return id[i]; }
+};
+
 // Every element of a row, read from global memory (the exact path).
 template <bool kBF16>
 struct RowCands {
@@ -367,8 +378,9 @@ struct FinScratch {  // block-reduction slots for up to 8 warps
 
 // The r-th largest (1-based) of the 32-bit keys of the elements i < n for
 // which key(i, k) returns true: an MSB-first radix select, 8 bits per pass,
-// with shared-memory histograms (lanes with equal digits add once, by
-// __match_any_sync).  Returns the key; eq = elements equal to it, rank = its
+// with shared-memory histograms (plain atomics: measured faster here than
+// aggregating equal digits with __match_any_sync).  Returns the key; eq =
+// elements equal to it, rank = its
 // rank among them (eq - rank of the equal keys come after position r); rank
 // is 0 when fewer than r elements take part.
 // Every thread of the CTA calls this.
@@ -384,8 +396,7 @@ __device__ uint32_t rth_largest(int n, int r, KeyFn key, FinScratch& sc, int& eq
       uint32_t k = 0u;
       const bool ok = i < n && key(i, k) && (k & pmask) == prefix;
       const unsigned digit = ok ? ((k >> shift) & 255u) : 256u;
-      const unsigned peers = __match_any_sync(0xffffffffu, digit);
-      if (ok && lane == __ffs(peers) - 1) atomicAdd(&sc.hist[digit], (unsigned)__popc(peers));
+      if (ok) atomicAdd(&sc.hist[digit], 1u);
     }
     __syncthreads();
     if (threadIdx.x < 32) {
@@ -605,11 +616,21 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
   while (P < K) P <<= 1;
   for (int j = K + tid; j < P; j += kFinThreads) sel[j] = 0ull;
   __syncthreads();
-  for (int i = tid; i < n; i += kFinThreads) {
-    const uint32_t k = vkey(src.val(i));
-    const uint32_t id = (uint32_t)src.idx(i);
-    if (k > pre || (k == pre && id <= id_cut)) {
-      const int at = atomicAdd(&sc.n_sel, 1);
+  for (int i0 = tid & ~31; i0 < n; i0 += kFinThreads) {  // warp-uniform: one slot reservation per warp
+    const int i = i0 + (tid & 31);
+    uint32_t k = 0u, id = 0u;
+    bool take = false;
+    if (i < n) {
+      k = vkey(src.val(i));
+      id = (uint32_t)src.idx(i);
+      take = k > pre || (k == pre && id <= id_cut);
+    }
+    const unsigned takers = __ballot_sync(0xffffffffu, take);
+    int base = 0;
+    if ((tid & 31) == 0 && takers) base = atomicAdd(&sc.n_sel, __popc(takers));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (take) {
+      const int at = base + __popc(takers & ((1u << (tid & 31)) - 1u));
       if (at < K) sel[at] = ((unsigned long long)k << 32) | (unsigned long long)(~id);
     }
   }
@@ -711,6 +732,8 @@ __global__ void __launch_bounds__(kFinThreads, 8) cap_finalize_kernel(const CapP
   __shared__ CapPiece merged;
   __shared__ float rv[8];
   __shared__ int ri[8];
+  __shared__ float stage_v[kStage];
+  __shared__ int stage_i[kStage];
   wait_prior_grid();
   const int row = blockIdx.x;
   const int tid = threadIdx.x;
@@ -754,7 +777,20 @@ __global__ void __launch_bounds__(kFinThreads, 8) cap_finalize_kernel(const CapP
   }
   ge = __syncthreads_count(ge);
   const bool exact = p.force_exact || cnt > kCap || ns + ge < p.K;
-  if (!exact) {
+  if (!exact && ns + ragged <= kStage) {
+    const int2* cand = p.cand + (int64_t)row * kCap;
+    for (int i = tid; i < ns; i += kFinThreads) {
+      const int2 c = __ldg(cand + i);
+      stage_v[i] = __int_as_float(c.x);
+      stage_i[i] = c.y;
+    }
+    if (tid < ragged) {
+      stage_v[ns + tid] = rv[tid];
+      stage_i[ns + tid] = ri[tid];
+    }
+    __syncthreads();
+    capture_finish<kBF16>(p, row, SmemCands{stage_v, stage_i, ns + ragged}, merged.m, merged.T, merged.B, sel, sc);
+  } else if (!exact) {
     capture_finish<kBF16>(p, row, BufCands{p.cand + (int64_t)row * kCap, ns, rv, ri, ns + ragged}, merged.m,
                           merged.T, merged.B, sel, sc);
   } else {
