@@ -120,6 +120,8 @@ TEST_PROTOTYPES = {
     "kld_sparse_ref_score_split": (ctypes.c_int, [_P, ctypes.c_int, _I64, _I64, _I64, _P, _I32, _P, _P, _P, _P,
                                                   _P, _P, _P, _P, _SZ, _P, _P, _I32]),
     "kld_from_hidden_shared_head_withhold": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P, _P]),
+    "kld_reduce_stats_withhold": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _P, _I32, _P, _I32, _P, _P,
+                                                 _SZ, _P, _P]),
     "kld_full_vocab_split": (ctypes.c_int, [_P, _P, ctypes.c_int, _I64, _I64, _I64, _I64, _P, _P, _P,
                                             _P, _P, _P, _P, _SZ, _P, _P, _I32]),
 }

@@ -340,12 +340,11 @@ kld_status kld_from_hidden_shared_head_withhold(const void* h_ref, const void* h
 
 size_t kld_reduce_workspace_size(int64_t n) { return kld::reduce_workspace_bytes(n); }
 
-kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
-                            const uint8_t* top1, const float* ref_target_lp,
-                            const float* cand_target_lp, const uint8_t* mask, int64_t n,
-                            const double* quantiles, int32_t nq, const float* thresholds, int32_t nt,
-                            kld_stats* out, void* workspace, size_t workspace_bytes,
-                            int32_t* dev_status, void* stream) {
+static kld_status reduce_impl(const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
+                              const uint8_t* top1, const float* ref_target_lp, const float* cand_target_lp,
+                              const uint8_t* mask, int64_t n, const double* quantiles, int32_t nq,
+                              const float* thresholds, int32_t nt, kld_stats* out, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_status, void* stream, int withhold) {
   if (n < 0 || n > INT32_MAX) return KLD_ERR_INVALID_ARG;
   if (nq < 0 || nq > KLD_MAX_QUANTILES || nt < 0 || nt > KLD_MAX_THRESHOLDS) return KLD_ERR_INVALID_ARG;
   if ((nq > 0 && !quantiles) || (nt > 0 && !thresholds)) return KLD_ERR_INVALID_ARG;
@@ -375,7 +374,32 @@ kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const in
   a.out = out;
   a.workspace = workspace;
   a.dev_status = dev_status;
+  a.withhold = withhold;
   return cuda_status(kld::launch_reduce(a, static_cast<cudaStream_t>(stream)));
+}
+
+kld_status kld_reduce_stats(const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
+                            const uint8_t* top1, const float* ref_target_lp,
+                            const float* cand_target_lp, const uint8_t* mask, int64_t n,
+                            const double* quantiles, int32_t nq, const float* thresholds, int32_t nt,
+                            kld_stats* out, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
+  return reduce_impl(kl, ref_argmax, cand_argmax, top1, ref_target_lp, cand_target_lp, mask, n, quantiles, nq,
+                     thresholds, nt, out, workspace, workspace_bytes, dev_status, stream, 0);
+}
+
+// Test hook, not in kld.h: for more than 8192 positions (the cooperative
+// grid), CTA 0 leaves before the first grid barrier, so the other CTAs'
+// bounded waits run out and set KLD_DEV_TIMEOUT; the statistics are not
+// written.
+kld_status kld_reduce_stats_withhold(const float* kl, const int32_t* ref_argmax, const int32_t* cand_argmax,
+                                     const uint8_t* top1, const float* ref_target_lp,
+                                     const float* cand_target_lp, const uint8_t* mask, int64_t n,
+                                     const double* quantiles, int32_t nq, const float* thresholds, int32_t nt,
+                                     kld_stats* out, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream) {
+  return reduce_impl(kl, ref_argmax, cand_argmax, top1, ref_target_lp, cand_target_lp, mask, n, quantiles, nq,
+                     thresholds, nt, out, workspace, workspace_bytes, dev_status, stream, 1);
 }
 
 size_t kld_reduce_shard_block_bytes(void) { return kld::reduce_shard_block_bytes(); }

@@ -120,6 +120,7 @@ struct ReduceArgs {
   kld_stats* out;
   void* workspace;
   int32_t* dev_status;
+  int withhold;  // tests only (see reduce.cu)
 };
 size_t reduce_workspace_bytes(int64_t n);
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream);

@@ -80,6 +80,7 @@ struct ReduceParams {
   Partial* partials;  // shard protocol: [gridDim of pass 0]
   int32_t* dev_status;
   unsigned* hist_out; // shard protocol: where a pass adds its histogram
+  int withhold;       // tests only: the cooperative grid's CTA 0 leaves before the first barrier
 };
 
 __device__ __forceinline__ uint32_t f2key(float f) {
@@ -674,6 +675,9 @@ __global__ void __launch_bounds__(kCoopThreads, 1) reduce_coop_kernel(const Redu
     hist_keys<kTopBits, true>(keys, m, sel, 32 - kTopBits, hist);
     __syncthreads();
   }
+  // (tests only: CTA 0 never arrives, so every other CTA's bounded wait
+  // runs out and reports KLD_DEV_TIMEOUT)
+  if (p.withhold && blockIdx.x == 0) return;
   flush_and_arrive(hist, g->hist0, kTopBins, &g->arrive[0], &ticket);
   if (!grid_wait(&g->arrive[0], p.dev_status, &ok)) return;
   {  // every CTA: the whole first-pass histogram, the scored count, the first digits
@@ -894,6 +898,7 @@ ReduceParams make_params(const ReduceArgs& a) {
   p.partials = nullptr;
   p.dev_status = a.dev_status;
   p.hist_out = nullptr;
+  p.withhold = a.withhold;
   return p;
 }
 

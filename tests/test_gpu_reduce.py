@@ -97,3 +97,29 @@ def test_deterministic_large(cuda_device):
     a = kq.kld_reduce_stats(*args)
     b = kq.kld_reduce_stats(*args)
     assert a == b or all((a[k] == b[k]) or (a[k] != a[k] and b[k] != b[k]) for k in a)
+
+
+def test_grid_barrier_timeout_is_reported(cuda_device):
+    """The cooperative reduction's grid barriers are bounded waits: with one
+    CTA withheld (a test hook) the others give up, report KLD_DEV_TIMEOUT and
+    return; the next call on the same context and workspace is correct."""
+    import ctypes
+    from quantization_fidelity_scoring_b200 import _lib
+    n = 100_000
+    kl, ra, ca, lr, lc, mask = make(n, seed=6, nan_every=17)
+    T = lambda a: torch.tensor(a, device=cuda_device)
+    dk, dra, dca, dlr, dlc, dm = (T(a) for a in (kl, ra, ca, lr, lc, mask))
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=cuda_device)
+    out = torch.zeros(280, dtype=torch.uint8, device=cuda_device)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    qs = (ctypes.c_double * len(QS))(*QS)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    rc = _lib.load().kld_reduce_stats_withhold(p(dk), p(dra), p(dca), None, p(dlr), p(dlc), p(dm), n,
+                                               ctypes.cast(qs, ctypes.c_void_p), len(QS), None, 0, p(out), p(ws),
+                                               ws.numel(), p(status),
+                                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert status.item() & 0x4                     # KLD_DEV_TIMEOUT
+    st = kq.kld_reduce_stats(dk, dra, dca, None, dlr, dlc, dm, QS, THR, workspace=ws)
+    compare(st, O.reduce_stats(kl, ra, ca, None, lr, lc, mask, quantiles=QS, thresholds=THR))
