@@ -123,3 +123,37 @@ def test_deterministic(cuda_device):
     a = run(d["ref_ids"], d["ref_lp"], d["cand_ids"], d["cand_lp"], d["vocab"])
     b = run(d["ref_ids"], d["ref_lp"], d["cand_ids"], d["cand_lp"], d["vocab"])
     assert torch.equal(a["kl"], b["kl"]) and torch.equal(a["n_matched"], b["n_matched"])
+
+
+def _table_slot(ids):
+    """The shared-memory table slot the kernel's matching hashes an id to (a
+    property of the implementation, used only to build colliding inputs)."""
+    ids = np.asarray(ids, dtype=np.uint64)
+    return ((ids * np.uint64(0x9E3779B1)) & np.uint64(0xFFFFFFFF)) >> np.uint64(24)
+
+
+def test_colliding_candidate_ids(cuda_device):
+    """Candidate lists whose ids all hash to one table slot (the longest
+    probe chains the matching can meet), with repeated ids among them, next
+    to a list of ordinary ids: every case matches the oracle."""
+    V, k = (1 << 25) - 1, 64                     # the largest vocabulary the library takes
+    rng = np.random.default_rng(11)
+    pool = rng.choice(V, 1 << 20, replace=False).astype(np.int64)
+    h = _table_slot(pool)
+    same = pool[h == h[0]][:k]
+    assert same.shape[0] == k
+    rows = []
+    for r in range(6):
+        cand = rng.choice(same, k, replace=True) if r % 2 else rng.permutation(same)
+        if r == 4:
+            cand = rng.choice(V, k, replace=False)          # an ordinary row in the same launch
+        ref = np.where(rng.random(k) < 0.7, cand[rng.permutation(k)], rng.choice(V, k))
+        rows.append((ref.astype(np.int32), cand.astype(np.int32)))
+    ri = np.stack([a for a, _ in rows])
+    ci = np.stack([b for _, b in rows])
+    lp = np.sort(np.log(rng.dirichlet(np.ones(80), (6,))[:, :k]), axis=1)[:, ::-1].astype(np.float16)
+    cl = np.sort(np.log(rng.dirichlet(np.ones(80), (6,))[:, :k]), axis=1)[:, ::-1].astype(np.float16)
+    t = [torch.tensor(np.ascontiguousarray(a), device=cuda_device) for a in (ri, lp, ci, cl)]
+    res = run(*t, V)
+    assert res["status"] == 0
+    check(res, *t, V)
