@@ -362,7 +362,9 @@ def run_ours(args) -> int:
                                    "sparse_ref": measure_sparse_ref(args, kq, dev),
                                    "sparse_capture": measure_sparse_capture(args, kq, dev),
                                    "shared_head": measure_shared_head(args, kq, dev),
-                                   "paired": measure_paired(args, kq, dev)}
+                                   "paired": measure_paired(args, kq, dev),
+                                   "batched_f32": measure_batched(args, kq, dev)}
+            torch.cuda.empty_cache()
         if world == 1 and not args.no_cpu_baseline:
             rows = list(range(0, n, max(1, n // args.cpu_rows)))[:args.cpu_rows]
             dt = oracle_rows(ref, cand, targets, rows)
@@ -578,6 +580,65 @@ def measure_reduce(args, kq, dev, n=N_ROWS, steps=None) -> dict:
             "launches_per_step": launches_per_step(n) - 2}
 
 
+def measure_batched(args, kq, dev, steps=None) -> dict:
+    """Batched full-vocabulary scoring (16 windows x 2047 rows of f32
+    logits, 32.5 GB per side, resident): kld_full_vocab + kld_reduce_stats
+    per step, inputs far larger than L2."""
+    import torch
+    from synth import workloads as W
+    t0 = time.perf_counter()
+    d = W.batched_full_vocab(device=dev)
+    torch.cuda.synchronize()
+    gen_s = time.perf_counter() - t0
+    ref, cand, targets = d["ref"], d["cand"], d["targets"]
+    n = ref.shape[0]
+    kl = torch.empty(n, dtype=torch.float32, device=dev)
+    ra = torch.empty(n, dtype=torch.int32, device=dev)
+    ca = torch.empty(n, dtype=torch.int32, device=dev)
+    lpr = torch.empty(n, dtype=torch.float32, device=dev)
+    lpc = torch.empty(n, dtype=torch.float32, device=dev)
+    fws = torch.empty(kq.kld_full_vocab_workspace_size(n), dtype=torch.uint8, device=dev)
+    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
+    out = torch.empty(280, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        kq.kld_full_vocab(ref, cand, targets, kl=kl, ref_argmax=ra, cand_argmax=ca, ref_target_lp=lpr,
+                          cand_target_lp=lpc, workspace=fws, dev_status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=out, workspace=ws,
+                            dev_status=status, stream=stream, to_host=False)
+
+    steps = steps or max(1, min(args.steps, 20))
+    for _ in range(3):
+        step()
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(steps):
+        step(kev[i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    assert status.item() == 0, f"device status {status.item()}"
+    ms = start.elapsed_time(stop) / steps
+    k_ms = statistics.mean(a.elapsed_time(b) for a, b in kev)
+    alg = 2 * n * VOCAB * 4 + n * (4 + 4 * 5)
+    peak, _ = measured_peaks()
+    del d, ref, cand
+    return {"workload": f"batched full-vocabulary scoring: {n} positions x 248,320 f32 logits (16 windows)",
+            "value": n / (ms / 1e3), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+            "step": "kld_full_vocab + kld_reduce_stats", "gpu_launches_per_step": 2 + 2,
+            "generate_s": gen_s,
+            "roofline": {"bound": "hbm", "achieved": alg / (k_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": alg / (k_ms / 1e3) / 1e9 / peak,
+                         "kernel": "kld::stream_kernel<f32> + kld::merge_kernel<f32>", "kernel_ms": k_ms}}
+
+
 def measure_paired(args, kq, dev, steps=None) -> dict:
     """Two candidates compared paired per context over one whole suite
     (5,120 contexts x 2,047 positions, 842 source clusters) with a
@@ -779,6 +840,8 @@ def main(argv=None) -> int:
                     help="only time the sparse-reference score on ROWS positions (for profiling)")
     ap.add_argument("--profile-capture", type=int, metavar="ROWS",
                     help="only time the sparse capture on ROWS positions (for profiling)")
+    ap.add_argument("--profile-batched", action="store_true",
+                    help="only time the batched f32 workload (16 windows, 65 GB of logits)")
     ap.add_argument("--profile-paired", action="store_true",
                     help="only time the paired comparison of two candidates over one suite (for profiling)")
     ap.add_argument("--profile-reduce", type=int, metavar="POSITIONS",
@@ -812,6 +875,12 @@ def main(argv=None) -> int:
         kq.load_library()
         print(json.dumps(measure_sparse_capture(args, kq, torch.device("cuda:0"), n_rows=args.profile_capture,
                                                 steps=args.steps)), flush=True)
+        return 0
+    if args.profile_batched:
+        import torch
+        import quantization_fidelity_scoring_b200 as kq
+        kq.load_library()
+        print(json.dumps(measure_batched(args, kq, torch.device("cuda:0"), steps=args.steps)), flush=True)
         return 0
     if args.profile_paired:
         import torch
