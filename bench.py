@@ -379,11 +379,11 @@ def run_ours(args) -> int:
 
 def launches_per_step(n: int, world: int = 1) -> int:
     """Library kernels per step: streaming pass + piece merge + reduction
-    (one CTA up to 65,536 positions, else zero + 4 passes + final; across
-    ranks the five shard steps: 3 + 3 x 3 + 2 kernels)."""
+    (one CTA up to 8192 positions, else a clearing launch + one cooperative
+    grid; across ranks the five shard steps: 3 + 3 x 3 + 2 kernels)."""
     if world > 1:
         return 2 + 14
-    return 2 + (1 if n <= 65536 else 6)
+    return 2 + (1 if n <= 8192 else 2)
 
 
 def measure_topk(args, kq, dev, windows=512, steps=None) -> dict:
