@@ -475,8 +475,7 @@ size_t kld_paired_workspace_size(int64_t n_ctx, int32_t n_clusters, int32_t n_bo
  *   resample       int32 [n_boot, n_clusters], the draws (the caller's random
  *                  numbers); out-of-range draws set KLD_DEV_BAD_ID and are skipped.
  *                  May be NULL when n_boot == 0.
- *   n_boot         0 .. 2^20 replicates; n_boot * n_clusters < 2^31 (the percentiles
- *                  compare every pair of replicates: O(n_boot^2) work).
+ *   n_boot         >= 0 replicates; n_boot * n_clusters < 2^31.
  *   quantiles      HOST double [nq] in [0, 1]; nq <= KLD_MAX_QUANTILES.
  *   out            DEVICE kld_paired, 8-byte aligned.
  *   boot_stats     DEVICE double [n_boot] for the replicate statistics, or NULL.

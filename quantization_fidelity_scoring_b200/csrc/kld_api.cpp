@@ -460,7 +460,7 @@ kld_status kld_paired_compare(const float* kl_a, const float* kl_b, const uint8_
                               int32_t* dev_status, void* stream) {
   if (n_ctx < 0 || ctx_len < 1 || n_clusters < 1 || n_boot < 0) return KLD_ERR_INVALID_ARG;
   if (n_ctx > ((int64_t)1 << 40) / ctx_len || n_ctx > INT32_MAX) return KLD_ERR_INVALID_ARG;
-  if ((int64_t)n_boot * n_clusters >= ((int64_t)1 << 31) || n_boot > (1 << 20)) return KLD_ERR_INVALID_ARG;
+  if ((int64_t)n_boot * n_clusters >= ((int64_t)1 << 31)) return KLD_ERR_INVALID_ARG;
   if (nq < 0 || nq > KLD_MAX_QUANTILES || (nq > 0 && !quantiles)) return KLD_ERR_INVALID_ARG;
   for (int i = 0; i < nq; ++i)
     if (!(quantiles[i] >= 0.0 && quantiles[i] <= 1.0)) return KLD_ERR_INVALID_ARG;

@@ -9,7 +9,7 @@
 // and the "compare against a published candidate" step).  The page gives
 // no formulas; kld.h states the reading implemented here.
 //
-// Six launches, all deterministic (f64 sums in fixed orders, integer
+// Five launches, all deterministic (f64 sums in fixed orders, integer
 // counts):
 //   ctx      one warp per context: sums of A's and B's counted KL (exact in
 //            f64 for ordinary spreads of f32 values), the count, the means
@@ -18,12 +18,12 @@
 //            context order; more blocks sum chunks of 1024 contexts (means,
 //            win and tie counts) for the finish to add in order.
 //   boot     one warp per replicate: the draws' D and N gathered and summed.
-//   count    every replicate counts the replicates below and equal to it,
-//            one tile of 1024 replicates per block row;
-//   pick     the replicate whose rank range holds a target rank is that
-//            order statistic (exact, ties included).
+//   select   one CTA finds the replicates' order statistics at the target
+//            ranks exactly (bucketed 64-bit keys, a few passes);
 //   finish   one warp writes the result.
 #include <math_constants.h>
+
+#include <mutex>
 
 #include "kld_common.cuh"
 #include "launch.h"
@@ -34,7 +34,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTargets = 2 * KLD_MAX_QUANTILES;
-constexpr int kRankTile = 1024;  // replicates staged in shared memory at a time
 constexpr int kIdTile = 4096;    // cluster ids staged in shared memory at a time
 constexpr int kBootThreads = 1024;
 constexpr int kBootSmemClusters = 2048;  // clusters whose sums a boot CTA keeps in shared memory
@@ -73,8 +72,6 @@ struct PairedParams {
   int32_t* ctx_n;
   double* Dk;
   long long* Nk;
-  unsigned* less;  // [n_boot] replicates below each replicate
-  unsigned* eq;    // [n_boot] replicates equal to it (itself included)
   PairedPart* parts;  // [ceil(n_ctx / kTotChunk)]
   PairedTotals* tot;
   int32_t* dev_status;
@@ -273,9 +270,6 @@ __global__ void __launch_bounds__(kBootThreads) paired_boot_kernel(const PairedP
     }
   }
   __syncthreads();
-  __shared__ unsigned cta_valid;
-  if (threadIdx.x == 0) cta_valid = 0u;
-  __syncthreads();
   const int lane = threadIdx.x & 31;
   const long long r = (long long)blockIdx.x * (kBootThreads / 32) + (threadIdx.x >> 5);
   const int32_t* draws = p.resample + r * p.n_clusters;
@@ -307,54 +301,211 @@ __global__ void __launch_bounds__(kBootThreads) paired_boot_kernel(const PairedP
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_dev_status(p.dev_status, 0x2 /* KLD_DEV_BAD_ID */);
   D = warp_sum(D);
   N = warp_sum(N);
-  if (lane == 0 && r < p.n_boot) {
-    p.boot[r] = N ? D / (double)N : CUDART_NAN;
-    p.less[r] = 0u;
-    p.eq[r] = 0u;
-    if (N) atomicAdd(&cta_valid, 1u);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0 && cta_valid) atomicAdd(&p.tot->n_valid, cta_valid);
+  if (lane == 0 && r < p.n_boot) p.boot[r] = N ? D / (double)N : CUDART_NAN;
 }
 
-// Block (x, y): replicates x*256 .. +255 against tile y of all replicates;
-// counts of the tile's values below and equal to each are added (integers,
-// so the order does not matter).
-__global__ void __launch_bounds__(kThreads) paired_count_kernel(const PairedParams p) {
-  __shared__ double tile[kRankTile];
-  wait_prior_grid();
-  const long long t0 = (long long)blockIdx.y * kRankTile;
-  for (int i = threadIdx.x; i < kRankTile; i += blockDim.x)
-    tile[i] = (t0 + i < p.n_boot) ? p.boot[t0 + i] : CUDART_NAN;
-  __syncthreads();
-  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= p.n_boot) return;
-  const double se = p.boot[e];
-  if (se != se) return;
-  unsigned lt = 0, et = 0;
-#pragma unroll 8
-  for (int j = 0; j < kRankTile; ++j) {
-    const double v = tile[j];
-    lt += v < se;
-    et += v == se;
-  }
-  if (lt) atomicAdd(p.less + e, lt);
-  if (et) atomicAdd(p.eq + e, et);
+// Exact order statistics of the replicate statistics (NaN left out) at the
+// target ranks, in one CTA, on order-preserving 64-bit keys of the doubles.
+// The keys in [klo, khi] are spread over kBuckets buckets by the monotone
+// map (key - klo) * kBuckets / (khi - klo + 1), which puts klo and khi in
+// different buckets and divides the key range ~4096-fold; the bucket holding
+// the target rank is either small enough to gather into shared memory and
+// rank exactly by pairwise counting, or becomes the next [klo, khi] (its own
+// least and greatest key).  64-bit keys need at most six such rounds.
+constexpr int kSelThreads = 1024;
+constexpr int kBuckets = 4096;
+constexpr int kGather = 1024;
+
+struct SelShared {
+  unsigned hist[kBuckets];
+  unsigned long long gather[kGather];
+  unsigned long long rk[2][32];
+  unsigned ru[32];
+  unsigned long long answer;
+  unsigned n_gather, bucket, before;
+};
+
+__device__ __forceinline__ unsigned long long dkey(double v) {
+  unsigned long long u = (unsigned long long)__double_as_longlong(v);
+  if (u == 0x8000000000000000ull) u = 0ull;  // -0 sorts with +0
+  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// The replicate whose rank range [less, less + eq) holds a target rank is
-// that order statistic (equal replicates write the same value).
-__global__ void __launch_bounds__(kThreads) paired_pick_kernel(const PairedParams p) {
+__device__ __forceinline__ double dval(unsigned long long k) {
+  const unsigned long long u = (k & 0x8000000000000000ull) ? (k & 0x7fffffffffffffffull) : ~k;
+  return __longlong_as_double((long long)u);
+}
+
+__device__ __forceinline__ int key_bucket(unsigned long long k, unsigned long long klo, double scale) {
+  const int b = (int)((double)(k - klo) * scale);
+  return b < kBuckets - 1 ? b : kBuckets - 1;
+}
+
+// Block-wide (min, max) of 64-bit keys; returned to every thread.
+__device__ void block_key_range(unsigned long long& mn, unsigned long long& mx, SelShared& S) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, mn, off);
+    const unsigned long long b = __shfl_xor_sync(0xffffffffu, mx, off);
+    mn = a < mn ? a : mn;
+    mx = b > mx ? b : mx;
+  }
+  if (lane == 0) {
+    S.rk[0][w] = mn;
+    S.rk[1][w] = mx;
+  }
+  __syncthreads();
+  mn = S.rk[0][0];
+  mx = S.rk[1][0];
+  for (int j = 1; j < nw; ++j) {
+    mn = S.rk[0][j] < mn ? S.rk[0][j] : mn;
+    mx = S.rk[1][j] > mx ? S.rk[1][j] : mx;
+  }
+  __syncthreads();
+}
+
+constexpr int kStageKeys = 20480;  // replicates whose keys the select keeps in shared memory
+
+// Key of replicate i: from shared memory when staged, else recomputed from
+// global memory; 0 (no double's key) marks NaN.
+struct KeySrc {
+  const double* boot;
+  const unsigned long long* staged;  // or null
+  __device__ __forceinline__ unsigned long long at(long long i) const {
+    if (staged) return staged[i];
+    const double v = boot[i];
+    return (v == v) ? dkey(v) : 0ull;
+  }
+};
+
+__global__ void __launch_bounds__(kSelThreads) paired_select_kernel(const PairedParams p) {
+  __shared__ SelShared S;
+  extern __shared__ __align__(16) unsigned long long sk[];  // kStageKeys keys when staged
   wait_prior_grid();
-  const long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= p.n_boot) return;
-  const double se = p.boot[e];
-  const long long n = p.tot->n_valid;
-  if (se != se || n == 0) return;
-  const long long lo = p.less[e], hi = lo + p.eq[e];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  const long long B = p.n_boot;
+  const bool staged = B <= kStageKeys;
+  // the keys (staged), their range and count; loads four at a time
+  unsigned long long kmin = ~0ull, kmax = 0ull;
+  unsigned cnt = 0u;
+  for (long long i0 = tid; i0 < B; i0 += 4 * blockDim.x) {
+    double v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + (long long)u * blockDim.x;
+      v[u] = (i < B) ? p.boot[i] : CUDART_NAN;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + (long long)u * blockDim.x;
+      const unsigned long long k = (v[u] == v[u]) ? dkey(v[u]) : 0ull;
+      if (staged && i < B) sk[i] = k;
+      if (k) {
+        ++cnt;
+        kmin = k < kmin ? k : kmin;
+        kmax = k > kmax ? k : kmax;
+      }
+    }
+  }
+  block_key_range(kmin, kmax, S);  // its barriers also publish sk[]
+  cnt = __reduce_add_sync(0xffffffffu, cnt);
+  if (lane == 0) S.ru[w] = cnt;
+  __syncthreads();
+  long long n = 0;
+  for (int j = 0; j < nw; ++j) n += S.ru[j];
+  __syncthreads();
+  if (tid == 0) p.tot->n_valid = (unsigned)n;
+  if (n == 0) return;
+  const KeySrc src{p.boot, staged ? sk : nullptr};
+
   for (int t = 0; t < 2 * p.nq; ++t) {
-    const long long r = target_rank(p, n, t);
-    if (lo <= r && r < hi) p.tot->ostat[t] = se;
+    long long r = target_rank(p, n, t);  // rank among all non-NaN values
+    unsigned long long klo = kmin, khi = kmax;
+    unsigned long long ans;
+    for (;;) {
+      if (klo == khi) {  // one key left
+        ans = klo;
+        break;
+      }
+      const double scale = (double)kBuckets / ((double)(khi - klo) + 1.0);
+      for (int b = tid; b < kBuckets; b += blockDim.x) S.hist[b] = 0u;
+      if (tid == 0) S.n_gather = 0u;
+      __syncthreads();
+      for (long long i = tid; i < B; i += blockDim.x) {
+        const unsigned long long k = src.at(i);
+        if (k && k >= klo && k <= khi) atomicAdd(&S.hist[key_bucket(k, klo, scale)], 1u);
+      }
+      __syncthreads();
+      // the bucket holding rank r: every thread sums 4 buckets, a block scan
+      // of those sums, and the thread whose run holds r walks it
+      unsigned c4[4], run = 0u;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        c4[q] = S.hist[4 * tid + q];
+        run += c4[q];
+      }
+      unsigned incl = run;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      if (lane == 31) S.ru[w] = incl;
+      __syncthreads();
+      unsigned wbase = 0u;
+      for (int j = 0; j < w; ++j) wbase += S.ru[j];
+      const long long before_run = (long long)wbase + incl - run;
+      if (before_run <= r && r < before_run + (long long)run) {
+        long long acc = before_run;
+        int q = 0;
+        while (q < 3 && acc + (long long)c4[q] <= r) acc += c4[q++];
+        S.bucket = 4 * tid + q;
+        S.before = (unsigned)acc;
+      }
+      __syncthreads();
+      const int bk = (int)S.bucket;
+      const long long rr = r - (long long)S.before;  // rank inside the bucket
+      const unsigned in_bucket = S.hist[bk];
+      __syncthreads();
+      if (in_bucket <= (unsigned)kGather) {
+        for (long long i = tid; i < B; i += blockDim.x) {
+          const unsigned long long k = src.at(i);
+          if (k && k >= klo && k <= khi && key_bucket(k, klo, scale) == bk) S.gather[atomicAdd(&S.n_gather, 1u)] = k;
+        }
+        __syncthreads();
+        const int m = (int)S.n_gather;
+        if (tid < m) {
+          const unsigned long long k = S.gather[tid];
+          int less = 0, eq = 0;
+          for (int j = 0; j < m; ++j) {
+            const unsigned long long u = S.gather[j];
+            less += u < k;
+            eq += u == k;
+          }
+          if (less <= rr && rr < less + eq) S.answer = k;  // equal keys write the same value
+        }
+        __syncthreads();
+        ans = S.answer;
+        __syncthreads();
+        break;
+      }
+      // too many: the bucket's own least and greatest key become [klo, khi]
+      unsigned long long bmn = ~0ull, bmx = 0ull;
+      for (long long i = tid; i < B; i += blockDim.x) {
+        const unsigned long long k = src.at(i);
+        if (k && k >= klo && k <= khi && key_bucket(k, klo, scale) == bk) {
+          bmn = k < bmn ? k : bmn;
+          bmx = k > bmx ? k : bmx;
+        }
+      }
+      block_key_range(bmn, bmx, S);
+      r = rr;
+      klo = bmn;
+      khi = bmx;
+    }
+    if (tid == 0) p.tot->ostat[t] = dval(ans);
+    __syncthreads();
   }
 }
 
@@ -424,8 +575,7 @@ size_t paired_workspace_bytes(int64_t n_ctx, int32_t n_clusters, int32_t n_boot)
   const size_t parts = (nc + kTotChunk - 1) / kTotChunk + 1;
   return align256(sizeof(PairedTotals)) + align256(sizeof(PairedPart) * parts) + 3 * align256(sizeof(double) * nc) +
          align256(sizeof(int32_t) * nc) +
-         align256(sizeof(double) * k) + align256(sizeof(long long) * k) + 2 * align256(sizeof(unsigned) * b) +
-         align256(sizeof(double) * b);
+         align256(sizeof(double) * k) + align256(sizeof(long long) * k) + align256(sizeof(double) * b);
 }
 
 cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
@@ -462,10 +612,6 @@ cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
   ws += align256(sizeof(double) * k);
   p.Nk = reinterpret_cast<long long*>(ws);
   ws += align256(sizeof(long long) * k);
-  p.less = reinterpret_cast<unsigned*>(ws);
-  ws += align256(sizeof(unsigned) * b);
-  p.eq = reinterpret_cast<unsigned*>(ws);
-  ws += align256(sizeof(unsigned) * b);
   p.boot = a.boot_stats ? a.boot_stats : reinterpret_cast<double*>(ws);
 
   cudaError_t e = cudaSuccess;
@@ -482,11 +628,23 @@ cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
     e = launch_dependent(paired_boot_kernel, dim3((unsigned)((b + kBootWarps - 1) / kBootWarps)),
                          dim3(kBootThreads), stream, p);
     if (e != cudaSuccess) return e;
-    const unsigned gx = (unsigned)((b + kThreads - 1) / kThreads);
-    const unsigned gy = (unsigned)((b + kRankTile - 1) / kRankTile);
-    e = launch_dependent(paired_count_kernel, dim3(gx, gy), dim3(kThreads), stream, p);
-    if (e != cudaSuccess) return e;
-    e = launch_dependent(paired_pick_kernel, dim3(gx), dim3(kThreads), stream, p);
+    {
+      // the staged keys need more than the default 48 KB of shared memory
+      static std::mutex mu;
+      static unsigned long long done = 0ull;
+      int dev = 0;
+      e = cudaGetDevice(&dev);
+      if (e != cudaSuccess) return e;
+      std::lock_guard<std::mutex> lock(mu);
+      if (dev >= 64 || !((done >> dev) & 1ull)) {
+        e = cudaFuncSetAttribute(paired_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(sizeof(unsigned long long) * kStageKeys));
+        if (e != cudaSuccess) return e;
+        if (dev < 64) done |= 1ull << dev;
+      }
+    }
+    const size_t smem = (b <= (size_t)kStageKeys) ? sizeof(unsigned long long) * b : 0;
+    e = launch_dependent_smem(paired_select_kernel, dim3(1), dim3(kSelThreads), smem, stream, p);
     if (e != cudaSuccess) return e;
   }
   return launch_dependent(paired_finish_kernel, dim3(1), dim3(32), stream, p, n_parts);

@@ -56,7 +56,8 @@ def compare(r, boot, want, quantiles=QS):
         assert close(g, w, dscale)
 
 
-@pytest.mark.parametrize("n_ctx,L,C,B", [(1, 1, 1, 1), (37, 53, 7, 300), (64, 129, 64, 257), (300, 31, 1, 100)])
+@pytest.mark.parametrize("n_ctx,L,C,B", [(1, 1, 1, 1), (37, 53, 7, 300), (64, 129, 64, 257), (300, 31, 1, 100),
+                                          (40, 12, 6, 25_000)])
 def test_against_oracle(cuda_device, n_ctx, L, C, B):
     d = W.paired_candidates(seed=90 + n_ctx, device=cuda_device, n_ctx=n_ctx, ctx_len=L, n_clusters=C,
                             n_boot=B)
@@ -129,3 +130,32 @@ def test_suite_size_sampled(cuda_device):
     vals = np.sort(boot)
     assert r["ci"] == [O.quantile_linear(vals, q)[0] for q in QS]
     assert r["ci"][0] < r["diff"] < r["ci"][1]
+
+
+def test_infinite_and_undefined_context_means(cuda_device):
+    """A context whose A mean is +inf (a position with infinite KL) gives
+    +inf replicates wherever its cluster is drawn; a context with +inf on
+    both sides has an undefined difference (NaN), which poisons the
+    replicates that draw it.  Counts and the exact percentiles still match
+    the oracle."""
+    d = W.paired_candidates(seed=93, device=cuda_device, n_ctx=30, ctx_len=20, n_clusters=10, n_boot=400)
+    d["kl_a"][2, 5] = float("inf")
+    d["kl_a"][17, 3] = float("inf")
+    d["kl_b"][17, 9] = float("inf")
+    qs = (0.0, 0.1, 0.5, 0.9, 1.0)
+    r, boot = run(d, quantiles=qs)
+    want = oracle(d, quantiles=qs)
+    assert np.isinf(boot).any() and np.isnan(boot).any()
+    for key in ("n_ctx", "n_pos", "n_boot"):
+        assert r[key] == want[key], key
+    ok = ~np.isnan(want["boot"])
+    assert np.array_equal(np.isnan(boot), ~ok)
+    fin = ok & np.isfinite(want["boot"])
+    assert np.array_equal(np.isinf(boot[ok]), np.isinf(want["boot"][ok]))
+    dscale = float(np.nanmax(np.abs(want["boot"][fin])))
+    assert np.all(np.abs(boot[fin] - want["boot"][fin]) <= 1e-12 * dscale)
+    vals = np.sort(boot[ok])
+    for q, g, wv in zip(qs, r["ci"], want["ci"]):
+        e = O.quantile_linear(vals, q)[0]
+        assert (g == e) or (math.isnan(g) and math.isnan(e))
+        assert (math.isnan(g) and math.isnan(wv)) or g == wv or abs(g - wv) <= 1e-12 * dscale
