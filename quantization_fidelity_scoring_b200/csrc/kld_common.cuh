@@ -21,6 +21,8 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <mutex>
+
 namespace kld {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -183,6 +185,22 @@ __device__ __forceinline__ void set_dev_status(int32_t* dev_status, int bits) {
 // wait_prior_grid() before touching memory the previous kernels use (the
 // wait returns at once when the kernel was launched the ordinary way).
 __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Raises a kernel's dynamic shared-memory limit (required above 48 KB) on
+// the current device, once per device and kernel.
+template <auto Kernel>
+inline cudaError_t allow_dynamic_smem(size_t bytes) {
+  static std::mutex mu;
+  static unsigned long long done = 0ull;  // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 64 && ((done >> dev) & 1ull)) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev < 64) done |= 1ull << dev;
+  return e;
+}
 
 template <typename... KArgs, typename... Args>
 cudaError_t launch_dependent_smem(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem_bytes,

@@ -23,8 +23,6 @@
 //   finish   one warp writes the result.
 #include <math_constants.h>
 
-#include <mutex>
-
 #include "kld_common.cuh"
 #include "launch.h"
 
@@ -628,21 +626,8 @@ cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
     e = launch_dependent(paired_boot_kernel, dim3((unsigned)((b + kBootWarps - 1) / kBootWarps)),
                          dim3(kBootThreads), stream, p);
     if (e != cudaSuccess) return e;
-    {
-      // the staged keys need more than the default 48 KB of shared memory
-      static std::mutex mu;
-      static unsigned long long done = 0ull;
-      int dev = 0;
-      e = cudaGetDevice(&dev);
-      if (e != cudaSuccess) return e;
-      std::lock_guard<std::mutex> lock(mu);
-      if (dev >= 64 || !((done >> dev) & 1ull)) {
-        e = cudaFuncSetAttribute(paired_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(sizeof(unsigned long long) * kStageKeys));
-        if (e != cudaSuccess) return e;
-        if (dev < 64) done |= 1ull << dev;
-      }
-    }
+    e = allow_dynamic_smem<paired_select_kernel>(sizeof(unsigned long long) * kStageKeys);
+    if (e != cudaSuccess) return e;
     const size_t smem = (b <= (size_t)kStageKeys) ? sizeof(unsigned long long) * b : 0;
     e = launch_dependent_smem(paired_select_kernel, dim3(1), dim3(kSelThreads), smem, stream, p);
     if (e != cudaSuccess) return e;

@@ -24,8 +24,6 @@
 // what the shards exchange.
 #include <math_constants.h>
 
-#include <mutex>
-
 #include "kld_common.cuh"
 #include "launch.h"
 
@@ -902,21 +900,6 @@ ReduceParams make_params(const ReduceArgs& a) {
   return p;
 }
 
-// Kernels that take more than 48 KB of dynamic shared memory must say so,
-// once per device.
-template <typename Kernel>
-cudaError_t allow_smem(Kernel kernel, size_t bytes, unsigned long long* done_mask) {
-  static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(mu);
-  if (dev < 64 && ((*done_mask >> dev) & 1ull)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess && dev < 64) *done_mask |= 1ull << dev;
-  return e;
-}
-
 // Cooperative grid for n positions: about eight positions per thread, at
 // most as many CTAs as can be resident at once.
 cudaError_t coop_grid(long long n, int* grid) {
@@ -968,14 +951,12 @@ size_t reduce_shard_workspace_bytes(int64_t n) {
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t stream) {
   const ReduceParams p = make_params(a);
   if (a.n <= kSmallN) {
-    static unsigned long long small_ok = 0;
-    cudaError_t e = allow_smem(reduce_small_kernel, kSmallSmemMax, &small_ok);
+    cudaError_t e = allow_dynamic_smem<reduce_small_kernel>(kSmallSmemMax);
     if (e != cudaSuccess) return e;
     return launch_dependent_smem(reduce_small_kernel, dim3(1), dim3(kSmallThreads), sizeof(uint32_t) * (size_t)a.n,
                                  stream, p);
   }
-  static unsigned long long coop_ok = 0;
-  cudaError_t e = allow_smem(reduce_coop_kernel, kCoopSmem, &coop_ok);
+  cudaError_t e = allow_dynamic_smem<reduce_coop_kernel>(kCoopSmem);
   int grid = 0;
   if (e == cudaSuccess) e = coop_grid(a.n, &grid);
   if (e != cudaSuccess) return e;

@@ -447,8 +447,7 @@ cudaError_t launch_shared_head(const SharedHeadArgs& a, cudaStream_t stream) {
   int dev = 0, sms = 148;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  // opt in to the large dynamic shared memory (idempotent, per device)
-  e = cudaFuncSetAttribute(head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  e = allow_dynamic_smem<head_kernel>(kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = p.ntiles < sms ? p.ntiles : sms;
