@@ -306,6 +306,20 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(const MergeParams p) {
   const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld_x * kElemBytes;
   const char* yrow = reinterpret_cast<const char*>(p.y) + (int64_t)row * p.ld_y * kElemBytes;
 
+  // the target logits first: their two dependent loads overlap the merge
+  bool have_t = false, bad_t = false;
+  float xt = 0.f, yt = 0.f;
+  if (p.targets) {
+    const int tg = p.targets[row];
+    if (tg >= 0 && tg < p.vocab) {
+      have_t = true;
+      xt = El::load1(xrow, tg);
+      yt = El::load1(yrow, tg);
+    } else {
+      bad_t = true;
+    }
+  }
+
   RowState acc = row_empty();
   if (p.nvec > 0) {
     const int64_t f = (int64_t)row * p.nvec;
@@ -326,18 +340,7 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(const MergeParams p) {
     side_push(acc.y, yv, i, wy, scy, acc.bad);
     acc.A = acc.A * scx + wx * fmaxf(xv - yv, -FLT_MAX);
   }
-  bool have_t = false;
-  float xt = 0.f, yt = 0.f;
-  if (p.targets) {
-    const int tg = p.targets[row];
-    if (tg >= 0 && tg < p.vocab) {
-      have_t = true;
-      xt = El::load1(xrow, tg);
-      yt = El::load1(yrow, tg);
-    } else {
-      set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
-    }
-  }
+  if (bad_t) set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
   const RowOut o = row_finish(acc, have_t, xt, yt);
   p.kl[row] = o.kl;
   if (p.ax) p.ax[row] = o.ax;

@@ -330,6 +330,10 @@ __global__ void __launch_bounds__(256) head_merge_kernel(const HeadParams p, flo
   const int lane = threadIdx.x & 31;
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (row >= p.n_rows) return;
+  // the target logits first: their loads overlap the merge
+  const int tg = p.targets ? p.targets[row] : -1;
+  const bool have_t = p.targets && tg >= 0 && tg < p.vocab;
+  const float2 t2 = have_t ? p.tv[row] : make_float2(0.f, 0.f);
   RowState acc = row_empty();
   for (int c = 0; c < p.nt; c += 32) {
     const int t = c + lane;
@@ -345,20 +349,8 @@ __global__ void __launch_bounds__(256) head_merge_kernel(const HeadParams p, flo
     acc = (c == 0) ? s : row_merge(acc, s);
   }
   if (lane != 0) return;
-  bool have_t = false;
-  float xt = 0.f, yt = 0.f;
-  if (p.targets) {
-    const int tg = p.targets[row];
-    if (tg >= 0 && tg < p.vocab) {
-      have_t = true;
-      const float2 t2 = p.tv[row];
-      xt = t2.x;
-      yt = t2.y;
-    } else {
-      set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
-    }
-  }
-  const RowOut o = row_finish(acc, have_t, xt, yt);
+  if (p.targets && !have_t) set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
+  const RowOut o = row_finish(acc, have_t, t2.x, t2.y);
   kl[row] = o.kl;
   if (ax) ax[row] = o.ax;
   if (ay) ay[row] = o.ay;

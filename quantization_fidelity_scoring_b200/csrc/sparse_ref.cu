@@ -398,6 +398,10 @@ __global__ void __launch_bounds__(kMergeThreads) sparse_merge_kernel(const Merge
   const float* gy = p.gy + (int64_t)row * p.K;
   float* ysw = ys[wl];
   float* lpw = lps[wl];
+  // the target logit first: its two dependent loads overlap the merge
+  const int tgt = p.lp_cand ? p.targets[row] : -1;
+  const bool tgt_ok = tgt >= 0 && tgt < p.vocab;
+  const float y_tgt = (p.lp_cand && tgt_ok) ? El::load1(yrow, tgt) : 0.f;
   const int64_t listed_end = (int64_t)p.nvec * E;  // ids below this were captured by the stream
 
   // tail state of the unlisted ids covered by the stream
@@ -507,9 +511,8 @@ __global__ void __launch_bounds__(kMergeThreads) sparse_merge_kernel(const Merge
   if (p.top1) p.top1[row] = (uint8_t)(valid && top[0].x == am);
   if (p.lp_cand) {
     float lpc = CUDART_NAN_F;
-    const int t = p.targets[row];
-    if (t >= 0 && t < p.vocab) {
-      if (valid) lpc = (float)(((double)El::load1(yrow, t) - (double)m) - logS);
+    if (tgt_ok) {
+      if (valid) lpc = (float)(((double)y_tgt - (double)m) - logS);
     } else {
       set_dev_status(p.dev_status, 0x1 /* KLD_DEV_BAD_TARGET */);
     }
