@@ -236,11 +236,13 @@ def run_reference(args) -> int:
     return 0
 
 
-def config_dict(rows: int = N_ROWS, world: int = 1) -> dict:
+def config_dict(rows: int = N_ROWS, world: int = 1, pipelined: bool = False) -> dict:
     workload = WORKLOAD if rows == N_ROWS else WORKLOAD.replace("2047 positions", f"{rows} positions") + \
         " (reduced profiling case)"
     return {"workload": workload, "n_rows": rows, "vocab": VOCAB, "input_dtype": "bf16",
-            "step": "kld_full_vocab + kld_reduce_stats (mean, p50, p99, p99.9, top-1, ppl)",
+            "step": "kld_full_vocab + kld_reduce_stats (mean, p50, p99, p99.9, top-1, ppl)" +
+                    ("; each window's statistics on a second stream, overlapping the next window's scoring"
+                     if pipelined else ""),
             "l2": f"inputs larger than L2: {2 * rows * VOCAB * 2 / 1e9:.2f} GB of logits per step",
             "parallelism": "dp (each rank scores its own window)" if world == 1 else
             f"dp{world}: each rank scores its own window; the statistics cover all ranks' positions "
@@ -266,35 +268,61 @@ def run_ours(args) -> int:
     ref, cand, targets = d["ref"], d["cand"], d["targets"]
     n = ref.shape[0]
     stream = torch.cuda.current_stream()
-    kl = torch.empty(n, dtype=torch.float32, device=dev)
-    ra = torch.empty(n, dtype=torch.int32, device=dev)
-    ca = torch.empty(n, dtype=torch.int32, device=dev)
-    lpr = torch.empty(n, dtype=torch.float32, device=dev)
-    lpc = torch.empty(n, dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    ws = torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev)
     fws = torch.empty(kq.kld_full_vocab_workspace_size(n), dtype=torch.uint8, device=dev)
-    stats_buf = torch.empty(280, dtype=torch.uint8, device=dev)
+
+    def outputs():
+        return dict(kl=torch.empty(n, dtype=torch.float32, device=dev),
+                    ra=torch.empty(n, dtype=torch.int32, device=dev),
+                    ca=torch.empty(n, dtype=torch.int32, device=dev),
+                    lpr=torch.empty(n, dtype=torch.float32, device=dev),
+                    lpc=torch.empty(n, dtype=torch.float32, device=dev),
+                    ws=torch.empty(kq.kld_reduce_workspace_size(n), dtype=torch.uint8, device=dev),
+                    stats=torch.empty(280, dtype=torch.uint8, device=dev))
+
+    # With one GPU the statistics of window i run on a second stream while
+    # window i + 1 is scored: the per-position outputs are double-buffered,
+    # and events keep a buffer from being rewritten before its statistics
+    # have read it.  (--serial runs them one after the other.)
+    pipelined = world == 1 and not args.serial
+    bufs = [outputs(), outputs()] if pipelined else [outputs()]
+    side = torch.cuda.Stream(device=dev) if pipelined else stream
+    scored = [torch.cuda.Event(), torch.cuda.Event()]
+    reduced = [torch.cuda.Event(), torch.cuda.Event()]
+    for e in reduced:
+        e.record(side)
+    count = [0]
 
     if world > 1:
         from quantization_fidelity_scoring_b200 import shards
         sws = torch.empty(kq.kld_reduce_shard_workspace_size(n), dtype=torch.uint8, device=dev)
 
     def step(ev=None):
+        i = count[0] % len(bufs)
+        count[0] += 1
+        o = bufs[i]
+        if pipelined:
+            stream.wait_event(reduced[i])  # this buffer's previous statistics are done
         if ev is not None:
             ev[0].record(stream)
-        kq.kld_full_vocab(ref, cand, targets, kl=kl, ref_argmax=ra, cand_argmax=ca, ref_target_lp=lpr,
-                          cand_target_lp=lpc, workspace=fws, dev_status=status, stream=stream)
+        kq.kld_full_vocab(ref, cand, targets, kl=o["kl"], ref_argmax=o["ra"], cand_argmax=o["ca"],
+                          ref_target_lp=o["lpr"], cand_target_lp=o["lpc"], workspace=fws, dev_status=status,
+                          stream=stream)
         if ev is not None:
             ev[1].record(stream)
         if world > 1:
             # the statistics of every rank's positions: shard steps with an
             # all-gather of each step's 16.5 KB block
-            shards.reduce_stats_across_ranks(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf,
-                                             workspace=sws, dev_status=status, to_host=False)
+            shards.reduce_stats_across_ranks(o["kl"], o["ra"], o["ca"], None, o["lpr"], o["lpc"], None, QUANTILES,
+                                             (), out=o["stats"], workspace=sws, dev_status=status, to_host=False)
         else:
-            kq.kld_reduce_stats(kl, ra, ca, None, lpr, lpc, None, QUANTILES, (), out=stats_buf,
-                                workspace=ws, dev_status=status, stream=stream, to_host=False)
+            if pipelined:
+                scored[i].record(stream)
+                side.wait_event(scored[i])
+            kq.kld_reduce_stats(o["kl"], o["ra"], o["ca"], None, o["lpr"], o["lpc"], None, QUANTILES, (),
+                                out=o["stats"], workspace=o["ws"], dev_status=status, stream=side, to_host=False)
+            if pipelined:
+                reduced[i].record(side)
 
     sampler = ClockSampler(local).start()
     # warm-up: at least W steps and about a second of load so the clocks settle
@@ -318,6 +346,7 @@ def run_ours(args) -> int:
     start.record(stream)
     for s in range(args.steps):
         step(kev[s])
+    stream.wait_stream(side)  # the last window's statistics are inside the timed region
     stop.record(stream)
     torch.cuda.synchronize()
     t1 = time.perf_counter()
@@ -353,7 +382,7 @@ def run_ours(args) -> int:
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded Zipf/Gumbel logits; no corpus or model)",
-            "config": config_dict(args.rows, world), "roofline": roofline,
+            "config": config_dict(args.rows, world, pipelined), "roofline": roofline,
             "clocks": sampler.summary(t0, t1), "gpu_launches": launches_per_step(n, world) * args.steps,
             "e2e": e2e,
         }
@@ -833,6 +862,8 @@ def main(argv=None) -> int:
     ap.add_argument("--ref-seconds", type=float, default=90.0,
                     help="reference arm: CPU seconds the timed and warm-up steps aim for")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serial", action="store_true",
+                    help="run each window's statistics after its scoring on one stream (no overlap)")
     ap.add_argument("--no-extra", action="store_true", help="skip the top-64 and shared-head lines")
     ap.add_argument("--profile-topk", type=int, metavar="WINDOWS",
                     help="only time the top-64 + tail path on WINDOWS windows (for profiling)")
