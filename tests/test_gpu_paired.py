@@ -57,7 +57,7 @@ def compare(r, boot, want, quantiles=QS):
 
 
 @pytest.mark.parametrize("n_ctx,L,C,B", [(1, 1, 1, 1), (37, 53, 7, 300), (64, 129, 64, 257), (300, 31, 1, 100),
-                                          (40, 12, 6, 25_000)])
+                                          (40, 12, 6, 25_000), (3000, 5, 2500, 150), (9000, 3, 40, 60)])
 def test_against_oracle(cuda_device, n_ctx, L, C, B):
     d = W.paired_candidates(seed=90 + n_ctx, device=cuda_device, n_ctx=n_ctx, ctx_len=L, n_clusters=C,
                             n_boot=B)

@@ -51,7 +51,7 @@ def compare(st, want):
             assert abs(st[key] - want[key]) <= 1e-12 * abs(want[key])
 
 
-@pytest.mark.parametrize("n", [1, 2, 3, 100, 2047, 65536, 65537, 300_001, 1_048_064])
+@pytest.mark.parametrize("n", [1, 2, 3, 100, 2047, 8192, 8193, 65536, 65537, 300_001, 1_048_064, 5_000_000])
 def test_against_oracle(cuda_device, n):
     kl, ra, ca, lr, lc, mask = make(n, seed=n, nan_every=53)
     T = lambda a: torch.tensor(a, device=cuda_device)
