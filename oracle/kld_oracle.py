@@ -26,7 +26,7 @@ Sources (web pages, cited by title and section):
 * "Qwen3.8-27B IQ8R (GPTQ int8, Hadamard-rotated) - radiance container",
   section "Quality" (mean KLD, KLD 99%, KLD 99.9%, top-1 agreement).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * Natural logarithms (entropy is reported in nats).
 * 0 * log 0 = 0: vocabulary entries with p_i = 0 contribute nothing.
