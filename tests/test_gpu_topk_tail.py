@@ -40,12 +40,29 @@ def test_full_size_windows(cuda_device):
     assert 0.85 < want["n_matched"].mean() / 64 < 0.95
 
 
-@pytest.mark.parametrize("k", [1, 2, 31, 32, 33, 63, 64])
+@pytest.mark.parametrize("k", [1, 2, 8, 16, 31, 32, 33, 40, 63, 64])
 def test_list_lengths(cuda_device, k):
     d = W.topk_tail_windows(seed=W.SEED_BASE + 600 + k, device=cuda_device, windows=3, positions=257,
                             vocab=50_000, k=k, sigma=0.3)
     res = run(d["ref_ids"], d["ref_lp"], d["cand_ids"], d["cand_lp"], 50_000)
     check(res, d["ref_ids"], d["ref_lp"], d["cand_ids"], d["cand_lp"], 50_000)
+
+
+def test_unaligned_rows(cuda_device):
+    """k = 64 lists that start 4 bytes (ids) and 2 bytes (log-probs) past a
+    16-byte boundary take the element-load path: same results as the oracle."""
+    d = W.topk_tail_windows(seed=W.SEED_BASE + 650, device=cuda_device, windows=2, positions=301,
+                            vocab=50_000, k=64, sigma=0.3)
+    shifted = []
+    for name in ("ref_ids", "ref_lp", "cand_ids", "cand_lp"):
+        a = d[name].reshape(-1, 64)
+        buf = torch.empty(a.numel() + 8, dtype=a.dtype, device=cuda_device)
+        view = buf[1:1 + a.numel()].view(a.shape)
+        view.copy_(a)
+        assert view.data_ptr() % 16 != 0
+        shifted.append(view)
+    res = run(*shifted, 50_000)
+    check(res, *shifted, 50_000)
 
 
 def test_small_vocab_brute_force_cases(cuda_device):
