@@ -136,6 +136,24 @@ __device__ void ring_flush(const CapParams& p, CapRing& R, int fill, int row, fl
 
 // 2. stream vectors [a, b) of one row; returns the piece's tail state
 // (identical in every lane) and appends the piece's candidates.
+// 1.0f when a >= b, else 0.0f (NaN compares false).
+__device__ __forceinline__ float set_ge(float a, float b) {
+  float r;
+  asm("set.ge.f32.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+// Both bf16 halves of w raised to at least the lowest finite bf16; NaN stays.
+__device__ __forceinline__ uint32_t bf16x2_floor(uint32_t w) {
+  uint32_t r;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(w), "r"(0xff7fff7fu));
+  return r;
+}
+
+// Shift that takes a candidate's exponent far below any real one: its
+// weight underflows to exactly 0.
+constexpr float kMaskShift = 1e30f;
+
 template <bool kBF16>
 __device__ CapPiece cap_piece(const CapParams& p, CapRing& R, int row, int a, int b, int lane, float tau) {
   using El = Elems<kBF16>;
@@ -224,19 +242,31 @@ __device__ CapPiece cap_piece(const CapParams& p, CapRing& R, int row, int a, in
     const float mo = (m == -CUDART_INF_F) ? 0.f : m;
     const float2 nm = make_float2(-mo, -mo);
     const float2 l2 = make_float2(kLog2e, kLog2e);
+    const float2 shove = make_float2(-kMaskShift, -kMaskShift);
 #pragma unroll
     for (int q = 0; q < kVecs; ++q) {
+      uint4 u = v[q];
+      if constexpr (kBF16) {
+        // -inf -> the lowest finite bf16 (NaN kept), so d below is finite
+        // and w * d never forms 0 * inf; its weight is exactly 0 either way
+        u.x = bf16x2_floor(u.x);
+        u.y = bf16x2_floor(u.y);
+        u.z = bf16x2_floor(u.z);
+        u.w = bf16x2_floor(u.w);
+      }
 #pragma unroll
       for (int k = 0; k < E / 2; ++k) {
-        const float2 X = El::pair(v[q], k);
+        const float2 X = El::pair(u, k);
         float2 d = __fadd2_rn(X, nm);
-        if (X.x >= tau) d.x = -CUDART_INF_F;
-        if (X.y >= tau) d.y = -CUDART_INF_F;
-        const float2 t = __fmul2_rn(d, l2);
+        // a candidate (X >= tau) is pushed far below the maximum: weight 0
+        const float2 c = make_float2(set_ge(X.x, tau), set_ge(X.y, tau));
+        const float2 t = __fmul2_rn(__ffma2_rn(c, shove, d), l2);
         const float2 w = make_float2(ex2(t.x), ex2(t.y));
         T2 = __fadd2_rn(T2, w);
-        d.x = fmaxf(d.x, -FLT_MAX);
-        d.y = fmaxf(d.y, -FLT_MAX);
+        if constexpr (!kBF16) {
+          d.x = fmaxf(d.x, -FLT_MAX);
+          d.y = fmaxf(d.y, -FLT_MAX);
+        }
         B2 = __ffma2_rn(w, d, B2);
       }
     }
@@ -384,11 +414,16 @@ struct FinScratch {  // block-reduction slots for up to 8 warps
 // rank among them (eq - rank of the equal keys come after position r); rank
 // is 0 when fewer than r elements take part.
 // Every thread of the CTA calls this.
-template <class KeyFn>
+// kLowBits: the keys' low kLowBits bits are fixed by the sign bit (all 0 for
+// a positive value, all 1 for a negative one), as for the key of a bf16 value
+// widened to f32; the passes over them, which would put every remaining
+// element into one bin, are skipped and the bits filled in.
+template <int kLowBits, class KeyFn>
 __device__ uint32_t rth_largest(int n, int r, KeyFn key, FinScratch& sc, int& eq, int& rank) {
+  static_assert(kLowBits == 0 || kLowBits == 16, "whole 8-bit digits, the sign digit always scanned");
   const int lane = threadIdx.x & 31;
   uint32_t prefix = 0u, pmask = 0u;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int shift = 24; shift >= kLowBits; shift -= 8) {
     for (int b = threadIdx.x; b < 256; b += blockDim.x) sc.hist[b] = 0u;
     __syncthreads();
     for (int i0 = threadIdx.x & ~31; i0 < n; i0 += blockDim.x) {  // warp-uniform trip count
@@ -443,6 +478,7 @@ __device__ uint32_t rth_largest(int n, int r, KeyFn key, FinScratch& sc, int& eq
     pmask |= 255u << shift;
     r = (int)sc.rank;
   }
+  if (kLowBits > 0 && r > 0 && !(prefix & 0x80000000u)) prefix |= (1u << kLowBits) - 1u;
   eq = (int)sc.eq;
   rank = r;
   return prefix;
@@ -548,7 +584,7 @@ __global__ void __launch_bounds__(kSampleThreads) cap_sample_kernel(const CapPar
   tmax[threadIdx.x] = mx;
   __syncthreads();
   int eq = 0, rank = 0;
-  const uint32_t kk = rth_largest(kSampleThreads, kSampleRank, [&](int i, uint32_t& k) {
+  const uint32_t kk = rth_largest<kBF16 ? 16 : 0>(kSampleThreads, kSampleRank, [&](int i, uint32_t& k) {
     const float v = tmax[i];
     k = vkey(v);
     return v == v;  // NaN (an invalid row) takes no part
@@ -597,14 +633,14 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
   // the K-th largest value, and which of the values tied with it join
   // (the lowest ids first): pre, then ids up to id_cut among the ties
   int eq = 0, need = 0;
-  const uint32_t pre = rth_largest(n, K, [&](int i, uint32_t& k) {
+  const uint32_t pre = rth_largest<kBF16 ? 16 : 0>(n, K, [&](int i, uint32_t& k) {
     k = vkey(src.val(i));
     return true;
   }, sc, eq, need);
   uint32_t id_cut = 0xffffffffu;
   if (need < eq) {
     int eq2 = 0, r2 = 0;
-    id_cut = ~rth_largest(n, need, [&](int i, uint32_t& k) {
+    id_cut = ~rth_largest<0>(n, need, [&](int i, uint32_t& k) {
       k = ~(uint32_t)src.idx(i);
       return vkey(src.val(i)) == pre;
     }, sc, eq2, r2);

@@ -94,11 +94,12 @@ def test_full_size_window_sampled_rows(cuda_device):
     assert torch.all(torch.abs(mass - 1.0) < 1e-5)
 
 
-def test_ties_nonfinite_and_bad_target(cuda_device):
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_ties_nonfinite_and_bad_target(cuda_device, dtype):
     V, k = 70_001, 64
     d = W.window_full_vocab(seed=W.SEED_BASE + 3100, device=cuda_device, n_rows=8, vocab=70_008,
                             dtype=torch.float32)
-    x = padded(d["ref"][:, :V].contiguous(), 4)
+    x = padded(d["ref"][:, :V].contiguous().to(dtype), 8 if dtype == torch.bfloat16 else 4)
     tg = torch.remainder(d["targets"], V).to(torch.int32)
     x[0] = 1.5                                      # every logit equal: the k lowest ids
     x[1, ::3] = x[1].max() + 1.0                    # 23,334 ties at the top: more than the buffer
