@@ -314,13 +314,19 @@ constexpr int kSelThreads = 1024;
 constexpr int kBuckets = 4096;
 constexpr int kGather = 1024;
 
+constexpr int kSelTargets = 2 * KLD_MAX_QUANTILES;
+
 struct SelShared {
   unsigned hist[kBuckets];
   unsigned long long gather[kGather];
+  int gather_bucket[kGather];
+  unsigned picked[kBuckets / 32];  // buckets gathered by the shared first round
   unsigned long long rk[2][32];
   unsigned ru[32];
   unsigned long long answer;
   unsigned n_gather, bucket, before;
+  unsigned t_bucket[kSelTargets], t_before[kSelTargets];
+  unsigned long long t_answer[kSelTargets];
 };
 
 __device__ __forceinline__ unsigned long long dkey(double v) {
@@ -416,8 +422,111 @@ __global__ void __launch_bounds__(kSelThreads) paired_select_kernel(const Paired
   if (tid == 0) p.tot->n_valid = (unsigned)n;
   if (n == 0) return;
   const KeySrc src{p.boot, staged ? sk : nullptr};
+  const int nt = 2 * p.nq;
 
-  for (int t = 0; t < 2 * p.nq; ++t) {
+  // Shared first round: one histogram over [kmin, kmax] serves every target;
+  // the buckets holding the targets' ranks are gathered together while they
+  // fit the gather buffer, and each target is ranked inside its bucket.
+  // A target whose bucket does not fit runs the narrowing loop below alone.
+  unsigned done = 0u;  // targets answered here (the same in every thread)
+  if (kmin == kmax) {
+    if (tid == 0)
+      for (int t = 0; t < nt; ++t) S.t_answer[t] = kmin;
+    done = (1u << nt) - 1u;
+    __syncthreads();
+  } else {
+    const double scale = (double)kBuckets / ((double)(kmax - kmin) + 1.0);
+    for (int b = tid; b < kBuckets; b += blockDim.x) S.hist[b] = 0u;
+    for (int b = tid; b < kBuckets / 32; b += blockDim.x) S.picked[b] = 0u;
+    if (tid == 0) S.n_gather = 0u;
+    __syncthreads();
+    for (long long i = tid; i < B; i += blockDim.x) {
+      const unsigned long long k = src.at(i);
+      if (k) atomicAdd(&S.hist[key_bucket(k, kmin, scale)], 1u);
+    }
+    __syncthreads();
+    unsigned c4[4], run = 0u;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      c4[q] = S.hist[4 * tid + q];
+      run += c4[q];
+    }
+    unsigned incl = run;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const unsigned o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) S.ru[w] = incl;
+    __syncthreads();
+    unsigned wbase = 0u;
+    for (int j = 0; j < w; ++j) wbase += S.ru[j];
+    const long long before_run = (long long)wbase + incl - run;
+    for (int t = 0; t < nt; ++t) {
+      const long long r = target_rank(p, n, t);
+      if (before_run <= r && r < before_run + (long long)run) {
+        long long acc = before_run;
+        int q = 0;
+        while (q < 3 && acc + (long long)c4[q] <= r) acc += c4[q++];
+        S.t_bucket[t] = 4 * tid + q;
+        S.t_before[t] = (unsigned)acc;
+      }
+    }
+    __syncthreads();
+    // which targets' buckets fit together (every thread decides alike)
+    unsigned total = 0u;
+    for (int t = 0; t < nt; ++t) {
+      const unsigned bk = S.t_bucket[t];
+      bool seen = false;
+      for (int u = 0; u < t; ++u) seen |= ((done >> u) & 1u) && S.t_bucket[u] == bk;
+      if (seen) {
+        done |= 1u << t;
+      } else if (total + S.hist[bk] <= (unsigned)kGather) {
+        total += S.hist[bk];
+        done |= 1u << t;
+        if (tid == 0) S.picked[bk >> 5] |= 1u << (bk & 31);
+      }
+    }
+    __syncthreads();
+    if (done) {
+      for (long long i = tid; i < B; i += blockDim.x) {
+        const unsigned long long k = src.at(i);
+        if (!k) continue;
+        const int b = key_bucket(k, kmin, scale);
+        if ((S.picked[b >> 5] >> (b & 31)) & 1u) {
+          const unsigned at = atomicAdd(&S.n_gather, 1u);
+          S.gather[at] = k;
+          S.gather_bucket[at] = b;
+        }
+      }
+      __syncthreads();
+      const int m = (int)S.n_gather;
+      for (int t = 0; t < nt; ++t) {
+        if (!((done >> t) & 1u)) continue;
+        const int bk = (int)S.t_bucket[t];
+        const long long rr = target_rank(p, n, t) - (long long)S.t_before[t];  // rank inside the bucket
+        for (int g = tid; g < m; g += blockDim.x) {
+          if (S.gather_bucket[g] != bk) continue;
+          const unsigned long long k = S.gather[g];
+          int less = 0, eq = 0;
+          for (int j = 0; j < m; ++j) {
+            if (S.gather_bucket[j] != bk) continue;
+            const unsigned long long u = S.gather[j];
+            less += u < k;
+            eq += u == k;
+          }
+          if (less <= rr && rr < less + eq) S.t_answer[t] = k;  // equal keys write the same value
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  for (int t = 0; t < nt; ++t) {
+    if ((done >> t) & 1u) {
+      if (tid == 0) p.tot->ostat[t] = dval(S.t_answer[t]);
+      continue;
+    }
     long long r = target_rank(p, n, t);  // rank among all non-NaN values
     unsigned long long klo = kmin, khi = kmax;
     unsigned long long ans;

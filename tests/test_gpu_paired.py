@@ -65,6 +65,19 @@ def test_against_oracle(cuda_device, n_ctx, L, C, B):
     compare(r, boot, oracle(d))
 
 
+def test_crowded_interval_buckets(cuda_device):
+    """One context far above the rest makes its cluster dominate every
+    replicate that draws it: the replicates bunch into a few narrow bands of
+    a wide range, so the buckets holding the interval ends overflow the
+    gather buffer and the select narrows them; 25,000 replicates also leave
+    the keys unstaged."""
+    d = W.paired_candidates(seed=93, device=cuda_device, n_ctx=400, ctx_len=16, n_clusters=40, n_boot=25_000)
+    d["kl_a"][5] += 1e6
+    for q in ((0.025, 0.975), (0.0, 0.3, 0.5, 0.7, 1.0)):
+        r, boot = run(d, quantiles=q)
+        compare(r, boot, oracle(d, quantiles=q), quantiles=q)
+
+
 def test_mask_and_nan(cuda_device):
     d = W.paired_candidates(seed=95, device=cuda_device, n_ctx=41, ctx_len=77, n_clusters=9, n_boot=211)
     d["kl_a"][3, ::5] = float("nan")
