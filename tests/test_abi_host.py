@@ -13,7 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_functions():
-    src = open(os.path.join(ROOT, "include", "kld.h")).read()
+    with open(os.path.join(ROOT, "include", "kld.h")) as f:
+        src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     names = re.findall(r"\b(kld_[a-z0-9_]+)\s*\(", src)
     return sorted(set(names))

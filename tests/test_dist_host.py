@@ -50,7 +50,7 @@ def _rank_main(rank, world, port, out_dir):
 def test_two_gloo_ranks_agree_on_slowest_time(tmp_path):
     world, port = 2, free_port()
     mp.start_processes(_rank_main, args=(world, port, str(tmp_path)), nprocs=world, start_method="spawn")
-    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    res = [json.loads((tmp_path / f"rank{r}.json").read_text()) for r in range(world)]
     for r, x in enumerate(res):
         assert x["env"] == [world, r, r]
         assert x["max"] == 2.5                       # the slowest rank, on every rank
@@ -123,5 +123,5 @@ def test_shard_exchange_two_gloo_ranks(tmp_path):
     world, port = 2, free_port()
     mp.start_processes(_shard_main, args=(world, port, str(tmp_path)), nprocs=world, start_method="spawn")
     for r in range(world):
-        res = json.load(open(tmp_path / f"shard{r}.json"))
+        res = json.loads((tmp_path / f"shard{r}.json").read_text())
         assert res["seen"] == [1, 2, 3, 4] and res["out"] == 7

@@ -630,7 +630,8 @@ def test_pin(pin):
 def test_golden_bf16_self_scores():
     """Reference vs itself: mean KLD 0 and top-1 agreement 100% (golden)."""
     path = os.path.join(ROOT, "tests", "golden", "bf16_self_scores.txt")
-    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    with open(path) as f:
+        rows = [ln.split() for ln in f if ln.strip() and not ln.startswith("#")]
     mean_kld, top1 = float(rows[0][0]), float(rows[0][1])
     rng = np.random.default_rng(12)
     X = rng.normal(0, 2, (16, 4096))
@@ -696,7 +697,8 @@ MUTANTS = [
 
 
 def _load_mutant(old, new):
-    src = open(ORACLE_SRC).read()
+    with open(ORACLE_SRC) as f:
+        src = f.read()
     assert src.count(old) == 1, f"mutant anchor not unique / missing: {old!r}"
     spec = importlib.util.spec_from_loader("oracle_mutant", loader=None)
     mod = importlib.util.module_from_spec(spec)
