@@ -55,10 +55,11 @@ def profiled_traffic():
     if not os.path.exists(PROFILE):
         return None
     vals = {}
-    for line in open(PROFILE):
-        if ":" in line:
-            k, v = line.split(":", 1)
-            vals[k.strip()] = v.strip()
+    with open(PROFILE) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
     if vals.get("kernel_source_digest") != kernel_digest():
         return None
     try:
