@@ -388,11 +388,13 @@ def run_ours(args) -> int:
             "e2e": e2e,
         }
         if not args.no_extra:
+            # the latency-bound paths before the seconds-long GEMM loop, whose
+            # power-capped clocks would otherwise linger into their timing
             line["extra_paths"] = {"topk_tail": measure_topk(args, kq, dev),
                                    "sparse_ref": measure_sparse_ref(args, kq, dev),
                                    "sparse_capture": measure_sparse_capture(args, kq, dev),
-                                   "shared_head": measure_shared_head(args, kq, dev),
                                    "paired": measure_paired(args, kq, dev),
+                                   "shared_head": measure_shared_head(args, kq, dev),
                                    "batched_f32": measure_batched(args, kq, dev)}
             torch.cuda.empty_cache()
         if world == 1 and not args.no_cpu_baseline:
