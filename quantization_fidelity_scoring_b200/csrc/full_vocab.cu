@@ -200,14 +200,15 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
     r.y1 = ld_stream(yl + o + 32 * 16);
   };
   auto step = [&](const StepRaw& cur, int st) {
-    const float cx0 = El::vmax(cur.x0), cx1 = El::vmax(cur.x1);
-    const float cy0 = El::vmax(cur.y0), cy1 = El::vmax(cur.y1);
-    const float CMX = warp_max(fmaxf(cx0, cx1));
-    const float CMY = warp_max(fmaxf(cy0, cy1));
+    const float CMX = warp_max(El::vmax2(cur.x0, cur.x1));
+    const float CMY = warp_max(El::vmax2(cur.y0, cur.y1));
     if (!((CMX > sx.m) || (CMY > sy.m) || (sx.a < 0) || (sy.a < 0))) {  // warp-uniform
       accumulate<kBF16, false>(cur, sx.m, sy.m, -1, -1, rx2, ry2, a2);
       return;
     }
+    // the per-vector maxima locate a new maximum (rare: computed only here)
+    const float cx0 = El::vmax(cur.x0), cx1 = El::vmax(cur.x1);
+    const float cy0 = El::vmax(cur.y0), cy1 = El::vmax(cur.y1);
     // a new maximum on either side, or a side still without a finite value:
     // fold the paired sums, move to the new maxima, weigh with the new
     // argmaxes masked out of r

@@ -43,6 +43,19 @@ struct Elems<true> {
     asm("max.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(a), "r"(b));
     return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xffff0000u));
   }
+  // Largest of the 16 elements of two vectors (NaN only if all are NaN,
+  // as for vmax).
+  __device__ __forceinline__ static float vmax2(const uint4& v, const uint4& w) {
+    uint32_t a, b, c, d, e, f, m;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(v.x), "r"(v.y));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(b) : "r"(v.z), "r"(v.w));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(w.x), "r"(w.y));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(w.z), "r"(w.w));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(e) : "r"(a), "r"(b));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(f) : "r"(c), "r"(d));
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(e), "r"(f));
+    return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xffff0000u));
+  }
   __device__ __forceinline__ static float load1(const void* base, int64_t i) {
     const unsigned short b = reinterpret_cast<const unsigned short*>(base)[i];
     return __uint_as_float(static_cast<uint32_t>(b) << 16);
@@ -59,6 +72,9 @@ struct Elems<false> {
   __device__ __forceinline__ static float vmax(const uint4& v) {
     return fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)),
                  fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
+  }
+  __device__ __forceinline__ static float vmax2(const uint4& v, const uint4& w) {
+    return fmaxf(vmax(v), vmax(w));
   }
   __device__ __forceinline__ static float load1(const void* base, int64_t i) {
     return reinterpret_cast<const float*>(base)[i];
