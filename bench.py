@@ -387,8 +387,10 @@ def run_ours(args) -> int:
             "clocks": sampler.summary(t0, t1), "gpu_launches": launches_per_step(n, world) * args.steps,
             "e2e": e2e,
         }
-        if not args.no_extra:
-            # the latency-bound paths before the seconds-long GEMM loop, whose
+        if world == 1 and not args.no_extra:
+            # one GPU only: under torchrun the other ranks would wait at the
+            # closing barrier, within the process group's timeout, meanwhile.
+            # The latency-bound paths run before the seconds-long GEMM loop, whose
             # power-capped clocks would otherwise linger into their timing
             line["extra_paths"] = {"topk_tail": measure_topk(args, kq, dev),
                                    "sparse_ref": measure_sparse_ref(args, kq, dev),
