@@ -320,7 +320,7 @@ struct SelShared {
   unsigned hist[kBuckets];
   unsigned long long gather[kGather];
   int gather_bucket[kGather];
-  unsigned picked[kBuckets / 32];  // buckets gathered by the shared first round
+  unsigned picked[kBuckets / 32];  // buckets gathered by the shared first pass
   unsigned long long rk[2][32];
   unsigned ru[32];
   unsigned long long answer;
@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kSelThreads) paired_select_kernel(const Paired
   const KeySrc src{p.boot, staged ? sk : nullptr};
   const int nt = 2 * p.nq;
 
-  // Shared first round: one histogram over [kmin, kmax] serves every target;
+  // Shared first pass: one histogram over [kmin, kmax] serves every target;
   // the buckets holding the targets' ranks are gathered together while they
   // fit the gather buffer, and each target is ranked inside its bucket.
   // A target whose bucket does not fit runs the narrowing loop below alone.
