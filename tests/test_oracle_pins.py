@@ -262,6 +262,31 @@ def pin_tail_spread_cases(O):
     assert _close(r["kl"], want, rtol=1e-12)
 
 
+def pin_tail_duplicates_vectorised(O):
+    # the hand-computed duplicate case through the [n, k] function: the
+    # candidate lists id 3 twice (0.3 then 0.2) and the first slot is the match
+    want = 0.5 * math.log(0.5 / 0.3) + 0.1 * math.log(0.1 / (0.5 / 18)) + 0.4 * math.log(0.4 / (1 - 0.3 - 0.5 / 18))
+    r = O.topk_tail(np.array([[3, 1], [1, 3]]), np.log([[0.5, 0.1], [0.1, 0.5]]), np.array([[3, 3], [3, 3]]),
+                    np.log([[0.3, 0.2], [0.3, 0.2]]), 20)
+    assert _close(r["kl"][0], want, rtol=1e-12) and _close(r["kl"][1], want, rtol=1e-12)
+    assert list(r["n_matched"]) == [1, 1] and list(r["top1"]) == [1, 0]
+    # random lists drawn with repetition (distinct log-probs at repeated ids):
+    # the [n, k] function agrees with the per-position one, which the brute
+    # force and the hand-computed cases pin
+    rng = np.random.default_rng(9)
+    n, k, V = 200, 12, 40
+    ri = rng.integers(0, 16, (n, k))
+    ci = rng.integers(0, 16, (n, k))
+    assert any(len(set(row)) < k for row in ci)
+    rl = np.log(rng.dirichlet(np.ones(k + 4), n)[:, :k])
+    cl = np.log(rng.dirichlet(np.ones(k + 4), n)[:, :k])
+    vec = O.topk_tail(ri, rl, ci, cl, V, chunk=64)
+    for i in range(n):
+        row = O.topk_tail_row(ri[i], rl[i], ci[i], cl[i], V)
+        assert _close(vec["kl"][i], row["kl"], rtol=1e-12, atol=1e-15)
+        assert vec["n_matched"][i] == row["n_matched"] and vec["top1"][i] == row["top1"]
+
+
 def pin_tail_self(O):
     rng = np.random.default_rng(8)
     ids = np.stack([rng.permutation(1000)[:64] for _ in range(50)])
@@ -521,6 +546,82 @@ def pin_shared_head_matmul(O):
         assert _close(res2["kl"][i], O.full_vocab_row(H[i] @ W.T, (H[i] + 0.1) @ W.T)["kl"], rtol=1e-12)
 
 
+def pin_logit_error_bound_closed_form(O):
+    # K = 2, h = (1, -2), w = (3, 0.5): sum |h_k w_k| = 3 + 1 = 4 and
+    # gamma_2 = 2 u, so the bound is 8 u = 2^-21 at u = 2^-24, exactly.
+    assert O.logit_error_bound(np.array([1.0, -2.0]), np.array([3.0, 0.5])) == 2.0 ** -21
+    # K = 3 with cancelling products: |h.w| = 0 but sum |h_k w_k| = 6, so
+    # the bound is gamma_3 * 6 = 18 u (a bound on |h.w| alone would be 0)
+    assert O.logit_error_bound(np.array([1.0, 1.0, 1.0]), np.array([2.0, -3.0, 1.0])) == 18.0 * 2.0 ** -24
+    # the unit roundoff is a parameter: bf16 (u = 2^-8), K = 1, |h w| = 0.75
+    assert O.logit_error_bound(np.array([-0.5]), np.array([1.5]), unit_roundoff=2.0 ** -8) == 0.75 * 2.0 ** -8
+
+
+def pin_argmax_ambiguous_threshold(O):
+    # K = 1, h = (1): logits are the head's single column w_v.  With top two
+    # logits 1 and 1 - d, the bounds are u and u (1 - d), so the row is
+    # ambiguous exactly when d < 2 (u + u (1 - d)), i.e. d < 4u / (1 + 2u).
+    u = 2.0 ** -24
+    edge = 4 * u / (1 + 2 * u)
+    h = np.array([1.0])
+    for d, amb in ((edge * 0.98, True), (edge * 1.02, False), (0.0, True), (0.5, False)):
+        W = np.array([[0.0], [1.0], [-3.0], [1.0 - d]])
+        z = W @ h
+        assert bool(O.argmax_ambiguous(z, h, W)) is amb, (d, amb)
+    # K = 2, h = (1, 1), rows (3, -2) -> 1 and (2, -1 - d) -> 1 - d: the sums
+    # of |h_k w_k| are 5 and 3 + d, so the threshold is 2 * 2u * (8 + d)
+    # ~ 2^-19, far above the 2 * 2u * (2 - d) that |h.w| alone would give.
+    h = np.array([1.0, 1.0])
+    for d, amb in ((2.0 ** -20, True), (2.0 ** -19 * 1.01, False), (2.0 ** -19 * 0.99, True)):
+        W = np.array([[3.0, -2.0], [0.0, 0.0], [2.0, -1.0 - d]])
+        z = W @ h
+        assert bool(O.argmax_ambiguous(z, h, W)) is amb, (d, amb)
+    # the top two are found by value, whatever their positions
+    W = np.array([[0.0, 0.0], [2.0, -1.0 - 2.0 ** -20], [-1.0, 0.0], [3.0, -2.0]])
+    assert bool(O.argmax_ambiguous(W @ h, h, W)) is True
+
+
+def pin_argmax_ambiguous_covers_f32_sums(O):
+    # Sequential float32 sums of float32 products, in several orders: any row
+    # whose f32 argmax differs from the float64 one must be flagged.  Each
+    # row plants a near-twin of its leading head row, at logit gaps from
+    # 1e-7 to 1 (log-uniform).
+    rng = np.random.default_rng(21)
+    K, V, n = 256, 6, 120
+    f32 = lambda a: np.asarray(a, dtype=np.float32).astype(np.float64)
+    flips = flagged = 0
+    for _ in range(n):
+        h = f32(rng.normal(0, 1, K))
+        W = f32(rng.normal(0, 0.05, (V, K)))
+        W[0] = f32(W[0] + 0.25 * np.sign(h))             # a clear leader ...
+        j = int(np.argmax(np.abs(h)))
+        W[1] = W[0].copy()                               # ... and a near-twin
+        W[1, j] = f32(W[0, j] + rng.choice([-1.0, 1.0]) * 10 ** rng.uniform(-7, 0) / abs(h[j]))
+        z = W @ h
+        best = int(np.argmax(z))
+        amb = bool(O.argmax_ambiguous(z, h, W))
+        flagged += amb
+        prods = (W * h).astype(np.float32)               # the correctly rounded f32 products
+        sums = []
+        for order in (np.arange(K), np.arange(K)[::-1], rng.permutation(K)):
+            acc = np.zeros(V, dtype=np.float32)
+            for k in order:
+                acc = acc + prods[:, k]
+            sums.append(acc)
+        # blocks of 16 summed first, then the block sums in order
+        blocks = prods.reshape(V, K // 16, 16).sum(axis=2, dtype=np.float32)
+        acc = np.zeros(V, dtype=np.float32)
+        for b in range(K // 16):
+            acc = acc + blocks[:, b]
+        sums.append(acc)
+        for acc in sums:
+            if int(np.argmax(acc)) != best:
+                flips += 1
+                assert amb, ("an f32 argmax differs on a row not flagged ambiguous", z[0] - z[1])
+    assert flips > 0            # the planted gaps do reach f32's rounding
+    assert 0 < flagged < n      # and the bound separates wide gaps from narrow ones
+
+
 # ---------------------------------------------------------------------------
 # paired comparison
 # ---------------------------------------------------------------------------
@@ -693,6 +794,26 @@ MUTANTS = [
      "out[\"a_lower\"] = sum(1 for c in counted if d[c] <= 0)"),
     ("transposed head", "return np.asarray(H, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T",
      "return (np.asarray(W, dtype=np.float64) @ np.asarray(H, dtype=np.float64).T).T[:, ::-1]"),
+    ("vectorised top-k: last matching slot wins", "slot = np.argmax(eq, axis=2)",
+     "slot = k - 1 - np.argmax(eq[:, :, ::-1], axis=2)"),
+    ("per-position top-k: last matching slot wins", "first_slot.setdefault(cid, s)", "first_slot[cid] = s"),
+    ("error bound without the length factor",
+     "return H_row.shape[0] * unit_roundoff * float(h @ np.abs(np.asarray(W_row, dtype=np.float64)))",
+     "return unit_roundoff * float(h @ np.abs(np.asarray(W_row, dtype=np.float64)))"),
+    ("error bound from |h.w|",
+     "return H_row.shape[0] * unit_roundoff * float(h @ np.abs(np.asarray(W_row, dtype=np.float64)))",
+     "return H_row.shape[0] * unit_roundoff * abs(float(np.asarray(H_row) @ np.asarray(W_row)))"),
+    ("ambiguity threshold ten times too wide", "return (z[i1] - z[i2]) < 2.0 * (b1 + b2)",
+     "return (z[i1] - z[i2]) < 20.0 * (b1 + b2)"),
+    ("ambiguity threshold without the factor two", "return (z[i1] - z[i2]) < 2.0 * (b1 + b2)",
+     "return (z[i1] - z[i2]) < (b1 + b2)"),
+    ("ambiguity bound from |h.w|",
+     "b1 = gamma * float(h @ np.abs(np.asarray(W[i1], dtype=np.float64)))\n"
+     "    b2 = gamma * float(h @ np.abs(np.asarray(W[i2], dtype=np.float64)))",
+     "b1 = gamma * abs(float(np.asarray(H_row) @ np.asarray(W[i1])))\n"
+     "    b2 = gamma * abs(float(np.asarray(H_row) @ np.asarray(W[i2])))"),
+    ("ambiguity against the lowest logit", "i1, i2 = int(order[0]), int(order[1])",
+     "i1, i2 = int(order[0]), int(order[-1])"),
 ]
 
 
