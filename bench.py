@@ -189,100 +189,24 @@ def oracle_rows(ref, cand, targets, rows):
     return time.perf_counter() - t0
 
 
-def host_cores() -> int:
-    try:
-        return len(os.sched_getaffinity(0))
-    except AttributeError:
-        return os.cpu_count() or 1
-
-
-def _oracle_chunk(job):
-    """Process-pool worker: the f64 oracle on rows [a, b) of a window whose
-    bf16 bits (reference then candidate) and int32 targets sit in files."""
-    bits_path, tg_path, n, vocab, a, b = job
-    import numpy as np
-    from oracle import kld_oracle as O
-    bits = np.memmap(bits_path, dtype=np.uint16, mode="r", shape=(2, n, vocab))
-    T = np.fromfile(tg_path, dtype=np.int32)[a:b]
-    return O.full_vocab(O.bf16_bits_to_f64(np.asarray(bits[0, a:b])),
-                        O.bf16_bits_to_f64(np.asarray(bits[1, a:b])), T)
-
-
-def _noop(_):
-    return 0
-
-
-class OraclePool:
-    """The f64 oracle spread over the host's cores: one spawned worker per
-    core (spawn, so no worker inherits a CUDA context), rows handed out in
-    small jobs.  Inputs go through files in a temporary directory, so only
-    row ranges cross the process boundary."""
-
-    def __init__(self, cores=None):
-        import multiprocessing as mp
-        import tempfile
-        self.cores = cores or host_cores()
-        env_threads = os.environ.get("OMP_NUM_THREADS")
-        os.environ["OMP_NUM_THREADS"] = "1"     # one thread per worker process
-        self.pool = mp.get_context("spawn").Pool(self.cores)
-        if env_threads is None:
-            del os.environ["OMP_NUM_THREADS"]
-        else:
-            os.environ["OMP_NUM_THREADS"] = env_threads
-        self.pool.map(_noop, range(4 * self.cores))   # workers started before any timing
-        self.dir = tempfile.mkdtemp(prefix="kld_oracle_")
-        self.n = self.vocab = 0
-
-    def load(self, ref_bits, cand_bits, targets):
-        """Stage one window's inputs: uint16 [n, V] bit arrays and int32 targets."""
-        import numpy as np
-        self.n, self.vocab = ref_bits.shape
-        self.bits = os.path.join(self.dir, "bits.u16")
-        self.tg = os.path.join(self.dir, "targets.i32")
-        mm = np.memmap(self.bits, dtype=np.uint16, mode="w+", shape=(2, self.n, self.vocab))
-        mm[0] = ref_bits
-        mm[1] = cand_bits
-        mm.flush()
-        del mm
-        np.asarray(targets, dtype=np.int32).tofile(self.tg)
-
-    def score(self, a, b, rows_per_job=4):
-        """Oracle results of rows [a, b), in row order, and the reduction over them."""
-        import numpy as np
-        from oracle import kld_oracle as O
-        jobs = [(self.bits, self.tg, self.n, self.vocab, i, min(b, i + rows_per_job))
-                for i in range(a, b, rows_per_job)]
-        parts = self.pool.map(_oracle_chunk, jobs, chunksize=1)
-        res = {k: np.concatenate([p[k] for p in parts]) for k in parts[0]}
-        O.reduce_stats(res["kl"], res["ref_argmax"], res["cand_argmax"], None, res["ref_target_lp"],
-                       res["cand_target_lp"], quantiles=QUANTILES)
-        return res
-
-    def close(self):
-        import shutil
-        self.pool.terminate()
-        self.pool.join()
-        shutil.rmtree(self.dir, ignore_errors=True)
-
-
 def cpu_baseline(ref, cand, targets, single_rows: int) -> dict:
     """The f64 oracle timed on the host: every row of the window over all
     cores (the reported value), and a sample of rows on one thread."""
-    import numpy as np
-    import torch
+    from oracle import kld_oracle as O
+    from oracle.pool import OraclePool
     n = ref.shape[0]
     rows = list(range(0, n, max(1, n // single_rows)))[:single_rows]
     dt1 = oracle_rows(ref, cand, targets, rows)
-    pool = OraclePool()
-    try:
-        pool.load(ref.cpu().view(torch.int16).numpy().view(np.uint16),
-                  cand.cpu().view(torch.int16).numpy().view(np.uint16), targets.cpu().numpy())
+    with OraclePool() as pool:
+        staged = {"X": pool.stage("x", ref, "bf16"), "Y": pool.stage("y", cand, "bf16"),
+                  "targets": pool.stage("t", targets, "int")}
         t0 = time.perf_counter()
-        pool.score(0, n)
+        res = pool.run("full_vocab", staged, n)
+        O.reduce_stats(res["kl"], res["ref_argmax"], res["cand_argmax"], None, res["ref_target_lp"],
+                       res["cand_target_lp"], quantiles=QUANTILES)
         dt = time.perf_counter() - t0
-    finally:
-        pool.close()
-    return {"value": n / dt, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
+        cores = pool.cores
+    return {"value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"all {n} rows of the window (f64 numpy oracle + reductions), one process per core",
             "single_thread": {"value": round(len(rows) / dt1, 2), "cores": 1, "sample": f"{len(rows)} rows"}}
 
@@ -290,28 +214,30 @@ def cpu_baseline(ref, cand, targets, single_rows: int) -> dict:
 def run_reference(args) -> int:
     """Reference arm: the f64 oracle on the host's cores, a bounded sample of
     the window's rows per step, spread over one process per core."""
-    import numpy as np
     import torch
+    from oracle import kld_oracle as O
+    from oracle.pool import OraclePool
     from synth import workloads as W
     world, rank, _ = rank_env(default_world=args.gpus)
     if rank != 0:
         return 0
-    pool = OraclePool()          # spawned before the first CUDA call
-    try:
+    with OraclePool() as pool:          # spawned before the first CUDA call
         # inputs drawn on the GPU when there is one (same bytes as our arm), else on the host
         dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
         per_row_s = 0.012 / pool.cores
         rows_per_step = int(args.ref_seconds / ((args.steps + args.warmup) * per_row_s))
         rows_per_step = max(pool.cores, min(N_ROWS, rows_per_step))
-        d = W.window_full_vocab(seed=W.seed_for(2), device=dev, n_rows=min(N_ROWS, max(2 * rows_per_step, 64)))
-        pool.load(d["ref"].cpu().view(torch.int16).numpy().view(np.uint16),
-                  d["cand"].cpu().view(torch.int16).numpy().view(np.uint16), d["targets"].cpu().numpy())
-        n_avail = d["ref"].shape[0]
+        n_avail = min(N_ROWS, max(2 * rows_per_step, 64))
+        d = W.window_full_vocab(seed=W.seed_for(2), device=dev, n_rows=n_avail)
+        staged = {"X": pool.stage("x", d["ref"], "bf16"), "Y": pool.stage("y", d["cand"], "bf16"),
+                  "targets": pool.stage("t", d["targets"], "int")}
         del d
 
         def step(i):
             a = (i * rows_per_step) % (n_avail - rows_per_step + 1)
-            pool.score(a, a + rows_per_step)
+            res = pool.run("full_vocab", staged, rows_per_step, start=a)
+            O.reduce_stats(res["kl"], res["ref_argmax"], res["cand_argmax"], None, res["ref_target_lp"],
+                           res["cand_target_lp"], quantiles=QUANTILES)
 
         for i in range(args.warmup):
             step(i)
@@ -319,8 +245,7 @@ def run_reference(args) -> int:
         for i in range(args.steps):
             step(i)
         dt = time.perf_counter() - t0
-    finally:
-        pool.close()
+        cores = pool.cores
     value = rows_per_step * args.steps / dt
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
@@ -328,9 +253,9 @@ def run_reference(args) -> int:
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded Zipf/Gumbel logits; no corpus or model)",
         "config": config_dict(),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{rows_per_step} rows of the window per step, f64 numpy oracle, "
-                                   f"{pool.cores} processes (one per host core)"},
+                                   f"{cores} processes (one per host core)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -23,14 +23,20 @@ def reduce_stats_across_ranks(kl, ref_argmax=None, cand_argmax=None, top1=None, 
     """The kld_reduce_stats statistics of every rank's positions together.
 
     Collective: every rank of `group` calls this with the same quantiles and
-    thresholds.  `step_fn` replaces the library step (tests of the exchange
-    on hosts without a GPU)."""
+    thresholds.  With NCCL the blocks move device to device; with gloo (which
+    gathers host tensors) a rank's device block goes through host memory.
+    `step_fn` replaces the library step (tests of the exchange on hosts
+    without a GPU)."""
     step_fn = api.kld_reduce_shard_step if step_fn is None else step_fn
     world = dist.get_world_size(group)
     dev = kl.device
     bb = api.kld_reduce_shard_block_bytes() if step_fn is api.kld_reduce_shard_step else step_fn.block_bytes
     block = torch.empty(bb, dtype=torch.uint8, device=dev)
     gathered = [torch.empty(world * bb, dtype=torch.uint8, device=dev) for _ in range(2)]
+    via_host = dev.type == "cuda" and dist.get_backend(group) == "gloo"
+    if via_host:
+        host_block = torch.empty(bb, dtype=torch.uint8)
+        host_gathered = torch.empty(world * bb, dtype=torch.uint8)
     if workspace is None and step_fn is api.kld_reduce_shard_step:
         workspace = torch.empty(api.kld_reduce_shard_workspace_size(kl.shape[0]), dtype=torch.uint8, device=dev)
     if out is None:
@@ -42,7 +48,16 @@ def reduce_stats_across_ranks(kl, ref_argmax=None, cand_argmax=None, top1=None, 
                 out=out if last else None, workspace=workspace, dev_status=dev_status, stream=stream)
         if not last:
             # alternate buffers, so a step never overwrites the blocks it is still reading
-            dist.all_gather_into_tensor(gathered[step % 2], block, group=group)
+            if via_host:
+                if stream is not None:
+                    stream.synchronize()
+                host_block.copy_(block)          # waits for the step on the current stream
+                dist.all_gather_into_tensor(host_gathered, host_block, group=group)
+                gathered[step % 2].copy_(host_gathered)
+                if stream is not None:           # the next step reads it on `stream`
+                    stream.wait_stream(torch.cuda.current_stream(dev))
+            else:
+                dist.all_gather_into_tensor(gathered[step % 2], block, group=group)
     if not to_host:
         return out
     return api.stats_from_device(out) if step_fn is api.kld_reduce_shard_step else out

@@ -95,14 +95,16 @@ def test_deterministic(cuda_device):
 
 
 def test_full_size_sampled(cuda_device):
-    """8192 positions x 5120 hidden through a 248,320 x 5120 head: 40 seeded
-    rows against the oracle, every row finite."""
+    """8192 positions x 5120 hidden through a 248,320 x 5120 head: 256 seeded
+    rows against the oracle (its f64 logits cost 5.1 GFLOP per row), every
+    row finite."""
     d = W.shared_head_states(device=cuda_device)
     res = run(d)
     assert res["status"] == 0
     n = d["h_ref"].shape[0]
     g = torch.Generator().manual_seed(11)
-    rows = np.unique(np.concatenate([torch.randperm(n, generator=g)[:38].numpy(), [0, n - 1]]))
+    rows = np.unique(np.concatenate([torch.randperm(n - 2, generator=g)[:254].numpy() + 1, [0, n - 1]]))
+    assert len(rows) == 256
     check(res, d, rows)
     kl = res["kl"].cpu().numpy()
     assert np.all(np.isfinite(kl)) and kl.min() >= -1e-5

@@ -6,6 +6,7 @@ import torch
 
 import quantization_fidelity_scoring_b200 as kq
 from oracle import kld_oracle as O
+from oracle.pool import OraclePool
 from quantization_fidelity_scoring_b200 import _lib
 from synth import workloads as W
 from tests.helpers import to_f64
@@ -33,33 +34,36 @@ def padded(t, per16):
     return base[:, :t.shape[1]]
 
 
-def check(res, x, k, targets, rows=None, chunk=64):
-    n = x.shape[0]
-    rows = np.arange(n) if rows is None else np.asarray(rows)
+def compare(res, want, rows):
+    """Library capture outputs on `rows` against the oracle's for those rows."""
     ids = res["ids"].cpu().numpy()[rows]
     lp = res["lp"].cpu().numpy().astype(np.float64)[rows]
     out = res["rows"].cpu().numpy().astype(np.float64)[rows]
+    assert np.array_equal(ids, want["ids"]), "ids differ"
+    w_lp, g_lp = want["lp"], lp
+    assert np.array_equal(np.isnan(g_lp), np.isnan(w_lp))
+    ok = ~np.isnan(w_lp)
+    assert np.all(np.abs(g_lp[ok] - w_lp[ok]) <= LP_RTOL * np.abs(w_lp[ok]) + LP_ATOL), "lp"
+    g, w = out, want["rows"]
+    assert np.array_equal(np.isnan(g), np.isnan(w))
+    ok = ~np.isnan(w)
+    inf = np.isinf(w)
+    assert np.array_equal(np.isinf(g), inf) and np.array_equal(g[inf], w[inf])  # a target at -inf: NLL +inf
+    ok &= ~inf
+    for col, rt, at in ((0, LP_RTOL, LP_ATOL), (1, H_RTOL, H_ATOL), (2, TAIL_RTOL, TAIL_ATOL)):
+        m = ok[:, col]
+        err = np.abs(g[m, col] - w[m, col])
+        assert np.all(err <= rt * np.abs(w[m, col]) + at), (col, err.max())
+
+
+def check(res, x, k, targets, rows=None, chunk=64):
+    n = x.shape[0]
+    rows = np.arange(n) if rows is None else np.asarray(rows)
     T = None if targets is None else targets.cpu().numpy()[rows]
     for a in range(0, len(rows), chunk):
         r = rows[a:a + chunk]
         X = to_f64(x[torch.as_tensor(r, device=x.device)])
-        want = O.sparse_capture(X, k, None if T is None else T[a:a + chunk])
-        sl = slice(a, a + len(r))
-        assert np.array_equal(ids[sl], want["ids"]), "ids differ"
-        w_lp, g_lp = want["lp"], lp[sl]
-        assert np.array_equal(np.isnan(g_lp), np.isnan(w_lp))
-        ok = ~np.isnan(w_lp)
-        assert np.all(np.abs(g_lp[ok] - w_lp[ok]) <= LP_RTOL * np.abs(w_lp[ok]) + LP_ATOL), "lp"
-        g, w = out[sl], want["rows"]
-        assert np.array_equal(np.isnan(g), np.isnan(w))
-        ok = ~np.isnan(w)
-        inf = np.isinf(w)
-        assert np.array_equal(np.isinf(g), inf) and np.array_equal(g[inf], w[inf])  # a target at -inf: NLL +inf
-        ok &= ~inf
-        for col, rt, at in ((0, LP_RTOL, LP_ATOL), (1, H_RTOL, H_ATOL), (2, TAIL_RTOL, TAIL_ATOL)):
-            m = ok[:, col]
-            err = np.abs(g[m, col] - w[m, col])
-            assert np.all(err <= rt * np.abs(w[m, col]) + at), (col, err.max())
+        compare(res, O.sparse_capture(X, k, None if T is None else T[a:a + chunk]), r)
 
 
 @pytest.mark.parametrize("n,V,k,dtype", [
@@ -81,15 +85,17 @@ def test_shapes_all_rows(cuda_device, n, V, k, dtype, exact):
     check(res, x, k, tg)
 
 
-def test_full_size_window_sampled_rows(cuda_device):
-    """2047 positions x 248,320 bf16, K = 512: 300 seeded rows against the
-    oracle, every row's listed masses plus tail making 1."""
+def test_full_size_window_all_rows(cuda_device):
+    """2047 positions x 248,320 bf16, K = 512: every row against the oracle
+    (one oracle process per host core), every row's listed masses plus tail
+    making 1."""
     d = W.window_full_vocab(device=cuda_device)
     res = run(d["ref"], 512, d["targets"])
     assert res["status"] == 0
-    g = torch.Generator().manual_seed(5)
-    rows = np.unique(np.concatenate([torch.randperm(2047, generator=g)[:298].numpy(), [0, 2046]]))
-    check(res, d["ref"], 512, d["targets"], rows)
+    with OraclePool() as pool:
+        staged = {"X": pool.stage("x", d["ref"], "bf16"), "targets": pool.stage("t", d["targets"], "int")}
+        want = pool.run("sparse_capture", staged, d["ref"].shape[0], rows_per_job=4, k=512)
+    compare(res, want, np.arange(d["ref"].shape[0]))
     mass = torch.exp(res["lp"].double()).sum(1) + res["rows"][:, 2].double()
     assert torch.all(torch.abs(mass - 1.0) < 1e-5)
 
