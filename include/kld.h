@@ -150,8 +150,9 @@ size_t kld_full_vocab_workspace_size(int64_t n_rows);
  *   - The array takes about 1.2 MB on every GPU that loads the library and
  *     stays allocated until the process exits.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current, and so does the first
+ *     call in a new context of that device (e.g. after cudaDeviceReset);
+ *     make that first call before any stream capture.
  *   - Every call on a device shares the one array.  Calls that may overlap
  *     on the GPU (different streams, or several host threads) race and can
  *     corrupt each other's results: serialise them.  The array keeps the last

@@ -19,6 +19,7 @@
 // score" (KL over cells); "Qwopus3.8-27B-Coder-Flash: quality-eval
 // reference", "Method" (exact argmax top-1, perplexity from the true-token
 // log-prob).
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cfloat>
 #include <mutex>
@@ -35,6 +36,7 @@ constexpr int kWarpsPerCta = kThreads / 32;
 constexpr int kStepVecs = 64;                    // vectors a warp covers per step
 constexpr int kMinVecsPerWarp = 8 * kStepVecs;   // below this, use fewer warps
 constexpr int kMaxStreamWarps = kFullVocabMaxWarps;
+constexpr int kFlushSteps = 16;                  // steps whose sums meet before joining the row's
 
 // Partial state of one warp over one row piece (32 bytes).
 struct Piece {
@@ -115,17 +117,34 @@ __device__ __forceinline__ float side_new_max(WarpSide& s, float cm, const uint4
   return sc;
 }
 
-// Accumulate one step: weights exp(z - m) on paired f32x2 arithmetic.  With
+// The exponent offset of a side: c = -m log2(e) rounded to f32 (0 before a
+// finite value), so a weight is 2^(z log2(e) + c) from one fused
+// multiply-add; c misses -m log2(e) by rho = -m log2(e) - c (exact, from a
+// second fused multiply-add), so those weights are exp(z - m) 2^-rho, and
+// sums formed with c are multiplied by fix = 2^rho when they join the row's.
+struct Offset {
+  float c, fix;
+};
+
+__device__ __forceinline__ Offset offset_of(const WarpSide& s) {
+  if (s.a < 0) return Offset{0.f, 1.f};
+  const float c = __fmul_rn(-s.m, kLog2e);
+  const float rho = fmaf(-s.m, kLog2e, -c);
+  return Offset{c, ex2(rho)};
+}
+
+// Accumulate one step: weights exp(z - m) 2^-rho on paired f32x2 arithmetic
+// (see Offset; cx, cy are the sides' offsets c).  With
 // kMasked, the slots ex_x / ex_y (the new argmaxes) are weighed as -inf so
 // they stay out of r; the reference argmax's own A term, 1 * (x - y), is
 // added by the caller.
 template <bool kBF16, bool kMasked>
-__device__ __forceinline__ void accumulate(const StepRaw& raw, float mx, float my, int ex_x, int ex_y,
+__device__ __forceinline__ void accumulate(const StepRaw& raw, float cx, float cy, int ex_x, int ex_y,
                                            float2& rx2, float2& ry2, float2& a2) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
-  const float2 nmx = make_float2(-mx, -mx);
-  const float2 nmy = make_float2(-my, -my);
+  const float2 nmx = make_float2(cx, cx);
+  const float2 nmy = make_float2(cy, cy);
   const float2 l2 = make_float2(kLog2e, kLog2e);
   const float2 neg1 = make_float2(-1.f, -1.f);
 #pragma unroll
@@ -142,8 +161,8 @@ __device__ __forceinline__ void accumulate(const StepRaw& raw, float mx, float m
         if (ex_y == j) YW.x = -CUDART_INF_F;
         if (ex_y == j + 1) YW.y = -CUDART_INF_F;
       }
-      const float2 tx = __fmul2_rn(__fadd2_rn(XW, nmx), l2);
-      const float2 ty = __fmul2_rn(__fadd2_rn(YW, nmy), l2);
+      const float2 tx = __ffma2_rn(XW, l2, nmx);  // x log2(e) + c, one rounding
+      const float2 ty = __ffma2_rn(YW, l2, nmy);
       const float2 ex = make_float2(ex2(tx.x), ex2(tx.y));
       const float2 ey = make_float2(ex2(ty.x), ex2(ty.y));
       rx2 = __fadd2_rn(rx2, ex);
@@ -184,8 +203,24 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
   constexpr uint32_t kNegInfWord = kBF16 ? 0xff80ff80u : 0xff800000u;
   const uint4 neg_inf = make_uint4(kNegInfWord, kNegInfWord, kNegInfWord, kNegInfWord);
 
+  // Sums on two levels of f32: lanes add each step's weights into rx2, ry2,
+  // a2 (formed with the sides' offsets), which join the side's r and aA
+  // (times the offsets' fix) every kFlushSteps steps and whenever a maximum
+  // moves.  No f32 sum then has more than about a hundred terms however long
+  // the row: a row's thousands of terms in one running sum lost up to 1e-5 of
+  // a target log-prob.
   WarpSide sx{-CUDART_INF_F, -1, 0.f}, sy{-CUDART_INF_F, -1, 0.f};
+  Offset ox{0.f, 1.f}, oy{0.f, 1.f};
   float2 rx2 = make_float2(0.f, 0.f), ry2 = rx2, a2 = rx2;
+  float aA = 0.f;
+  int since = 0;
+  auto fold = [&]() {
+    sx.r += (rx2.x + rx2.y) * ox.fix;
+    sy.r += (ry2.x + ry2.y) * oy.fix;
+    aA += (a2.x + a2.y) * ox.fix;
+    rx2 = ry2 = a2 = make_float2(0.f, 0.f);
+    since = 0;
+  };
 
   const int n = b - a;
   const int nfull = n / kStepVecs;
@@ -203,30 +238,29 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
     const float CMX = warp_max(El::vmax2(cur.x0, cur.x1));
     const float CMY = warp_max(El::vmax2(cur.y0, cur.y1));
     if (!((CMX > sx.m) || (CMY > sy.m) || (sx.a < 0) || (sy.a < 0))) {  // warp-uniform
-      accumulate<kBF16, false>(cur, sx.m, sy.m, -1, -1, rx2, ry2, a2);
-      return;
+      accumulate<kBF16, false>(cur, ox.c, oy.c, -1, -1, rx2, ry2, a2);
+    } else {
+      // the per-vector maxima locate a new maximum (rare: computed only here)
+      const float cx0 = El::vmax(cur.x0), cx1 = El::vmax(cur.x1);
+      const float cy0 = El::vmax(cur.y0), cy1 = El::vmax(cur.y1);
+      // a new maximum on either side, or a side still without a finite
+      // value: fold the step sums in, move to the new maxima, weigh the step
+      // with the new argmaxes masked out of r
+      fold();
+      const int i0 = (a + st * kStepVecs + lane) * E;
+      const int i1 = i0 + 32 * E;
+      int ex_x, ex_y;
+      const float scx = side_new_max<kBF16>(sx, CMX, cur.x0, cur.x1, cx0, cx1, i0, i1, lane, ex_x);
+      side_new_max<kBF16>(sy, CMY, cur.y0, cur.y1, cy0, cy1, i0, i1, lane, ex_y);
+      aA *= scx;
+      if (ex_x >= 0) aA += slot_diff<kBF16>(cur, ex_x);
+      // a side with no finite value yet has only -inf (weight 0) or NaN
+      // (poisons r, marking the row invalid); any finite offset serves
+      ox = offset_of(sx);
+      oy = offset_of(sy);
+      accumulate<kBF16, true>(cur, ox.c, oy.c, ex_x, ex_y, rx2, ry2, a2);
     }
-    // the per-vector maxima locate a new maximum (rare: computed only here)
-    const float cx0 = El::vmax(cur.x0), cx1 = El::vmax(cur.x1);
-    const float cy0 = El::vmax(cur.y0), cy1 = El::vmax(cur.y1);
-    // a new maximum on either side, or a side still without a finite value:
-    // fold the paired sums, move to the new maxima, weigh with the new
-    // argmaxes masked out of r
-    sx.r += rx2.x + rx2.y;
-    sy.r += ry2.x + ry2.y;
-    float A = a2.x + a2.y;
-    const int i0 = (a + st * kStepVecs + lane) * E;
-    const int i1 = i0 + 32 * E;
-    int ex_x, ex_y;
-    const float scx = side_new_max<kBF16>(sx, CMX, cur.x0, cur.x1, cx0, cx1, i0, i1, lane, ex_x);
-    side_new_max<kBF16>(sy, CMY, cur.y0, cur.y1, cy0, cy1, i0, i1, lane, ex_y);
-    A *= scx;
-    if (ex_x >= 0) A += slot_diff<kBF16>(cur, ex_x);
-    rx2 = ry2 = make_float2(0.f, 0.f);
-    a2 = make_float2(A, 0.f);
-    // a side with no finite value yet has only -inf (weight 0) or NaN
-    // (poisons r, marking the row invalid); any finite offset serves
-    accumulate<kBF16, true>(cur, sx.a < 0 ? 0.f : sx.m, sy.a < 0 ? 0.f : sy.m, ex_x, ex_y, rx2, ry2, a2);
+    if (++since == kFlushSteps) fold();  // warp-uniform
   };
 
   // full steps: the warp's four 16-byte loads per lane for step st + 1 are
@@ -251,9 +285,10 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
     step(A, st);
   }
 
-  float rxs = sx.r + (rx2.x + rx2.y);
-  float rys = sy.r + (ry2.x + ry2.y);
-  float as = a2.x + a2.y;
+  fold();
+  float rxs = sx.r;
+  float rys = sy.r;
+  float as = aA;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     rxs += __shfl_xor_sync(0xffffffffu, rxs, off);
@@ -369,24 +404,65 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(Piece) *
 
 }  // namespace
 
+namespace {
+
+// A process-unique id of the context current on this thread (a context made
+// again after a device reset gets a new one).  False when there is no
+// current context or the driver cannot tell.
+bool current_context_id(unsigned long long* id) {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t noalloc_scratch(void** ptr, size_t* bytes) {
   // Host code cannot use g_noalloc_scratch's name as a device address: look
-  // the address up once per device, with that device current, and cache it.
+  // the address up with the device current and cache it, per device, for the
+  // context it was found in; a different context (e.g. after a device reset)
+  // looks it up again.
   constexpr int kMaxDevices = 64;
+  struct Entry {
+    unsigned long long ctx_id;
+    void* ptr;
+  };
   static std::mutex mu;
-  static void* cached[kMaxDevices] = {};
+  static Entry cached[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
   std::lock_guard<std::mutex> lock(mu);
-  if (cached[dev] == nullptr) {
+  if (!have_id || cached[dev].ptr == nullptr || cached[dev].ctx_id != id) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the device's context current if it was not
     if (e != cudaSuccess) return e;
-    cached[dev] = p;
+    if (!have_id) have_id = current_context_id(&id);
+    cached[dev] = Entry{have_id ? id : 0ull, have_id ? p : nullptr};  // unknown context: look up every call
+    *ptr = p;
+  } else {
+    *ptr = cached[dev].ptr;
   }
-  *ptr = cached[dev];
   *bytes = sizeof(g_noalloc_scratch);
   return cudaSuccess;
 }

@@ -168,7 +168,7 @@ static kld_status sparse_ref_impl(const void* cand_logits, kld_dtype dtype, int6
   if (!ref_rows && ref_target_lp) return KLD_ERR_INVALID_ARG;
   if (n_rows == 0) return KLD_OK;
   if (!cand_logits || !ref_top || !kl) return KLD_ERR_INVALID_ARG;
-  if (n_rows > (int64_t)INT32_MAX - kld::kFullVocabMaxWarps) return KLD_ERR_UNSUPPORTED;
+  if (n_rows > (int64_t)INT32_MAX - kld::kSparseMaxWarps) return KLD_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < kld::sparse_ref_workspace_bytes(n_rows, k)) return KLD_ERR_WORKSPACE;
   const int64_t esize = dtype == KLD_BF16 ? 2 : 4;
   if (!aligned(workspace, 256) || !aligned(cand_logits, 16) || (ld_cand * esize) % 16 != 0)
@@ -238,7 +238,7 @@ static kld_status sparse_capture_impl(const void* logits, kld_dtype dtype, int64
   if (vocab > (int64_t(1) << 22)) return KLD_ERR_UNSUPPORTED;
   if (n_rows == 0) return KLD_OK;
   if (!logits || !top || !rows) return KLD_ERR_INVALID_ARG;
-  if (n_rows > (int64_t)INT32_MAX - kld::kFullVocabMaxWarps) return KLD_ERR_UNSUPPORTED;
+  if (n_rows > (int64_t)INT32_MAX - kld::kSparseMaxWarps) return KLD_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < kld::sparse_capture_workspace_bytes(n_rows)) return KLD_ERR_WORKSPACE;
   const int64_t esize = dtype == KLD_BF16 ? 2 : 4;
   if (!aligned(workspace, 256) || !aligned(logits, 16) || (ld * esize) % 16 != 0) return KLD_ERR_ALIGNMENT;

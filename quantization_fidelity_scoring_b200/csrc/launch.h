@@ -29,6 +29,9 @@ struct FullVocabArgs {
 // device): three CTAs of eight warps per SM on 148 SMs.
 constexpr int kStreamCtasPerSm = 3;
 constexpr int kFullVocabMaxWarps = 148 * kStreamCtasPerSm * 8;
+// The sparse-reference and capture streams: at most three CTAs of eight
+// persistent warps per SM of a 148-SM part (their row slots are row + warp).
+constexpr int kSparseMaxWarps = 148 * 3 * 8;
 size_t full_vocab_workspace_bytes(int64_t n_rows);
 cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream);
 // Rows the library-owned scratch of kld_full_vocab_noalloc can hold.

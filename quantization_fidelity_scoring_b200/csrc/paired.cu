@@ -9,19 +9,26 @@
 // and the "compare against a published candidate" step).  The page gives
 // no formulas; kld.h states the reading implemented here.
 //
-// Five launches, all deterministic (f64 sums in fixed orders, integer
+// Four launches, all deterministic (f64 sums in fixed orders, integer
 // counts):
 //   ctx      one warp per context: sums of A's and B's counted KL (exact in
 //            f64 for ordinary spreads of f32 values), the count, the means
 //            and their difference d_c.
-//   cluster  one warp per cluster: D[k] and N[k] over the contexts in
-//            context order; more blocks sum chunks of 1024 contexts (means,
-//            win and tie counts) for the finish to add in order.
+//   cluster  one thread per context adds d_c to its cluster's D[k] as a
+//            64-bit fixed-point integer (scaled to the largest |d_c|, so the
+//            integer sums are exact and their order does not matter) and 1
+//            to N[k]; non-finite d_c set flags instead.  More blocks sum
+//            chunks of 1024 contexts (means, win and tie counts) for the
+//            finish to add in order.
 //   boot     one warp per replicate: the draws' D and N gathered and summed.
 //   select   one CTA finds the replicates' order statistics at the target
-//            ranks exactly (bucketed 64-bit keys, a few passes);
-//   finish   one warp writes the result.
+//            ranks exactly (bucketed 64-bit keys, a few passes), then one of
+//            its warps writes the result (the finish kernel does that alone
+//            when there are no replicates).
 #include <math_constants.h>
+
+#include <algorithm>
+#include <cfloat>
 
 #include "kld_common.cuh"
 #include "launch.h"
@@ -32,7 +39,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTargets = 2 * KLD_MAX_QUANTILES;
-constexpr int kIdTile = 4096;    // cluster ids staged in shared memory at a time
 constexpr int kBootThreads = 1024;
 constexpr int kBootSmemClusters = 2048;  // clusters whose sums a boot CTA keeps in shared memory
 
@@ -47,8 +53,13 @@ struct PairedPart {
 struct PairedTotals {
   unsigned n_valid;  // replicates whose draws hold a counted context
   unsigned pad;
+  int shift;         // one unit of the clusters' fixed-point sums is 2^shift
+  int pad2;
   double ostat[kMaxTargets];
 };
+
+// Flags of a cluster whose contexts include non-finite differences.
+constexpr int kFlagPosInf = 1, kFlagNegInf = 2, kFlagNaN = 4;
 
 struct PairedParams {
   const float* a;
@@ -68,7 +79,10 @@ struct PairedParams {
   double* ctx_b;
   double* ctx_d;
   int32_t* ctx_n;
-  double* Dk;
+  double* blk_max;    // [ctx blocks] largest finite |d_c| of each block of the context pass
+  int n_ctx_blocks;
+  long long* Dq;      // [n_clusters] fixed-point sums of d_c
+  int32_t* Dflag;     // [n_clusters] kFlag* bits
   long long* Nk;
   PairedPart* parts;  // [ceil(n_ctx / kTotChunk)]
   PairedTotals* tot;
@@ -107,95 +121,121 @@ __device__ __forceinline__ void add_pair(float va, float vb, bool in, double& sa
 }
 
 __global__ void __launch_bounds__(kThreads) paired_ctx_kernel(const PairedParams p) {
+  __shared__ double wmax[kWarps];
   wait_prior_grid();
   if (blockIdx.x == 0 && threadIdx.x == 0) p.tot->n_valid = 0u;
-  const int lane = threadIdx.x & 31;
-  const long long c = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (c >= p.n_ctx) return;
-  const long long base = c * p.ctx_len;
-  const float* a = p.a + base;
-  const float* b = p.b + base;
-  const uint8_t* m = p.mask ? p.mask + base : nullptr;
-  const int L = p.ctx_len;
-  double sa = 0.0, sb = 0.0;
-  unsigned cnt = 0;
-  // the row's head up to a 16-byte boundary (both rows share the offset),
-  // then 16-byte vectors, then the tail
-  const int head = (int)((4 - (base & 3)) & 3) < L ? (int)((4 - (base & 3)) & 3) : L;
-  if (lane < head) add_pair(a[lane], b[lane], !m || m[lane], sa, sb, cnt);
-  const int nvec = (L - head) >> 2;
-  const float4* a4 = reinterpret_cast<const float4*>(a + head);
-  const float4* b4 = reinterpret_cast<const float4*>(b + head);
-  constexpr int U = 2;  // vectors in flight per lane and row
-  for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
-    float4 va[U], vb[U];
+  // the clusters' accumulators start at zero (the cluster pass runs after this kernel)
+  for (long long k = (long long)blockIdx.x * blockDim.x + threadIdx.x; k < p.n_clusters;
+       k += (long long)gridDim.x * blockDim.x) {
+    p.Dq[k] = 0ll;
+    p.Nk[k] = 0ll;
+    p.Dflag[k] = 0;
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const long long c = (long long)blockIdx.x * kWarps + w;
+  double dmax = 0.0;  // largest finite |d_c| of this warp's context
+  if (c < p.n_ctx) {
+    const long long base = c * p.ctx_len;
+    const float* a = p.a + base;
+    const float* b = p.b + base;
+    const uint8_t* m = p.mask ? p.mask + base : nullptr;
+    const int L = p.ctx_len;
+    double sa = 0.0, sb = 0.0;
+    unsigned cnt = 0;
+    // the row's head up to a 16-byte boundary (both rows share the offset),
+    // then 16-byte vectors, then the tail
+    const int head = (int)((4 - (base & 3)) & 3) < L ? (int)((4 - (base & 3)) & 3) : L;
+    if (lane < head) add_pair(a[lane], b[lane], !m || m[lane], sa, sb, cnt);
+    const int nvec = (L - head) >> 2;
+    const float4* a4 = reinterpret_cast<const float4*>(a + head);
+    const float4* b4 = reinterpret_cast<const float4*>(b + head);
+    constexpr int U = 2;  // vectors in flight per lane and row
+    for (int v0 = lane; v0 < nvec; v0 += 32 * U) {
+      float4 va[U], vb[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int v = v0 + 32 * u;
-      if (v < nvec) {
-        va[u] = __ldcs(a4 + v);
-        vb[u] = __ldcs(b4 + v);
-      } else {
-        va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < nvec) {
+          va[u] = __ldcs(a4 + v);
+          vb[u] = __ldcs(b4 + v);
+        } else {
+          va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + 32 * u;
+        const bool live = v < nvec;
+        const int i = head + 4 * v;
+        add_pair(va[u].x, vb[u].x, live && (!m || m[i]), sa, sb, cnt);
+        add_pair(va[u].y, vb[u].y, live && (!m || m[i + 1]), sa, sb, cnt);
+        add_pair(va[u].z, vb[u].z, live && (!m || m[i + 2]), sa, sb, cnt);
+        add_pair(va[u].w, vb[u].w, live && (!m || m[i + 3]), sa, sb, cnt);
       }
     }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int v = v0 + 32 * u;
-      const bool live = v < nvec;
-      const int i = head + 4 * v;
-      add_pair(va[u].x, vb[u].x, live && (!m || m[i]), sa, sb, cnt);
-      add_pair(va[u].y, vb[u].y, live && (!m || m[i + 1]), sa, sb, cnt);
-      add_pair(va[u].z, vb[u].z, live && (!m || m[i + 2]), sa, sb, cnt);
-      add_pair(va[u].w, vb[u].w, live && (!m || m[i + 3]), sa, sb, cnt);
+    const int tail0 = head + 4 * nvec;
+    if (tail0 + lane < L) add_pair(a[tail0 + lane], b[tail0 + lane], !m || m[tail0 + lane], sa, sb, cnt);
+    sa = warp_sum(sa);
+    sb = warp_sum(sb);
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (lane == 0) {
+      const double ma = cnt ? sa / (double)cnt : 0.0;
+      const double mb = cnt ? sb / (double)cnt : 0.0;
+      const double d = ma - mb;
+      p.ctx_n[c] = (int32_t)cnt;
+      p.ctx_a[c] = ma;
+      p.ctx_b[c] = mb;
+      p.ctx_d[c] = d;
+      if (cnt && fabs(d) <= DBL_MAX) dmax = fabs(d);
     }
   }
-  const int tail0 = head + 4 * nvec;
-  if (tail0 + lane < L) add_pair(a[tail0 + lane], b[tail0 + lane], !m || m[tail0 + lane], sa, sb, cnt);
-  sa = warp_sum(sa);
-  sb = warp_sum(sb);
-  cnt = __reduce_add_sync(0xffffffffu, cnt);
-  if (lane == 0) {
-    const double ma = cnt ? sa / (double)cnt : 0.0;
-    const double mb = cnt ? sb / (double)cnt : 0.0;
-    p.ctx_n[c] = (int32_t)cnt;
-    p.ctx_a[c] = ma;
-    p.ctx_b[c] = mb;
-    p.ctx_d[c] = ma - mb;
+  if (lane == 0) wmax[w] = dmax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double mx = wmax[0];
+    for (int j = 1; j < kWarps; ++j) mx = fmax(mx, wmax[j]);
+    p.blk_max[blockIdx.x] = mx;
   }
 }
 
-// Blocks [0, cluster_blocks): one warp per cluster.  Block cluster_blocks:
-// the totals over all counted contexts.
+// Blocks [0, cluster_blocks): one thread per context adds it to its
+// cluster.  Every block first finds the largest finite |d_c| (the same in
+// every block) and scales d_c so that the sum over all contexts fits 62 bits:
+// the fixed-point sums are then exact and independent of the order of the
+// atomics.  Block cluster_blocks on: the totals over all counted contexts.
 __global__ void __launch_bounds__(kThreads) paired_cluster_kernel(const PairedParams p, int cluster_blocks) {
   wait_prior_grid();
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   if ((int)blockIdx.x < cluster_blocks) {
-    // the block's warps scan the cluster ids from shared memory, a tile at
-    // a time; lane l takes contexts l, l + 32, ... in order
-    __shared__ int32_t ids[kIdTile];
-    const int k = blockIdx.x * kWarps + w;
-    double D = 0.0;
-    long long N = 0;
-    for (long long c0 = 0; c0 < p.n_ctx; c0 += kIdTile) {
-      const int m = (p.n_ctx - c0 < kIdTile) ? (int)(p.n_ctx - c0) : kIdTile;
-      __syncthreads();
-      for (int i = threadIdx.x; i < m; i += blockDim.x) ids[i] = __ldg(p.cluster + c0 + i);
-      __syncthreads();
-      if (k < p.n_clusters) {
-        for (int i = lane; i < m; i += 32) {
-          if (ids[i] == k && p.ctx_n[c0 + i] > 0) {
-            D += p.ctx_d[c0 + i];
-            ++N;
-          }
-        }
+    __shared__ double wmax[kWarps];
+    double mx = 0.0;
+    for (int j = threadIdx.x; j < p.n_ctx_blocks; j += blockDim.x) mx = fmax(mx, p.blk_max[j]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) wmax[w] = mx;
+    __syncthreads();
+    mx = wmax[0];
+    for (int j = 1; j < kWarps; ++j) mx = fmax(mx, wmax[j]);
+    int lg = 0;
+    while ((1ll << lg) < p.n_ctx + 1) ++lg;
+    // mx = f 2^e with f in [0.5, 1) (e = 0 when mx = 0); units of 2^shift
+    // make every |d_c| < 2^(62 - lg), so the n_ctx terms sum to less than
+    // 2^62.  Scaling by a power of two (ldexp) is exact at any magnitude.
+    int e = 0;
+    frexp(mx, &e);
+    const int shift = lg - 62 + e;
+    if (blockIdx.x == 0 && threadIdx.x == 0) p.tot->shift = shift;
+    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < p.n_ctx;
+         c += (long long)cluster_blocks * blockDim.x) {
+      const int k = p.cluster[c];
+      if (k < 0 || k >= p.n_clusters || p.ctx_n[c] <= 0) continue;  // bad ids are flagged by the totals
+      const double d = p.ctx_d[c];
+      if (fabs(d) <= DBL_MAX) {
+        atomicAdd(reinterpret_cast<unsigned long long*>(p.Dq + k), (unsigned long long)__double2ll_rn(ldexp(d, -shift)));
+      } else {
+        atomicOr(p.Dflag + k, d != d ? kFlagNaN : (d > 0.0 ? kFlagPosInf : kFlagNegInf));
       }
-    }
-    D = warp_sum(D);
-    N = warp_sum(N);
-    if (lane == 0 && k < p.n_clusters) {
-      p.Dk[k] = D;
-      p.Nk[k] = N;
+      atomicAdd(reinterpret_cast<unsigned long long*>(p.Nk + k), 1ull);
     }
     return;
   }
@@ -253,6 +293,15 @@ __global__ void __launch_bounds__(kThreads) paired_cluster_kernel(const PairedPa
   }
 }
 
+// D[k] from its fixed-point sum, or the IEEE sum of its non-finite
+// differences (NaN when it holds NaN or both infinities).
+__device__ __forceinline__ double cluster_sum(const PairedParams& p, int k, int shift) {
+  const int f = p.Dflag[k];
+  if (f == 0) return ldexp((double)p.Dq[k], shift);
+  if ((f & kFlagNaN) || (f & (kFlagPosInf | kFlagNegInf)) == (kFlagPosInf | kFlagNegInf)) return CUDART_NAN;
+  return (f & kFlagPosInf) ? CUDART_INF : -CUDART_INF;
+}
+
 // One warp per replicate; the clusters' sums sit in shared memory when
 // there are at most kBootSmemClusters of them.  Draws are loaded four per
 // lane before their sums are gathered.
@@ -261,45 +310,50 @@ __global__ void __launch_bounds__(kBootThreads) paired_boot_kernel(const PairedP
   __shared__ int sN[kBootSmemClusters];  // counts of contexts, < 2^31
   wait_prior_grid();
   const bool staged = p.n_clusters <= kBootSmemClusters;
+  const int shift = p.tot->shift;
   if (staged) {
     for (int k = threadIdx.x; k < p.n_clusters; k += blockDim.x) {
-      sD[k] = p.Dk[k];
+      sD[k] = cluster_sum(p, k, shift);
       sN[k] = (int)p.Nk[k];
     }
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
-  const long long r = (long long)blockIdx.x * (kBootThreads / 32) + (threadIdx.x >> 5);
-  const int32_t* draws = p.resample + r * p.n_clusters;
-  const int C = (r < p.n_boot) ? p.n_clusters : 0;  // warps past the last replicate idle
-  double D = 0.0;
-  long long N = 0;
+  // a fixed grid (one wave); warps stride over the replicates
+  const long long n_warps = (long long)gridDim.x * (kBootThreads / 32);
   bool bad = false;
-  constexpr int U = 4;
-  for (int j0 = lane; j0 < C; j0 += 32 * U) {
-    int k[U];
+  for (long long r = (long long)blockIdx.x * (kBootThreads / 32) + (threadIdx.x >> 5); r < p.n_boot;
+       r += n_warps) {
+    const int32_t* draws = p.resample + r * p.n_clusters;
+    const int C = p.n_clusters;
+    double D = 0.0;
+    long long N = 0;
+    constexpr int U = 4;  // draws in flight per lane
+    for (int j0 = lane; j0 < C; j0 += 32 * U) {
+      int k[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) k[u] = (j0 + 32 * u < C) ? __ldcs(draws + j0 + 32 * u) : 0;
+      for (int u = 0; u < U; ++u) k[u] = (j0 + 32 * u < C) ? __ldcs(draws + j0 + 32 * u) : 0;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (j0 + 32 * u >= C) continue;
-      if (k[u] < 0 || k[u] >= C) {
-        bad = true;
-        continue;
-      }
-      if (staged) {
-        D += sD[k[u]];
-        N += sN[k[u]];
-      } else {
-        D += __ldg(p.Dk + k[u]);
-        N += __ldg(p.Nk + k[u]);
+      for (int u = 0; u < U; ++u) {
+        if (j0 + 32 * u >= C) continue;
+        if (k[u] < 0 || k[u] >= C) {
+          bad = true;
+          continue;
+        }
+        if (staged) {
+          D += sD[k[u]];
+          N += sN[k[u]];
+        } else {
+          D += cluster_sum(p, k[u], shift);
+          N += __ldg(p.Nk + k[u]);
+        }
       }
     }
+    D = warp_sum(D);
+    N = warp_sum(N);
+    if (lane == 0) p.boot[r] = N ? D / (double)N : CUDART_NAN;
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_dev_status(p.dev_status, 0x2 /* KLD_DEV_BAD_ID */);
-  D = warp_sum(D);
-  N = warp_sum(N);
-  if (lane == 0 && r < p.n_boot) p.boot[r] = N ? D / (double)N : CUDART_NAN;
 }
 
 // Exact order statistics of the replicate statistics (NaN left out) at the
@@ -383,7 +437,10 @@ struct KeySrc {
   }
 };
 
-__global__ void __launch_bounds__(kSelThreads) paired_select_kernel(const PairedParams p) {
+__device__ void finish_warp(const PairedParams& p, int n_parts);
+
+// (its last step writes the result, so no separate launch is needed)
+__global__ void __launch_bounds__(kSelThreads) paired_select_kernel(const PairedParams p, int n_parts) {
   __shared__ SelShared S;
   extern __shared__ __align__(16) unsigned long long sk[];  // kStageKeys keys when staged
   wait_prior_grid();
@@ -420,7 +477,11 @@ __global__ void __launch_bounds__(kSelThreads) paired_select_kernel(const Paired
   for (int j = 0; j < nw; ++j) n += S.ru[j];
   __syncthreads();
   if (tid == 0) p.tot->n_valid = (unsigned)n;
-  if (n == 0) return;
+  if (n == 0) {  // no replicate to rank: the result alone
+    __syncthreads();
+    if (tid < 32) finish_warp(p, n_parts);
+    return;
+  }
   const KeySrc src{p.boot, staged ? sk : nullptr};
   const int nt = 2 * p.nq;
 
@@ -614,13 +675,16 @@ __global__ void __launch_bounds__(kSelThreads) paired_select_kernel(const Paired
     if (tid == 0) p.tot->ostat[t] = dval(ans);
     __syncthreads();
   }
+  __syncthreads();  // the statistics above are written; one warp writes the result
+  if (tid < 32) finish_warp(p, n_parts);
 }
 
 // One warp: the chunks' sums (lane l adds chunks l, l + 32, ... in order,
 // then a fixed tree), the interval ends, the result.
-__global__ void paired_finish_kernel(const PairedParams p, int n_parts) {
-  wait_prior_grid();
-  const int lane = threadIdx.x;
+// The result, written by one warp: the totals' chunks added in order, the
+// interval ends from the replicates' order statistics.
+__device__ void finish_warp(const PairedParams& p, int n_parts) {
+  const int lane = threadIdx.x & 31;
   const PairedTotals* t = p.tot;
   kld_paired* o = p.out;
   const double nan = CUDART_NAN;
@@ -671,6 +735,11 @@ __global__ void paired_finish_kernel(const PairedParams p, int n_parts) {
   }
 }
 
+__global__ void paired_finish_kernel(const PairedParams p, int n_parts) {
+  wait_prior_grid();
+  finish_warp(p, n_parts);
+}
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
@@ -680,9 +749,10 @@ size_t paired_workspace_bytes(int64_t n_ctx, int32_t n_clusters, int32_t n_boot)
   const size_t k = n_clusters > 0 ? (size_t)n_clusters : 0;
   const size_t b = n_boot > 0 ? (size_t)n_boot : 0;
   const size_t parts = (nc + kTotChunk - 1) / kTotChunk + 1;
+  const size_t blocks = (nc + kWarps - 1) / kWarps + 1;
   return align256(sizeof(PairedTotals)) + align256(sizeof(PairedPart) * parts) + 3 * align256(sizeof(double) * nc) +
-         align256(sizeof(int32_t) * nc) +
-         align256(sizeof(double) * k) + align256(sizeof(long long) * k) + align256(sizeof(double) * b);
+         align256(sizeof(int32_t) * nc) + align256(sizeof(double) * blocks) + align256(sizeof(long long) * k) +
+         align256(sizeof(int32_t) * k) + align256(sizeof(long long) * k) + align256(sizeof(double) * b);
 }
 
 cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
@@ -715,31 +785,37 @@ cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
   ws += align256(sizeof(double) * nc);
   p.ctx_n = reinterpret_cast<int32_t*>(ws);
   ws += align256(sizeof(int32_t) * nc);
-  p.Dk = reinterpret_cast<double*>(ws);
-  ws += align256(sizeof(double) * k);
+  const unsigned ctx_grid = (unsigned)((nc + kWarps - 1) / kWarps);
+  p.n_ctx_blocks = ctx_grid > 0 ? (int)ctx_grid : 1;
+  p.blk_max = reinterpret_cast<double*>(ws);
+  ws += align256(sizeof(double) * (size_t)(p.n_ctx_blocks + 1));
+  p.Dq = reinterpret_cast<long long*>(ws);
+  ws += align256(sizeof(long long) * k);
+  p.Dflag = reinterpret_cast<int32_t*>(ws);
+  ws += align256(sizeof(int32_t) * k);
   p.Nk = reinterpret_cast<long long*>(ws);
   ws += align256(sizeof(long long) * k);
   p.boot = a.boot_stats ? a.boot_stats : reinterpret_cast<double*>(ws);
 
   cudaError_t e = cudaSuccess;
-  const unsigned ctx_grid = (unsigned)((nc + kWarps - 1) / kWarps);
   if (ctx_grid > 0) e = launch_dependent(paired_ctx_kernel, dim3(ctx_grid), dim3(kThreads), stream, p);
   else e = launch_dependent(paired_ctx_kernel, dim3(1), dim3(kThreads), stream, p);  // clears the counter
   if (e != cudaSuccess) return e;
-  const int cluster_blocks = (int)((k + kWarps - 1) / kWarps);
+  // one thread per context, at most 128 blocks (grid-stride beyond)
+  const int cluster_blocks = (int)std::min<size_t>((nc + kThreads - 1) / kThreads, 128) + (nc == 0 ? 1 : 0);
   e = launch_dependent(paired_cluster_kernel, dim3(cluster_blocks + n_parts), dim3(kThreads), stream, p,
                        cluster_blocks);
   if (e != cudaSuccess) return e;
   if (b > 0) {
     constexpr int kBootWarps = kBootThreads / 32;
-    e = launch_dependent(paired_boot_kernel, dim3((unsigned)((b + kBootWarps - 1) / kBootWarps)),
-                         dim3(kBootThreads), stream, p);
+    // at most two 1024-thread CTAs per SM of a 148-SM part: one wave
+    const size_t boot_blocks = std::min<size_t>((b + kBootWarps - 1) / kBootWarps, 2 * 148);
+    e = launch_dependent(paired_boot_kernel, dim3((unsigned)boot_blocks), dim3(kBootThreads), stream, p);
     if (e != cudaSuccess) return e;
     e = allow_dynamic_smem<paired_select_kernel>(sizeof(unsigned long long) * kStageKeys);
     if (e != cudaSuccess) return e;
     const size_t smem = (b <= (size_t)kStageKeys) ? sizeof(unsigned long long) * b : 0;
-    e = launch_dependent_smem(paired_select_kernel, dim3(1), dim3(kSelThreads), smem, stream, p);
-    if (e != cudaSuccess) return e;
+    return launch_dependent_smem(paired_select_kernel, dim3(1), dim3(kSelThreads), smem, stream, p, n_parts);
   }
   return launch_dependent(paired_finish_kernel, dim3(1), dim3(32), stream, p, n_parts);
 }

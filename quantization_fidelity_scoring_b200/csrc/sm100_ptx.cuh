@@ -1,7 +1,8 @@
-// Thin inline-PTX wrappers for the sm_100a features the shared-head kernel
-// uses: mbarriers with time-bounded waits, 2-D TMA tile loads (no cluster
-// multicast), and the tcgen05 tensor-core path (TMEM allocation, MMA with
-// shared-memory descriptors, commit to an mbarrier, TMEM loads, fences).
+// Thin inline-PTX wrappers for the sm_100a features the kernels use:
+// mbarriers with time-bounded waits, 1-D bulk copies and 2-D TMA tile loads
+// (no cluster multicast), and the tcgen05 tensor-core path (TMEM allocation,
+// MMA with shared-memory descriptors, commit to an mbarrier, TMEM loads,
+// fences).
 #pragma once
 
 #include <cstdint>
@@ -72,6 +73,16 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* t
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(smem_addr(smem_dst)), "l"(tmap), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// 1-D bulk copy of `bytes` (a multiple of 16, both addresses 16-byte
+// aligned) from global to shared memory, counted on `bar` in bytes; no
+// cluster multicast.
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gmem_src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
 

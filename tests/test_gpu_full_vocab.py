@@ -7,6 +7,7 @@ import torch
 
 import quantization_fidelity_scoring_b200 as kq
 from oracle import kld_oracle as O
+from oracle.pool import OraclePool, concat
 from synth import workloads as W
 from tests.helpers import assert_kl_close, assert_lp_close, check_full_vocab, to_f64
 
@@ -73,25 +74,42 @@ def test_one_window_bf16_full_size(cuda_device):
     check_full_vocab(res, X, Y, d["targets"].cpu().numpy())
 
 
-def test_batched_f32_full_size_sampled(cuda_device):
-    """16 windows x 2047 rows of f32 logits (65 GB): 192 seeded rows plus every
-    row whose candidate argmax was forced to differ, against the oracle."""
+def oracle_streamed(ref, cand, targets, kind, chunk_rows=512):
+    """The f64 oracle over every row of device inputs too large for the host
+    at once: row chunks (~1 GB at 512 rows of 248,320 f32 per side) are
+    copied back and staged while the previous chunk is scored by one oracle
+    process per host core."""
+    n = ref.shape[0]
+    parts, pending = [], None
+    with OraclePool() as pool:
+        for i, a in enumerate(range(0, n, chunk_rows)):
+            b, tag = min(n, a + chunk_rows), i % 2
+            staged = {"X": pool.stage(f"x{tag}", ref[a:b], kind), "Y": pool.stage(f"y{tag}", cand[a:b], kind),
+                      "targets": pool.stage(f"t{tag}", targets[a:b], "int")}
+            job = pool.run_async("full_vocab", staged, b - a, rows_per_job=8)
+            if pending is not None:
+                parts.append(concat(pending.get()))   # the chunk staged two rounds ago is free again
+            pending = job
+        parts.append(concat(pending.get()))
+    return {k: np.concatenate([p[k] for p in parts]) for k in parts[0]}
+
+
+def test_batched_f32_full_size_all_rows(cuda_device):
+    """16 windows x 2047 rows of f32 logits (65 GB): every one of the 32,752
+    rows against the oracle, and every row whose candidate argmax was forced
+    to differ does differ."""
     d = W.batched_full_vocab(device=cuda_device)
     res = run(d["ref"], d["cand"], d["targets"])
     assert res["status"] == 0
-    n = d["ref"].shape[0]
-    g = torch.Generator().manual_seed(7)
-    rows = torch.randperm(n, generator=g)[:192]
-    rows = torch.unique(torch.cat([rows, d["forced_rows"].cpu(), torch.tensor([0, n - 1])])).numpy()
-    X = to_f64(d["ref"][torch.as_tensor(rows, device=cuda_device)])
-    Y = to_f64(d["cand"][torch.as_tensor(rows, device=cuda_device)])
-    T = d["targets"].cpu().numpy()[rows]
-    check_full_vocab(res, X, Y, T, rows=rows)
-    forced = d["forced_rows"].cpu().numpy()
+    want = oracle_streamed(d["ref"], d["cand"], d["targets"], "f32")
+    assert_kl_close(res["kl"].cpu().numpy(), want["kl"])
     ra = res["ref_argmax"].cpu().numpy()
     ca = res["cand_argmax"].cpu().numpy()
-    assert np.all(ra[forced] != ca[forced])
-    # every KL is finite and non-negative up to the tolerance, at full size
+    assert np.array_equal(ra, want["ref_argmax"]) and np.array_equal(ca, want["cand_argmax"])
+    assert_lp_close(res["ref_target_lp"].cpu().numpy(), want["ref_target_lp"], "ref lp")
+    assert_lp_close(res["cand_target_lp"].cpu().numpy(), want["cand_target_lp"], "cand lp")
+    forced = d["forced_rows"].cpu().numpy()
+    assert len(forced) > 0 and np.all(ra[forced] != ca[forced])
     kl = res["kl"].cpu().numpy()
     assert np.all(np.isfinite(kl)) and kl.min() >= -1e-5
 
