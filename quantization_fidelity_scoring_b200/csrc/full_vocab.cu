@@ -117,22 +117,6 @@ __device__ __forceinline__ float side_new_max(WarpSide& s, float cm, const uint4
   return sc;
 }
 
-// The exponent offset of a side: c = -m log2(e) rounded to f32 (0 before a
-// finite value), so a weight is 2^(z log2(e) + c) from one fused
-// multiply-add; c misses -m log2(e) by rho = -m log2(e) - c (exact, from a
-// second fused multiply-add), so those weights are exp(z - m) 2^-rho, and
-// sums formed with c are multiplied by fix = 2^rho when they join the row's.
-struct Offset {
-  float c, fix;
-};
-
-__device__ __forceinline__ Offset offset_of(const WarpSide& s) {
-  if (s.a < 0) return Offset{0.f, 1.f};
-  const float c = __fmul_rn(-s.m, kLog2e);
-  const float rho = fmaf(-s.m, kLog2e, -c);
-  return Offset{c, ex2(rho)};
-}
-
 // Accumulate one step: weights exp(z - m) 2^-rho on paired f32x2 arithmetic
 // (see Offset; cx, cy are the sides' offsets c).  With
 // kMasked, the slots ex_x / ex_y (the new argmaxes) are weighed as -inf so

@@ -39,7 +39,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxTargets = 2 * KLD_MAX_QUANTILES;
-constexpr int kBootThreads = 1024;
+constexpr int kBootThreads = 512;
 constexpr int kBootSmemClusters = 2048;  // clusters whose sums a boot CTA keeps in shared memory
 
 constexpr int kTotChunk = 1024;  // contexts per totals block
@@ -305,7 +305,7 @@ __device__ __forceinline__ double cluster_sum(const PairedParams& p, int k, int 
 // One warp per replicate; the clusters' sums sit in shared memory when
 // there are at most kBootSmemClusters of them.  Draws are loaded four per
 // lane before their sums are gathered.
-__global__ void __launch_bounds__(kBootThreads) paired_boot_kernel(const PairedParams p) {
+__global__ void __launch_bounds__(kBootThreads, 2) paired_boot_kernel(const PairedParams p) {
   __shared__ double sD[kBootSmemClusters];
   __shared__ int sN[kBootSmemClusters];  // counts of contexts, < 2^31
   wait_prior_grid();
@@ -328,25 +328,44 @@ __global__ void __launch_bounds__(kBootThreads) paired_boot_kernel(const PairedP
     const int C = p.n_clusters;
     double D = 0.0;
     long long N = 0;
-    constexpr int U = 4;  // draws in flight per lane
-    for (int j0 = lane; j0 < C; j0 += 32 * U) {
-      int k[U];
+    // the row's draws: up to three before its first 16-byte boundary and up
+    // to three after its last one one by one, the rest as 16-byte vectors,
+    // kVecRound per lane issued together (one round trip for rows of up to
+    // 32 * 4 * kVecRound draws); nothing outside the row is read
+    constexpr int kVecRound = 7;
+    const int head = min(C, (int)((4 - ((reinterpret_cast<uintptr_t>(draws) >> 2) & 3)) & 3));
+    const int nvec = (C - head) >> 2;
+    const int tail = C - head - 4 * nvec;
+    const int4* dv = reinterpret_cast<const int4*>(draws + head);
+    auto take = [&](int k) {
+      if (k < 0 || k >= C) {
+        bad = true;
+        return;
+      }
+      if (staged) {
+        D += sD[k];
+        N += sN[k];
+      } else {
+        D += cluster_sum(p, k, shift);
+        N += __ldg(p.Nk + k);
+      }
+    };
+    if (lane < head) take(__ldcs(draws + lane));
+    if (lane < tail) take(__ldcs(draws + head + 4 * nvec + lane));
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kVecRound) {
+      int4 q[kVecRound];
 #pragma unroll
-      for (int u = 0; u < U; ++u) k[u] = (j0 + 32 * u < C) ? __ldcs(draws + j0 + 32 * u) : 0;
+      for (int u = 0; u < kVecRound; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < nvec) q[u] = __ldcs(dv + v);
+      }
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (j0 + 32 * u >= C) continue;
-        if (k[u] < 0 || k[u] >= C) {
-          bad = true;
-          continue;
-        }
-        if (staged) {
-          D += sD[k[u]];
-          N += sN[k[u]];
-        } else {
-          D += cluster_sum(p, k[u], shift);
-          N += __ldg(p.Nk + k[u]);
-        }
+      for (int u = 0; u < kVecRound; ++u) {
+        if (v0 + 32 * u >= nvec) continue;
+        take(q[u].x);
+        take(q[u].y);
+        take(q[u].z);
+        take(q[u].w);
       }
     }
     D = warp_sum(D);
@@ -808,7 +827,7 @@ cudaError_t launch_paired(const PairedArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (b > 0) {
     constexpr int kBootWarps = kBootThreads / 32;
-    // at most two 1024-thread CTAs per SM of a 148-SM part: one wave
+    // at most two 512-thread CTAs per SM of a 148-SM part: one wave
     const size_t boot_blocks = std::min<size_t>((b + kBootWarps - 1) / kBootWarps, 2 * 148);
     e = launch_dependent(paired_boot_kernel, dim3((unsigned)boot_blocks), dim3(kBootThreads), stream, p);
     if (e != cudaSuccess) return e;

@@ -47,6 +47,7 @@ constexpr int kMinVecsPerWarp = 4 * kStepVecs;
 constexpr int kStreamCtasPerSm = 3;
 constexpr int kMaxStreamWarps = 148 * kStreamCtasPerSm * kWarpsPerCta;
 constexpr int kWin = 256;                        // steps per bucket window
+constexpr int kFlushSteps = 16;                  // steps whose sums meet before joining the piece's
 constexpr int kMaxK = KLD_SPARSE_MAX_K;
 constexpr int kFlagRepeat = 1;
 constexpr uint32_t kSkip = 0x80000000u;
@@ -104,13 +105,14 @@ struct WarpLists {
 };
 static_assert(sizeof(uint32_t) * (kWin + 1) <= sizeof(uint4) * kStepVecs, "counts fit in the stage");
 
-// Weights exp(y - mo) of a lane's step, added to r2.  With kMasked the
+// Weights exp(y - m) 2^-rho of a lane's step (one paired FMA per pair for
+// the exponent, y log2 e + c; see Offset), added to r2.  With kMasked the
 // element slot `excl` (a new argmax) is weighed as -inf.
 template <bool kBF16, bool kMasked>
-__device__ __forceinline__ void accumulate(const uint4 (&v)[kVecs], float mo, int excl, float2& r2) {
+__device__ __forceinline__ void accumulate(const uint4 (&v)[kVecs], float c, int excl, float2& r2) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
-  const float2 nm = make_float2(-mo, -mo);
+  const float2 nm = make_float2(c, c);
   const float2 l2 = make_float2(kLog2e, kLog2e);
 #pragma unroll
   for (int q = 0; q < kVecs; ++q) {
@@ -121,7 +123,7 @@ __device__ __forceinline__ void accumulate(const uint4 (&v)[kVecs], float mo, in
         if (excl == q * E + 2 * k) Y.x = -CUDART_INF_F;
         if (excl == q * E + 2 * k + 1) Y.y = -CUDART_INF_F;
       }
-      const float2 t = __fmul2_rn(__fadd2_rn(Y, nm), l2);
+      const float2 t = __ffma2_rn(Y, l2, nm);
       r2 = __fadd2_rn(r2, make_float2(ex2(t.x), ex2(t.y)));
     }
   }
@@ -207,8 +209,18 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
   const int2* top = p.top + (int64_t)row * p.K;
   float* gy = p.gy + (int64_t)row * p.K;
 
+  // r2 holds the lane's step weights (formed with the offset o) for at most
+  // kFlushSteps steps, then joins s.r times o.fix: no f32 sum gets more than
+  // about a hundred terms however long the row
   WarpSide s{-CUDART_INF_F, -1, 0.f};
+  Offset o{0.f, 1.f};
   float2 r2 = make_float2(0.f, 0.f);
+  int since = 0;
+  auto fold = [&]() {
+    s.r += (r2.x + r2.y) * o.fix;
+    r2 = make_float2(0.f, 0.f);
+    since = 0;
+  };
   int flags = 0;
   const int n = b - a;
   const int nsteps = (n + kStepVecs - 1) / kStepVecs;
@@ -284,13 +296,13 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
       }
       const float CM = warp_max(cm);
       if (!(CM > s.m)) {  // warp-uniform: the common step
-        accumulate<kBF16, false>(v, (s.a < 0) ? 0.f : s.m, -1, r2);
+        accumulate<kBF16, false>(v, o.c, -1, r2);
+        if (++since == kFlushSteps) fold();
         continue;
       }
       // a new maximum: fold the pair sums, rescale to the new maximum, hand
       // the old maximum's own term to lane 0, find the first occurrence
-      s.r += r2.x + r2.y;
-      r2 = make_float2(0.f, 0.f);
+      fold();
       const float sc = (s.a < 0) ? 0.f : ex2((s.m - CM) * kLog2e);
       s.r = s.r * sc + ((lane == 0 && s.a >= 0) ? sc : 0.f);
       int part = kVecs - 1, src = 0;
@@ -320,11 +332,13 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
       }
       s.a = __shfl_sync(0xffffffffu, idx, src);
       s.m = CM;
-      accumulate<kBF16, true>(v, s.m, excl, r2);
+      o = offset_of(s);
+      accumulate<kBF16, true>(v, o.c, excl, r2);
     }
     __syncwarp();  // the lists are rebuilt for the next window
   }
-  float rs = s.r + (r2.x + r2.y);
+  fold();
+  float rs = s.r;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
   flags = __reduce_or_sync(0xffffffffu, flags);

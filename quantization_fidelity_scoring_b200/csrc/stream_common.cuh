@@ -7,6 +7,8 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "kld_common.cuh"
+
 namespace kld {
 
 // First flattened vector of warp w when `total` vectors are split evenly
@@ -109,5 +111,21 @@ struct WarpSide {
   int a;
   float r;
 };
+
+// The exponent offset of a side: c = -m log2(e) rounded to f32 (0 before a
+// finite value), so a weight is 2^(z log2(e) + c) from one fused
+// multiply-add; c misses -m log2(e) by rho = -m log2(e) - c (exact, from a
+// second fused multiply-add), so those weights are exp(z - m) 2^-rho, and
+// sums formed with c are multiplied by fix = 2^rho when they join the row's.
+struct Offset {
+  float c, fix;
+};
+
+__device__ __forceinline__ Offset offset_of(const WarpSide& s) {
+  if (s.a < 0) return Offset{0.f, 1.f};
+  const float c = __fmul_rn(-s.m, kLog2e);
+  const float rho = fmaf(-s.m, kLog2e, -c);
+  return Offset{c, ex2(rho)};
+}
 
 }  // namespace kld
