@@ -84,15 +84,16 @@ def _row_is_valid(z: np.ndarray) -> bool:
 
 
 def log_softmax(z: np.ndarray) -> np.ndarray:
-    """log p_i = z_i - log sum_j exp(z_j), computed around the row maximum.
+    """log p_i = z_i - log sum_j exp(z_j), computed around the row maximum m
+    as (z_i - m) - log sum_j exp(z_j - m).
 
     "Qwen3.8-27B Quantization Challenge", "How the references were made":
     the model's distribution over the whole vocabulary is the softmax of its
     logits.  The caller has checked that z holds a finite maximum.
     """
     m = np.max(z)
-    lse = m + math.log(float(np.sum(np.exp(z - m))))
-    return z - lse
+    log_s = math.log(float(np.sum(np.exp(z - m))))
+    return (z - m) - log_s          # z - m first: m + log_s would lose log_s when |m| is huge
 
 
 def full_vocab_row(x: np.ndarray, y: np.ndarray, target: int | None = None) -> dict:

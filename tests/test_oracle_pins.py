@@ -124,6 +124,21 @@ def pin_argmax_lowest_index(O):
     assert r["ref_argmax"] == 1 and r["cand_argmax"] == 0
 
 
+def pin_huge_logits_keep_the_normaliser(O):
+    # ties at a maximum near the largest f32 value: log p of each of the k
+    # tied ids is -ln k exactly, whatever the magnitude of the maximum
+    for base in (3.0e38, -3.0e38, 1.0e30, 0.0):
+        V = 50
+        x = np.full(V, -3.3e38 if base > -3.0e38 else -3.4e38)
+        y = x.copy()
+        x[[3, 7, 11]] = base
+        y[[3, 7, 11, 20]] = base
+        r = O.full_vocab_row(x, y, 7)
+        assert _close(r["ref_target_lp"], -math.log(3), rtol=1e-14)
+        assert _close(r["cand_target_lp"], -math.log(4), rtol=1e-14)
+        assert _close(r["kl"], math.log(4 / 3), rtol=1e-12)
+
+
 def pin_uniform_target(O):
     for V in (3, 4096):
         r = O.full_vocab_row(np.zeros(V), np.full(V, 2.5), 1)
@@ -753,9 +768,8 @@ def test_golden_bf16_self_scores():
 MUTANTS = [
     ("KL direction reversed", "terms = p[live] * (lp[live] - lq[live])",
      "terms = np.exp(lq[live]) * (lq[live] - lp[live])"),
-    ("log-softmax sign", "return z - lse", "return z + lse"),
-    ("normaliser without max", "lse = m + math.log(float(np.sum(np.exp(z - m))))",
-     "lse = math.log(float(np.sum(np.exp(z - m))))"),
+    ("log-softmax sign", "return (z - m) - log_s", "return (z - m) + log_s"),
+    ("normaliser without max", "return (z - m) - log_s", "return z - log_s"),
     ("argmax picks the last tie", "out[\"ref_argmax\"] = int(np.argmax(x))",
      "out[\"ref_argmax\"] = int(x.shape[0] - 1 - np.argmax(x[::-1]))"),
     ("candidate target from the reference", "out[\"cand_target_lp\"] = float(lq[t])",
