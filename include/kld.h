@@ -119,6 +119,10 @@ const char* kld_status_string(kld_status s);
  * NaN or +inf, or no finite logit, gives kl = NaN, argmax = -1 and NaN
  * target lps.  A target id outside [0, vocab) gives NaN target lps and sets
  * KLD_DEV_BAD_TARGET.
+ * Range: differences ref_i - cand_i and z_i - max(z) are formed in f32, so
+ * finite logits of any magnitude are scored as long as those differences
+ * stay within the f32 range (always so when every |logit| <= 1.7e38); a
+ * row where one overflows may give kl = inf or NaN.
  */
 kld_status kld_full_vocab(const void* ref_logits, const void* cand_logits, kld_dtype dtype,
                           int64_t n_rows, int64_t vocab, int64_t ld_ref, int64_t ld_cand,
@@ -241,6 +245,9 @@ kld_status kld_topk_tail(const int32_t* ref_ids, const uint16_t* ref_lp,
  * [0, vocab), or repeated within a row, gives kl NaN and sets
  * KLD_DEV_BAD_ID; a target outside [0, vocab) gives a NaN target log-prob
  * and sets KLD_DEV_BAD_TARGET.
+ * Range: differences z_i - max(z) of the candidate's logits are formed in
+ * f32, so finite logits of any magnitude are scored as long as those stay
+ * within the f32 range (always so when every |logit| <= 1.7e38).
  */
 #define KLD_SPARSE_MAX_K 1024
 typedef struct {

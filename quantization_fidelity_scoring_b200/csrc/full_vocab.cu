@@ -122,7 +122,7 @@ __device__ __forceinline__ float side_new_max(WarpSide& s, float cm, const uint4
 // kMasked, the slots ex_x / ex_y (the new argmaxes) are weighed as -inf so
 // they stay out of r; the reference argmax's own A term, 1 * (x - y), is
 // added by the caller.
-template <bool kBF16, bool kMasked>
+template <bool kBF16, bool kMasked, bool kExact>
 __device__ __forceinline__ void accumulate(const StepRaw& raw, float cx, float cy, int ex_x, int ex_y,
                                            float2& rx2, float2& ry2, float2& a2) {
   using El = Elems<kBF16>;
@@ -145,8 +145,9 @@ __device__ __forceinline__ void accumulate(const StepRaw& raw, float cx, float c
         if (ex_y == j) YW.x = -CUDART_INF_F;
         if (ex_y == j + 1) YW.y = -CUDART_INF_F;
       }
-      const float2 tx = __ffma2_rn(XW, l2, nmx);  // x log2(e) + c, one rounding
-      const float2 ty = __ffma2_rn(YW, l2, nmy);
+      // x log2(e) + c, one rounding (exact offsets: (x - m) log2(e))
+      const float2 tx = kExact ? __fmul2_rn(__fadd2_rn(XW, nmx), l2) : __ffma2_rn(XW, l2, nmx);
+      const float2 ty = kExact ? __fmul2_rn(__fadd2_rn(YW, nmy), l2) : __ffma2_rn(YW, l2, nmy);
       const float2 ex = make_float2(ex2(tx.x), ex2(tx.y));
       const float2 ey = make_float2(ex2(ty.x), ex2(ty.y));
       rx2 = __fadd2_rn(rx2, ex);
@@ -194,7 +195,7 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
   // the row: a row's thousands of terms in one running sum lost up to 1e-5 of
   // a target log-prob.
   WarpSide sx{-CUDART_INF_F, -1, 0.f}, sy{-CUDART_INF_F, -1, 0.f};
-  Offset ox{0.f, 1.f}, oy{0.f, 1.f};
+  Offset ox{0.f, 1.f, false}, oy{0.f, 1.f, false};
   float2 rx2 = make_float2(0.f, 0.f), ry2 = rx2, a2 = rx2;
   float aA = 0.f;
   int since = 0;
@@ -222,7 +223,8 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
     const float CMX = warp_max(El::vmax2(cur.x0, cur.x1));
     const float CMY = warp_max(El::vmax2(cur.y0, cur.y1));
     if (!((CMX > sx.m) || (CMY > sy.m) || (sx.a < 0) || (sy.a < 0))) {  // warp-uniform
-      accumulate<kBF16, false>(cur, ox.c, oy.c, -1, -1, rx2, ry2, a2);
+      if (!ox.exact) accumulate<kBF16, false, false>(cur, ox.c, oy.c, -1, -1, rx2, ry2, a2);
+      else accumulate<kBF16, false, true>(cur, ox.c, oy.c, -1, -1, rx2, ry2, a2);
     } else {
       // the per-vector maxima locate a new maximum (rare: computed only here)
       const float cx0 = El::vmax(cur.x0), cx1 = El::vmax(cur.x1);
@@ -240,9 +242,9 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
       if (ex_x >= 0) aA += slot_diff<kBF16>(cur, ex_x);
       // a side with no finite value yet has only -inf (weight 0) or NaN
       // (poisons r, marking the row invalid); any finite offset serves
-      ox = offset_of(sx);
-      oy = offset_of(sy);
-      accumulate<kBF16, true>(cur, ox.c, oy.c, ex_x, ex_y, rx2, ry2, a2);
+      offsets_of(sx, sy, ox, oy);
+      if (!ox.exact) accumulate<kBF16, true, false>(cur, ox.c, oy.c, ex_x, ex_y, rx2, ry2, a2);
+      else accumulate<kBF16, true, true>(cur, ox.c, oy.c, ex_x, ex_y, rx2, ry2, a2);
     }
     if (++since == kFlushSteps) fold();  // warp-uniform
   };

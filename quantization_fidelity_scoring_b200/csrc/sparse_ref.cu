@@ -106,9 +106,10 @@ struct WarpLists {
 static_assert(sizeof(uint32_t) * (kWin + 1) <= sizeof(uint4) * kStepVecs, "counts fit in the stage");
 
 // Weights exp(y - m) 2^-rho of a lane's step (one paired FMA per pair for
-// the exponent, y log2 e + c; see Offset), added to r2.  With kMasked the
+// the exponent, y log2 e + c; see Offset; with kExact (y - m) log2 e),
+// added to r2.  With kMasked the
 // element slot `excl` (a new argmax) is weighed as -inf.
-template <bool kBF16, bool kMasked>
+template <bool kBF16, bool kMasked, bool kExact>
 __device__ __forceinline__ void accumulate(const uint4 (&v)[kVecs], float c, int excl, float2& r2) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
@@ -123,7 +124,7 @@ __device__ __forceinline__ void accumulate(const uint4 (&v)[kVecs], float c, int
         if (excl == q * E + 2 * k) Y.x = -CUDART_INF_F;
         if (excl == q * E + 2 * k + 1) Y.y = -CUDART_INF_F;
       }
-      const float2 t = __ffma2_rn(Y, l2, nm);
+      const float2 t = kExact ? __fmul2_rn(__fadd2_rn(Y, nm), l2) : __ffma2_rn(Y, l2, nm);
       r2 = __fadd2_rn(r2, make_float2(ex2(t.x), ex2(t.y)));
     }
   }
@@ -213,7 +214,7 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
   // kFlushSteps steps, then joins s.r times o.fix: no f32 sum gets more than
   // about a hundred terms however long the row
   WarpSide s{-CUDART_INF_F, -1, 0.f};
-  Offset o{0.f, 1.f};
+  Offset o{0.f, 1.f, false};
   float2 r2 = make_float2(0.f, 0.f);
   int since = 0;
   auto fold = [&]() {
@@ -296,7 +297,8 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
       }
       const float CM = warp_max(cm);
       if (!(CM > s.m)) {  // warp-uniform: the common step
-        accumulate<kBF16, false>(v, o.c, -1, r2);
+        if (!o.exact) accumulate<kBF16, false, false>(v, o.c, -1, r2);
+        else accumulate<kBF16, false, true>(v, o.c, -1, r2);
         if (++since == kFlushSteps) fold();
         continue;
       }
@@ -333,7 +335,8 @@ __device__ TailPiece stream_piece(const StreamParams& p, WarpLists& L, int row, 
       s.a = __shfl_sync(0xffffffffu, idx, src);
       s.m = CM;
       o = offset_of(s);
-      accumulate<kBF16, true>(v, o.c, excl, r2);
+      if (!o.exact) accumulate<kBF16, true, false>(v, o.c, excl, r2);
+      else accumulate<kBF16, true, true>(v, o.c, excl, r2);
     }
     __syncwarp();  // the lists are rebuilt for the next window
   }

@@ -117,15 +117,33 @@ struct WarpSide {
 // multiply-add; c misses -m log2(e) by rho = -m log2(e) - c (exact, from a
 // second fused multiply-add), so those weights are exp(z - m) 2^-rho, and
 // sums formed with c are multiplied by fix = 2^rho when they join the row's.
+// |rho| is at most half a unit in the last place of c, so the form needs a
+// small |c|: below |m| = 2^20 it is under 1/16 and t = z log2(e) + c is as
+// accurate as (z - m) log2(e); from 2^20 on it grows with |m| (2^-rho leaves
+// the f32 range near |m| = 2^31, and z log2(e) overflows near 2^127).  A side
+// with |m| >= 2^20 is therefore marked exact, and its weights are formed as
+// (z - m) log2(e) in two operations (c = -m, fix = 1).
 struct Offset {
   float c, fix;
+  bool exact;
 };
 
 __device__ __forceinline__ Offset offset_of(const WarpSide& s) {
-  if (s.a < 0) return Offset{0.f, 1.f};
+  if (s.a < 0) return Offset{0.f, 1.f, false};
+  if (!(fabsf(s.m) < 0x1p20f)) return Offset{-s.m, 1.f, true};
   const float c = __fmul_rn(-s.m, kLog2e);
   const float rho = fmaf(-s.m, kLog2e, -c);
-  return Offset{c, ex2(rho)};
+  return Offset{c, ex2(rho), false};
+}
+
+// The offsets of two sides, both in the exact form when either needs it.
+__device__ __forceinline__ void offsets_of(const WarpSide& x, const WarpSide& y, Offset& ox, Offset& oy) {
+  ox = offset_of(x);
+  oy = offset_of(y);
+  if (ox.exact || oy.exact) {
+    ox = Offset{x.a < 0 ? 0.f : -x.m, 1.f, true};
+    oy = Offset{y.a < 0 ? 0.f : -y.m, 1.f, true};
+  }
 }
 
 }  // namespace kld

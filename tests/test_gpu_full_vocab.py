@@ -226,3 +226,44 @@ def test_empty_batch(cuda_device):
     ref = torch.empty((0, 100), device=cuda_device)
     res = kq.kld_full_vocab(ref, ref.clone())
     assert res["kl"].numel() == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_logits_near_the_largest_finite_values(cuda_device, dtype):
+    """Rows whose maximum is large: near the largest finite value (where
+    x log2 e overflows f32), around 2^20 (where the one-FMA exponent gives
+    way to (x - m) log2 e) and past 2^31 (where it could not work at all):
+    ties at the maximum, values just below it, the rest far below, both
+    signs, the candidate's maximum equal to or above the reference's.  Every
+    id's difference x_i - y_i, and every x_i - m, stays finite in f32, as the
+    kernel's domain requires."""
+    V = 5000
+    rng = np.random.default_rng(123)
+    # (reference maximum, candidate maximum, fill value)
+    cases = [(3.0e38, 3.0e38, 1.0e37), (-3.0e38, -3.0e38, -3.3e38), (3.0e38, 3.2e38, 1.0e37),
+             (1.0e38, 1.0e38, -1.0e38), (-1.0e38, -1.0e38, -2.0e38), (8.4e37, 8.4e37, -8.0e37),
+             (-8.4e37, -8.0e37, -1.0e38), (1.0e9, 1.0e9, -1.0e9), (-3.0e9, -3.0e9 + 512, -3.1e9),
+             (1.0e6, 1.0e6 + 2.0, 1.0e6 - 40.0), (1.048e6, 1.048e6, 1.0e6), (3.0e6, 3.0e6, 2.9e6),
+             (-1.0e6, -1.0e6, -1.0e6 - 30.0)]
+    rows_x, rows_y, tgs = [], [], []
+    for i, (bx, by, fill) in enumerate(cases):
+        x = np.full(V, fill, dtype=np.float64)
+        some = rng.choice(V, 150, replace=False)
+        x[some[:100]] = rng.uniform(fill, fill + 0.5 * (bx - fill), 100)
+        x[some[100:]] = bx - rng.uniform(0.0, 12.0, 50)   # just below the maximum (ties where it is coarse)
+        y = x.copy()
+        tx = rng.choice(V, 3, replace=False)
+        x[tx] = bx
+        y[tx] = bx                            # x's maxima are in y too ...
+        ty = rng.choice(V, 2, replace=False)
+        y[ty] = by                            # ... with ties (or a larger maximum) of its own
+        rows_x.append(x)
+        rows_y.append(y)
+        tgs.append(int(tx[0]) if i % 2 == 0 else int(rng.integers(0, V)))
+    X = torch.tensor(np.array(rows_x), dtype=torch.float32).to(dtype).to(cuda_device)
+    Y = torch.tensor(np.array(rows_y), dtype=torch.float32).to(dtype).to(cuda_device)
+    tg = torch.tensor(tgs, dtype=torch.int32, device=cuda_device)
+    res = run(X, Y, tg)
+    assert res["status"] == 0
+    want = check_full_vocab(res, to_f64(X), to_f64(Y), tg.cpu().numpy())
+    assert np.isfinite(want["kl"]).all()

@@ -148,3 +148,40 @@ def test_edge_rows(cuda_device):
     assert np.isnan(kl[[0, 1, 2, 3, 7]]).all() and kl[4] == np.inf
     assert res["cand_argmax"][8].item() == unl and res["cand_argmax"][9].item() == lo_listed
     assert np.isnan(res["cand_target_lp"][5].item())
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_candidate_logits_near_the_largest_finite_values(cuda_device, dtype):
+    """Candidate rows whose maximum is large: near the largest finite value
+    (where y log2 e overflows f32), around 2^20 (where the one-FMA exponent
+    gives way to (y - m) log2 e) and past 2^31: ties at the maximum among
+    the listed ids, an unlisted one, values just below it, the rest far
+    below.  Every y_i - m stays finite in f32, as the kernel's domain
+    requires."""
+    V, K = 5000, 64
+    # (candidate maximum, fill value)
+    cases = [(3.0e38, 1.0e37), (-3.0e38, -3.3e38), (1.0e38, -1.0e38), (-1.0e38, -2.0e38), (8.4e37, -8.0e37),
+             (-8.4e37, -1.0e38), (1.0e9, -1.0e9), (-3.0e9, -3.1e9), (1.0e6, 1.0e6 - 40.0), (1.048e6, 1.0e6),
+             (3.0e6, 2.9e6), (-1.0e6, -1.0e6 - 30.0)]
+    d = W.sparse_ref_window(seed=W.SEED_BASE + 2500, device=cuda_device, n_rows=len(cases), vocab=V, k=K,
+                            dtype=torch.float32)
+    rng = np.random.default_rng(2500)
+    top, rows, tg = d["ref_top"], d["ref_rows"], d["targets"].clone()
+    cand = np.empty((len(cases), V))
+    for i, (m, fill) in enumerate(cases):
+        y = np.full(V, fill)
+        some = rng.choice(V, 150, replace=False)
+        y[some[:100]] = rng.uniform(fill, fill + 0.5 * (m - fill), 100)
+        y[some[100:]] = m - rng.uniform(0.0, 12.0, 50)    # just below the maximum
+        listed = top[i, :, 0].cpu().numpy()
+        unlisted = np.setdiff1d(np.arange(V), listed)
+        y[listed[[0, 5, 9]]] = m
+        y[unlisted[i]] = m
+        cand[i] = y
+        tg[i] = int(listed[0]) if i % 2 == 0 else int(unlisted[i + 1])
+    cand = torch.tensor(cand, dtype=torch.float32).to(dtype).to(cuda_device)
+    res = run(cand, top, rows, tg)
+    assert res["status"] == 0
+    want = oracle(cand, top, rows, tg)
+    check(res, want)
+    assert np.isfinite(want["kl"]).all()
