@@ -54,6 +54,7 @@ constexpr int kFinThreads = 128;     // finish: one CTA per row, 8 rows per SM
 constexpr int kSampleThreads = 256;  // sample: 16 sampled values per thread
 constexpr int kMaxK = KLD_SPARSE_MAX_K;
 constexpr int kStage = 2048;  // candidates a finish CTA keeps in shared memory
+constexpr int kTieCap = 256;  // values tied at the K-th that are ranked by counting
 
 // Tail state of one warp over one row piece (16 bytes): running maximum m
 // over all elements, and over the non-candidates T = sum e^{x-m},
@@ -638,7 +639,33 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
     return true;
   }, sc, eq, need);
   uint32_t id_cut = 0xffffffffu;
-  if (need < eq) {
+  if (need < eq && eq <= kTieCap) {
+    // the usual case: a few values tied at the K-th.  Collect their ids
+    // (sel is free until the gather below) and take the need-th lowest by
+    // counting, for each, the tied ids below it (ids are distinct)
+    uint32_t* ties = reinterpret_cast<uint32_t*>(sel);
+    if (tid == 0) sc.n_sel = 0;
+    __syncthreads();
+    for (int i0 = tid & ~31; i0 < n; i0 += kFinThreads) {  // warp-uniform: one reservation per warp
+      const int i = i0 + (tid & 31);
+      const bool tie = i < n && vkey(src.val(i)) == pre;
+      const unsigned tb = __ballot_sync(0xffffffffu, tie);
+      int base = 0;
+      if ((tid & 31) == 0 && tb) base = atomicAdd(&sc.n_sel, __popc(tb));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (tie) ties[base + __popc(tb & ((1u << (tid & 31)) - 1u))] = (uint32_t)src.idx(i);
+    }
+    __syncthreads();
+    for (int t = tid; t < eq; t += kFinThreads) {
+      const uint32_t id = ties[t];
+      int below = 0;
+      for (int u = 0; u < eq; ++u) below += ties[u] < id ? 1 : 0;
+      if (below == need - 1) sc.digit = id;  // exactly one tied id has this rank
+    }
+    __syncthreads();
+    id_cut = sc.digit;
+    __syncthreads();  // sc and sel are reused below
+  } else if (need < eq) {
     int eq2 = 0, r2 = 0;
     id_cut = ~rth_largest<0>(n, need, [&](int i, uint32_t& k) {
       k = ~(uint32_t)src.idx(i);
