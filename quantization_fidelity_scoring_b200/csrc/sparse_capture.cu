@@ -91,42 +91,54 @@ struct CapRing {
 };
 
 // Append the elements >= tau of the ring's `fill` vectors to the row's
-// candidate buffer (one atomic per 32 vectors reserves their places).
+// candidate buffer.  Lane l takes ring entries l, l + 32, ...: it counts
+// their candidates first, one warp scan of those counts gives every lane its
+// place, and one atomic reserves the whole flush (the order of a row's
+// candidates in the buffer does not matter).
 template <bool kBF16>
 __device__ void ring_flush(const CapParams& p, CapRing& R, int fill, int row, float tau, int lane) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
+  constexpr int kGroups = kRing / 32;
   int2* cand = p.cand + (int64_t)row * kCap;
   __syncwarp();
-  for (int j0 = 0; j0 < fill; j0 += 32) {  // warp-uniform
-    const int j = j0 + lane;
-    uint32_t em = 0u;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    int vid = 0;
+  uint32_t em[kGroups];
+  int mine = 0;
+#pragma unroll
+  for (int g = 0; g < kGroups; ++g) {
+    em[g] = 0u;
+    const int j = g * 32 + lane;
     if (j < fill) {
-      v = R.vec[j];
-      vid = R.vid[j];
+      const uint4 v = R.vec[j];
 #pragma unroll
       for (int k = 0; k < E / 2; ++k) {
         const float2 pr = El::pair(v, k);
-        em |= (pr.x >= tau) ? (1u << (2 * k)) : 0u;
-        em |= (pr.y >= tau) ? (1u << (2 * k + 1)) : 0u;
+        em[g] |= (pr.x >= tau) ? (1u << (2 * k)) : 0u;
+        em[g] |= (pr.y >= tau) ? (1u << (2 * k + 1)) : 0u;
       }
+      mine += __popc(em[g]);
     }
-    const int nc = __popc(em);
-    int incl = nc;
+  }
+  int incl = mine;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int o = __shfl_up_sync(0xffffffffu, incl, off);
-      if (lane >= off) incl += o;
-    }
-    const int tot = __shfl_sync(0xffffffffu, incl, 31);
-    int base = 0;
-    if (lane == 0 && tot > 0) base = atomicAdd(p.count + row, tot);
-    int pos = __shfl_sync(0xffffffffu, base, 0) + incl - nc;
-    while (em) {
-      const int e = __ffs(em) - 1;
-      em &= em - 1u;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const int tot = __shfl_sync(0xffffffffu, incl, 31);
+  int base = 0;
+  if (lane == 0 && tot > 0) base = atomicAdd(p.count + row, tot);
+  int pos = __shfl_sync(0xffffffffu, base, 0) + incl - mine;
+#pragma unroll
+  for (int g = 0; g < kGroups; ++g) {
+    uint32_t m = em[g];
+    if (m == 0u) continue;
+    const int j = g * 32 + lane;
+    const uint4 v = R.vec[j];
+    const int vid = R.vid[j];
+    while (m) {
+      const int e = __ffs(m) - 1;
+      m &= m - 1u;
       const float2 pr = El::pair(v, e >> 1);
       if (pos < kCap) cand[pos] = make_int2(__float_as_int((e & 1) ? pr.y : pr.x), vid * E + e);
       ++pos;
@@ -212,20 +224,30 @@ __device__ CapPiece cap_piece(const CapParams& p, CapRing& R, int row, int a, in
     unsigned hitq = 0u;
 #pragma unroll
     for (int q = 0; q < kVecs; ++q) hitq |= (c[q] >= tau) ? (1u << q) : 0u;
-    if (__any_sync(0xffffffffu, hitq != 0u)) {
+    const unsigned hm = __ballot_sync(0xffffffffu, hitq != 0u);
+    if (hm) {
+      // a lane's place in the ring: with at most one hit per lane (the
+      // usual case) the count of hitting lanes below it, else a warp scan
       const int nh = __popc(hitq);
-      int incl = nh;
+      int before, tot;
+      if (!__any_sync(0xffffffffu, nh > 1)) {
+        before = __popc(hm & ((1u << lane) - 1u));
+        tot = __popc(hm);
+      } else {
+        int incl = nh;
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += o;
+        for (int off = 1; off < 32; off <<= 1) {
+          const int o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        before = incl - nh;
+        tot = __shfl_sync(0xffffffffu, incl, 31);
       }
-      const int tot = __shfl_sync(0xffffffffu, incl, 31);
       if (fill + tot > kRing) {
         ring_flush<kBF16>(p, R, fill, row, tau, lane);
         fill = 0;
       }
-      int pos = fill + incl - nh;
+      int pos = fill + before;
 #pragma unroll
       for (int q = 0; q < kVecs; ++q) {
         if ((hitq >> q) & 1u) {
@@ -492,13 +514,13 @@ __device__ uint32_t rth_largest(int n, int r, KeyFn key, FinScratch& sc, int& eq
 // memory, the only stages with a barrier).
 // One stage of partners J < R apart inside a thread (J fixed at compile
 // time so the registers are addressed statically).
-template <int R, int J>
-__device__ __forceinline__ void local_stage(unsigned long long (&a)[R], int t, int kk) {
+template <int R, int J, typename Key>
+__device__ __forceinline__ void local_stage(Key (&a)[R], int t, int kk) {
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     if ((r ^ J) > r) {
       const bool desc = ((t * R + r) & kk) == 0;
-      const unsigned long long x = a[r], y = a[r ^ J];
+      const Key x = a[r], y = a[r ^ J];
       const bool sw = desc ? (x < y) : (x > y);
       a[r] = sw ? y : x;
       a[r ^ J] = sw ? x : y;
@@ -506,27 +528,27 @@ __device__ __forceinline__ void local_stage(unsigned long long (&a)[R], int t, i
   }
 }
 
-template <int R>
-__device__ void sort_desc(unsigned long long* sel) {
+template <int R, typename Key>
+__device__ void sort_desc(Key* sel) {
   const int t = threadIdx.x;
-  unsigned long long a[R];
+  Key a[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) a[r] = sel[t * R + r];
   constexpr int P = kFinThreads * R;
   for (int kk = 2; kk <= P; kk <<= 1) {
     for (int jj = kk >> 1; jj > 0; jj >>= 1) {
       if (jj < R) {
-        if (jj == 1) local_stage<R, 1>(a, t, kk);
-        else if (jj == 2) local_stage<R, (R > 2 ? 2 : 1)>(a, t, kk);
-        else local_stage<R, (R > 4 ? 4 : 1)>(a, t, kk);
+        if (jj == 1) local_stage<R, 1, Key>(a, t, kk);
+        else if (jj == 2) local_stage<R, (R > 2 ? 2 : 1), Key>(a, t, kk);
+        else local_stage<R, (R > 4 ? 4 : 1), Key>(a, t, kk);
       } else if (jj / R < 32) {
         const int tm = jj / R;
         const bool lower = (t & tm) == 0;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const unsigned long long o = __shfl_xor_sync(0xffffffffu, a[r], tm);
+          const Key o = __shfl_xor_sync(0xffffffffu, a[r], tm);
           const bool desc = ((t * R + r) & kk) == 0;
-          const unsigned long long hi = a[r] > o ? a[r] : o, lo = a[r] > o ? o : a[r];
+          const Key hi = a[r] > o ? a[r] : o, lo = a[r] > o ? o : a[r];
           a[r] = (lower == desc) ? hi : lo;
         }
       } else {
@@ -538,9 +560,9 @@ __device__ void sort_desc(unsigned long long* sel) {
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const unsigned long long o = sel[(t ^ tm) * R + r];
+          const Key o = sel[(t ^ tm) * R + r];
           const bool desc = ((t * R + r) & kk) == 0;
-          const unsigned long long hi = a[r] > o ? a[r] : o, lo = a[r] > o ? o : a[r];
+          const Key hi = a[r] > o ? a[r] : o, lo = a[r] > o ? o : a[r];
           a[r] = (lower == desc) ? hi : lo;
         }
       }
@@ -673,11 +695,21 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
     }, sc, eq2, r2);
   }
 
-  // gather the K selected as descending-sortable keys (value key, ~id)
+  // gather the K selected as descending-sortable keys and sort them.  For
+  // bf16 values the key's low 16 bits are fixed by its sign, so a 32-bit
+  // sort key holds the value's top 16 key bits over 0xffff - gather slot,
+  // and the ids stay in a table by gather slot; values tied in the sorted
+  // order are put in id order when the outputs are written.  For f32 values
+  // the keys are 64-bit: value key over ~id.
+  uint32_t* sel32 = reinterpret_cast<uint32_t*>(sel);  // [P] keys (bf16)
+  uint32_t* slot_id = sel32 + kMaxK;                    // [K] ids by gather slot (bf16)
   if (tid == 0) sc.n_sel = 0;
   int P = kFinThreads;
   while (P < K) P <<= 1;
-  for (int j = K + tid; j < P; j += kFinThreads) sel[j] = 0ull;
+  for (int j = K + tid; j < P; j += kFinThreads) {
+    if constexpr (kBF16) sel32[j] = 0u;  // below every real key: its low half is at least 0xfc00
+    else sel[j] = 0ull;
+  }
   __syncthreads();
   for (int i0 = tid & ~31; i0 < n; i0 += kFinThreads) {  // warp-uniform: one slot reservation per warp
     const int i = i0 + (tid & 31);
@@ -694,15 +726,38 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
     base = __shfl_sync(0xffffffffu, base, 0);
     if (take) {
       const int at = base + __popc(takers & ((1u << (tid & 31)) - 1u));
-      if (at < K) sel[at] = ((unsigned long long)k << 32) | (unsigned long long)(~id);
+      if (at < K) {
+        if constexpr (kBF16) {
+          sel32[at] = (k & 0xffff0000u) | (0xffffu - (uint32_t)at);
+          slot_id[at] = id;
+        } else {
+          sel[at] = ((unsigned long long)k << 32) | (unsigned long long)(~id);
+        }
+      }
     }
   }
   __syncthreads();
   // sort, descending: P = 128 R >= K slots (the padding keys are 0)
-  if (P <= kFinThreads) sort_desc<1>(sel);
-  else if (P <= 2 * kFinThreads) sort_desc<2>(sel);
-  else if (P <= 4 * kFinThreads) sort_desc<4>(sel);
-  else sort_desc<8>(sel);
+  if constexpr (kBF16) {
+    if (P <= kFinThreads) sort_desc<1>(sel32);
+    else if (P <= 2 * kFinThreads) sort_desc<2>(sel32);
+    else if (P <= 4 * kFinThreads) sort_desc<4>(sel32);
+    else sort_desc<8>(sel32);
+  } else {
+    if (P <= kFinThreads) sort_desc<1>(sel);
+    else if (P <= 2 * kFinThreads) sort_desc<2>(sel);
+    else if (P <= 4 * kFinThreads) sort_desc<4>(sel);
+    else sort_desc<8>(sel);
+  }
+  // the 32-bit value key at sorted position j
+  const auto key_at = [&](int j) -> uint32_t {
+    if constexpr (kBF16) {
+      const uint32_t hi = sel32[j] & 0xffff0000u;
+      return (hi & 0x80000000u) ? hi : (hi | 0xffffu);  // a negative value's low key bits are all ones
+    } else {
+      return (uint32_t)(sel[j] >> 32);
+    }
+  };
 
   // listed terms in sorted order (a fixed share per thread): the largest
   // has weight exactly 1 and is left out of s1 so that log S = log1p(S - 1).
@@ -710,7 +765,7 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
   const double md = (double)m;
   double s1 = 0.0, b1 = 0.0;
   for (int j = tid; j < K; j += kFinThreads) {
-    const float d = keyv((uint32_t)(sel[j] >> 32)) - m;
+    const float d = keyv(key_at(j)) - m;
     const float w = ex2(d * kLog2e);
     if (j > 0) s1 += (double)w;
     if (w > 0.f) b1 += (double)w * (double)d;
@@ -721,8 +776,8 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
   // candidates left out of the list: every one weighs at most the K-th
   // weight wK, so their sums go to 64-bit fixed point scaled to that bound
   // (exact integer sums: the order candidates arrived in does not matter)
-  const unsigned long long kth = sel[K - 1];
-  const uint32_t kkey = (uint32_t)(kth >> 32), kid = ~(uint32_t)kth;
+  // (the K-th listed value is pre; the listed ids tied with it are those up to id_cut)
+  const uint32_t kkey = pre, kid = id_cut;
   const float dKf = keyv(kkey) - m;
   const double dK = (double)dKf;
   const double wK = (double)ex2(dKf * kLog2e);
@@ -768,9 +823,21 @@ __device__ void capture_finish(const CapParams& p, int row, const Src& src, floa
   const double S = 1.0 + s_minus_1;
 
   for (int j = tid; j < K; j += kFinThreads) {
-    const unsigned long long e = sel[j];
-    const double v = (double)keyv((uint32_t)(e >> 32));
-    top[j] = kld_top_entry{(int32_t)(~(uint32_t)e), (float)((v - md) - logS)};
+    const double v = (double)keyv(key_at(j));
+    if constexpr (kBF16) {
+      // position j holds one of a run of equal values in gather order: the
+      // run's ids go out ascending
+      const uint32_t e = sel32[j], v16 = e >> 16;
+      const uint32_t id = slot_id[0xffffu - (e & 0xffffu)];
+      int lo = j, hi = j + 1;
+      while (lo > 0 && (sel32[lo - 1] >> 16) == v16) --lo;
+      while (hi < K && (sel32[hi] >> 16) == v16) ++hi;
+      int at = lo;
+      for (int u = lo; u < hi; ++u) at += slot_id[0xffffu - (sel32[u] & 0xffffu)] < id ? 1 : 0;
+      top[at] = kld_top_entry{(int32_t)id, (float)((v - md) - logS)};
+    } else {
+      top[j] = kld_top_entry{(int32_t)(~(uint32_t)sel[j]), (float)((v - md) - logS)};
+    }
   }
   if (tid == 0) {
     float nll = CUDART_NAN_F;

@@ -403,23 +403,37 @@ __global__ void __launch_bounds__(kMergeThreads) sparse_merge_kernel(const Merge
   using El = Elems<kBF16>;
   constexpr int E = El::E;
   constexpr int kElemBytes = kBF16 ? 2 : 4;
-  __shared__ float ys[kMergeWarps][kMaxK];   // listed logits
+  __shared__ float ys[kMergeWarps][kMaxK];   // listed ids, then listed logits
   __shared__ float lps[kMergeWarps][kMaxK];  // listed reference log-probs
-  wait_prior_grid();
   const int lane = threadIdx.x & 31;
   const int wl = threadIdx.x >> 5;
   const int row = blockIdx.x * kMergeWarps + wl;
-  if (row >= p.n_rows) return;
+  const bool live = row < p.n_rows;
   const char* yrow = reinterpret_cast<const char*>(p.y) + (int64_t)row * p.ld * kElemBytes;
   const int2* top = p.top + (int64_t)row * p.K;
   const float* gy = p.gy + (int64_t)row * p.K;
   float* ysw = ys[wl];
   float* lpw = lps[wl];
-  // the target logit first: its two dependent loads overlap the merge
-  const int tgt = p.lp_cand ? p.targets[row] : -1;
+  const int64_t listed_end = (int64_t)p.nvec * E;  // ids below this were captured by the stream
+
+  // Before the streaming pass is waited for, only its inputs are read: the
+  // target logit (two dependent loads) and the reference entries, whose
+  // validity is checked here
+  const int tgt = (live && p.lp_cand) ? p.targets[row] : -1;
   const bool tgt_ok = tgt >= 0 && tgt < p.vocab;
   const float y_tgt = (p.lp_cand && tgt_ok) ? El::load1(yrow, tgt) : 0.f;
-  const int64_t listed_end = (int64_t)p.nvec * E;  // ids below this were captured by the stream
+  bool bad = false;   // an id outside [0, V), or a repeated id
+  if (live) {
+#pragma unroll 8
+    for (int j = lane; j < p.K; j += 32) {
+      const int2 t = top[j];
+      bad |= t.x < 0 || t.x >= p.vocab;
+      ysw[j] = __int_as_float(t.x);
+      lpw[j] = __int_as_float(t.y);
+    }
+  }
+  wait_prior_grid();
+  if (!live) return;
 
   // tail state of the unlisted ids covered by the stream
   TailPiece acc{-CUDART_INF_F, 0.f, -1, 0};
@@ -435,21 +449,18 @@ __global__ void __launch_bounds__(kMergeThreads) sparse_merge_kernel(const Merge
     }
   }
 
-  // listed logits; validity of the ids; the listed maximum
-  bool bad = false;   // an id outside [0, V), or a repeated id
+  // listed logits (the stream captured those below listed_end); the listed maximum
   bool nan = false;
   float lm = -CUDART_INF_F;
-#pragma unroll 4
+#pragma unroll 8
   for (int j = lane; j < p.K; j += 32) {
-    const int2 t = top[j];
+    const int id = __float_as_int(ysw[j]);
     const float g = gy[j];
     float y = -CUDART_INF_F;
-    if (t.x < 0 || t.x >= p.vocab) bad = true;
-    else y = (t.x < listed_end) ? g : El::load1(yrow, t.x);
+    if (id >= 0 && id < p.vocab) y = (id < listed_end) ? g : El::load1(yrow, id);
     nan |= (y != y);
     lm = fmaxf(lm, y);
     ysw[j] = y;
-    lpw[j] = __int_as_float(t.y);
   }
   __syncwarp();
   bad = __any_sync(0xffffffffu, bad) || (acc.flags & kFlagRepeat);
@@ -494,21 +505,34 @@ __global__ void __launch_bounds__(kMergeThreads) sparse_merge_kernel(const Merge
   nan = __any_sync(0xffffffffu, nan) || tail_nan || (acc.r != acc.r);
   const bool valid = !nan && !isinf(m) && cand != INT32_MAX;
 
-  // S = sum_R e^{y_j - m} + T, with T the tail mass relative to m
+  // S = sum_R e^{y_j - m} + T, with T the tail mass relative to m.  The
+  // listed weights are ex2 on the MUFU unit (relative error ~1e-7; a
+  // maximum's weight is exactly 1, so log S keeps its relative accuracy for
+  // near-certain rows), summed in f64.
   double sw = 0.0;
 #pragma unroll 4
-  for (int j = lane; j < p.K; j += 32) sw += exp((double)ysw[j] - (double)m);
+  for (int j = lane; j < p.K; j += 32) {
+    const float y = ysw[j];
+    sw += (y == m) ? 1.0 : (double)ex2((y - m) * kLog2e);
+  }
   sw = warp_sum(sw);
   const double T = have_tail ? (1.0 + (double)acc.r) * exp((double)acc.m - (double)m) : 0.0;
   const double S = sw + T;
   const double logS = log(S);
 
+  // p_j also from ex2 for the KL terms (in f64 where ex2 underflows, so that
+  // every p_j > 0 counts: against a candidate -inf it makes the KL +inf);
+  // without a stored tail the reference's tail mass is 1 - sum p_j, which
+  // cancels: that sum takes p_j in f64
+  const bool need_psum = p.ref_rows == nullptr;
   double kl = 0.0, psum = 0.0;
 #pragma unroll 4
   for (int j = lane; j < p.K; j += 32) {
-    const double lp = (double)lpw[j];
-    const double pj = exp(lp);
-    psum += pj;
+    const float lpf = lpw[j];
+    const double lp = (double)lpf;
+    const float pf = ex2(lpf * kLog2e);
+    const double pj = pf > 0.f ? (double)pf : exp(lp);
+    if (need_psum) psum += exp(lp);
     if (pj > 0.0) kl += pj * (lp - (((double)ysw[j] - (double)m) - logS));
   }
   kl = warp_sum(kl);
@@ -577,6 +601,11 @@ cudaError_t launch_sparse_ref(const SparseRefArgs& a, cudaStream_t stream) {
   MergeParams mp{a.y, a.ld, (int)a.vocab, nvec, (int)a.n_rows, nwarps, total, pieces, top, a.k, gy,
                  a.ref_rows, a.targets, a.kl, a.argmax, a.top1, a.lp_cand, a.lp_ref, a.dev_status};
   const unsigned mgrid = (unsigned)((a.n_rows + kMergeWarps - 1) / kMergeWarps);
+  if (total == 0) {  // no streaming pass: the merge reads its inputs at once, so no early launch
+    if (a.bf16) sparse_merge_kernel<true><<<mgrid, kMergeThreads, 0, stream>>>(mp);
+    else sparse_merge_kernel<false><<<mgrid, kMergeThreads, 0, stream>>>(mp);
+    return cudaGetLastError();
+  }
   if (a.bf16) return launch_dependent(sparse_merge_kernel<true>, dim3(mgrid), dim3(kMergeThreads), stream, mp);
   return launch_dependent(sparse_merge_kernel<false>, dim3(mgrid), dim3(kMergeThreads), stream, mp);
 }

@@ -123,6 +123,29 @@ def test_ties_nonfinite_and_bad_target(cuda_device, dtype):
     assert (res["ids"][2:5] == -1).all()
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_long_tie_runs(cuda_device, dtype):
+    """K = 1024 with long runs of equal values: a whole row equal, 600 equal
+    values at the top, 300 values tied at the K-th (more than are ranked by
+    counting), and runs of 40 equal values all through the list."""
+    V, k = 70_001, 1024
+    d = W.window_full_vocab(seed=W.SEED_BASE + 3200, device=cuda_device, n_rows=4, vocab=70_008,
+                            dtype=torch.float32)
+    x = padded(d["ref"][:, :V].contiguous().to(dtype), 8 if dtype == torch.bfloat16 else 4)
+    tg = torch.remainder(d["targets"], V).to(torch.int32)
+    x[0] = -2.0
+    x[1, 1000:1600] = x[1].max() + 1.0
+    srt = torch.sort(x[2].float(), descending=True).values
+    kth = float(srt[k - 1])
+    x[2, (x[2].float() == kth)] = kth - 1.0          # clear the natural ties there ...
+    x[2, 20_000:20_300] = kth                         # ... and plant 300 of them
+    order = torch.argsort(x[3].float(), descending=True)[:k]
+    x[3, order] = torch.repeat_interleave(x[3, order[::40]], 40)[:k]   # runs of 40 equal values
+    res = run(x, k, tg)
+    assert res["status"] == 0
+    check(res, x, k, tg)
+
+
 def test_round_trip_through_the_score(cuda_device):
     """A candidate equal to the captured reference scores 0 against it."""
     d = W.window_full_vocab(seed=W.SEED_BASE + 3200, device=cuda_device, n_rows=64, vocab=50_000)

@@ -140,12 +140,16 @@ def test_edge_rows(cuda_device):
     cand[9, unl9] = hi9
     # row 10: listed ids 100 .. 163, all inside the first streaming step
     top[10, :, 0] = torch.arange(100, 100 + K, device=cuda_device, dtype=torch.int32)
+    # row 11: a listed id with p = e^-100 (below the f32 range, not f64's)
+    # where the candidate logit is -inf: KL = +inf
+    top[11, K - 1, 1] = torch.tensor([-100.0], dtype=torch.float32).view(torch.int32).item()
+    cand[11, int(top[11, K - 1, 0])] = float("-inf")
     res = run(cand, top, rows, tg)
     assert res["status"] == (_lib.KLD_DEV_BAD_ID | _lib.KLD_DEV_BAD_TARGET)
     want = oracle(cand, top, rows, tg)
     check(res, want)
     kl = res["kl"].cpu().numpy()
-    assert np.isnan(kl[[0, 1, 2, 3, 7]]).all() and kl[4] == np.inf
+    assert np.isnan(kl[[0, 1, 2, 3, 7]]).all() and kl[4] == np.inf and kl[11] == np.inf
     assert res["cand_argmax"][8].item() == unl and res["cand_argmax"][9].item() == lo_listed
     assert np.isnan(res["cand_target_lp"][5].item())
 
