@@ -163,6 +163,16 @@ __device__ __forceinline__ uint32_t bf16x2_floor(uint32_t w) {
   return r;
 }
 
+// Both bf16 halves of w that are >= the bf16 halves of tau2 moved down by
+// the lowest finite bf16 (1.0 or 0.0 per half from the compare, then one
+// fused multiply-add); the others unchanged.
+__device__ __forceinline__ uint32_t bf16x2_mask_ge(uint32_t w, uint32_t tau2) {
+  uint32_t s, r;
+  asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(s) : "r"(w), "r"(tau2));
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(s), "r"(0xff7fff7fu), "r"(w));
+  return r;
+}
+
 // Shift that takes a candidate's exponent far below any real one: its
 // weight underflows to exactly 0.
 constexpr float kMaskShift = 1e30f;
@@ -266,24 +276,33 @@ __device__ CapPiece cap_piece(const CapParams& p, CapRing& R, int row, int a, in
     const float2 nm = make_float2(-mo, -mo);
     const float2 l2 = make_float2(kLog2e, kLog2e);
     const float2 shove = make_float2(-kMaskShift, -kMaskShift);
+    const uint32_t tau2 = kBF16 ? ((__float_as_uint(tau) >> 16) * 0x10001u) : 0u;  // tau is a bf16 value
 #pragma unroll
     for (int q = 0; q < kVecs; ++q) {
       uint4 u = v[q];
       if constexpr (kBF16) {
-        // -inf -> the lowest finite bf16 (NaN kept), so d below is finite
-        // and w * d never forms 0 * inf; its weight is exactly 0 either way
-        u.x = bf16x2_floor(u.x);
-        u.y = bf16x2_floor(u.y);
-        u.z = bf16x2_floor(u.z);
-        u.w = bf16x2_floor(u.w);
+        // a candidate (>= tau) is moved down by the lowest bf16, far below
+        // any maximum (weight 0); then whatever is -inf (a -inf logit, or a
+        // negative candidate moved past the lowest) is raised to the lowest
+        // finite bf16 (NaN kept), so d below is finite and w * d never
+        // forms 0 * inf
+        u.x = bf16x2_floor(bf16x2_mask_ge(u.x, tau2));
+        u.y = bf16x2_floor(bf16x2_mask_ge(u.y, tau2));
+        u.z = bf16x2_floor(bf16x2_mask_ge(u.z, tau2));
+        u.w = bf16x2_floor(bf16x2_mask_ge(u.w, tau2));
       }
 #pragma unroll
       for (int k = 0; k < E / 2; ++k) {
         const float2 X = El::pair(u, k);
         float2 d = __fadd2_rn(X, nm);
-        // a candidate (X >= tau) is pushed far below the maximum: weight 0
-        const float2 c = make_float2(set_ge(X.x, tau), set_ge(X.y, tau));
-        const float2 t = __fmul2_rn(__ffma2_rn(c, shove, d), l2);
+        float2 t;
+        if constexpr (kBF16) {
+          t = __fmul2_rn(d, l2);
+        } else {
+          // a candidate (X >= tau) is pushed far below the maximum: weight 0
+          const float2 c = make_float2(set_ge(X.x, tau), set_ge(X.y, tau));
+          t = __fmul2_rn(__ffma2_rn(c, shove, d), l2);
+        }
         const float2 w = make_float2(ex2(t.x), ex2(t.y));
         T2 = __fadd2_rn(T2, w);
         if constexpr (!kBF16) {
