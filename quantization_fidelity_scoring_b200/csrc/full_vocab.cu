@@ -2,8 +2,10 @@
 //
 // The rows' 16-byte vectors, flattened in (row, vector) order, are split
 // evenly over a fixed set of persistent warps.  Each warp streams its range
-// with 128-bit non-allocating loads, two vectors per lane per step, and
-// keeps an online log-sum-exp state (kld_common.cuh) whose running maximum and argmax are
+// two vectors per lane per side per step, copied by the lane itself with
+// 16-byte cp.async into a per-warp shared-memory ring three steps ahead of
+// the step it reads (no registers held for loads in flight), and keeps an
+// online log-sum-exp state (kld_common.cuh) whose running maximum and argmax are
 // warp-uniform: one redux.sync finds a step's maximum, and only a step that
 // raises it (a handful per row piece) takes the branch that rescales,
 // locates the new argmax and leaves it out of the sum.  Every other step is
@@ -181,8 +183,20 @@ __device__ __forceinline__ float slot_diff(const StepRaw& raw, int j) {
 
 // Stream vectors [a, b) of one row; returns the warp's partial state
 // (identical in every lane).
+// 16-byte asynchronous copy global -> shared (cached in L2 only), and the
+// group bookkeeping of such copies
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((unsigned)__cvta_generic_to_shared(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_two() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+constexpr int kRingSteps = 4;  // steps a warp's ring holds: the one read, three in flight
+
 template <bool kBF16>
-__device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow, int a, int b, int lane) {
+__device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow, int a, int b, int lane,
+                                              uint4* ring) {
   using El = Elems<kBF16>;
   constexpr int E = El::E;
   constexpr uint32_t kNegInfWord = kBF16 ? 0xff80ff80u : 0xff800000u;
@@ -212,13 +226,6 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
   const char* xl = xrow + (int64_t)(a + lane) * 16;
   const char* yl = yrow + (int64_t)(a + lane) * 16;
 
-  auto load_full = [&](StepRaw& r, int st) {
-    const int64_t o = (int64_t)st * kStepVecs * 16;
-    r.x0 = ld_stream(xl + o);
-    r.y0 = ld_stream(yl + o);
-    r.x1 = ld_stream(xl + o + 32 * 16);
-    r.y1 = ld_stream(yl + o + 32 * 16);
-  };
   auto step = [&](const StepRaw& cur, int st) {
     const float CMX = warp_max(El::vmax2(cur.x0, cur.x1));
     const float CMY = warp_max(El::vmax2(cur.y0, cur.y1));
@@ -249,17 +256,37 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
     if (++since == kFlushSteps) fold();  // warp-uniform
   };
 
-  // full steps: the warp's four 16-byte loads per lane for step st + 1 are
-  // issued before step st is processed, so one step of loads is always in
-  // flight per warp; other warps cover the rest of the latency
-  StepRaw A, B;
+  // full steps: each lane copies its four 16-byte vectors of step st + 3
+  // into the warp's shared-memory ring (cp.async: no registers held) before
+  // step st is processed, so three steps of loads are in flight per warp
+  auto issue = [&](int s) {
+    const int64_t o = (int64_t)s * kStepVecs * 16;
+    uint4* r = ring + (s % kRingSteps) * 4 * 32 + lane;
+    cp_async16(r, xl + o);
+    cp_async16(r + 32, yl + o);
+    cp_async16(r + 64, xl + o + 32 * 16);
+    cp_async16(r + 96, yl + o + 32 * 16);
+  };
+  StepRaw A;
   int st = 0;
-  if (nfull > 0) load_full(B, 0);
+  if (nfull > 0) issue(0);
+  cp_async_commit();
+  if (nfull > 1) issue(1);
+  cp_async_commit();
+  if (nfull > 2) issue(2);
+  cp_async_commit();
   for (; st < nfull; ++st) {
-    A = B;
-    if (st + 1 < nfull) load_full(B, st + 1);  // next step's loads stay in flight
+    cp_async_wait_two();  // every group but the two newest has landed: step st is in the ring
+    const uint4* r = ring + (st % kRingSteps) * 4 * 32 + lane;
+    A.x0 = r[0];
+    A.y0 = r[32];
+    A.x1 = r[64];
+    A.y1 = r[96];
+    if (st + 3 < nfull) issue(st + 3);  // into the slot read one step ago
+    cp_async_commit();
     step(A, st);
   }
+  cp_async_wait_all();
   // ragged last step: lanes past b read -inf
   if (st * kStepVecs < n) {
     const int v0 = st * kStepVecs + lane, v1 = v0 + 32;
@@ -287,6 +314,8 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
 template <bool kBF16>
 __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) stream_kernel(const StreamParams p) {
   constexpr int kElemBytes = kBF16 ? 2 : 4;
+  extern __shared__ __align__(16) uint4 rings_dyn[];
+  uint4 (*rings)[kRingSteps * 4 * 32] = reinterpret_cast<uint4 (*)[kRingSteps * 4 * 32]>(rings_dyn);
   const int lane = threadIdx.x & 31;
   const int w = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (w >= p.nwarps) return;  // the whole warp leaves together
@@ -299,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, kStreamCtasPerSm) stream_kernel(cons
     const int b = (int)min((int64_t)p.nvec, end - row0);
     const char* xrow = reinterpret_cast<const char*>(p.x) + (int64_t)row * p.ld_x * kElemBytes;
     const char* yrow = reinterpret_cast<const char*>(p.y) + (int64_t)row * p.ld_y * kElemBytes;
-    const Piece pc = stream_piece<kBF16>(xrow, yrow, a, b, lane);
+    const Piece pc = stream_piece<kBF16>(xrow, yrow, a, b, lane, rings[threadIdx.x >> 5]);
     if (lane == 0) p.pieces[row + w] = pc;
     pos = row0 + b;
   }
@@ -466,8 +495,16 @@ cudaError_t launch_full_vocab(const FullVocabArgs& a, cudaStream_t stream) {
   if (total > 0) {
     StreamParams sp{a.x, a.y, a.ld_x, a.ld_y, nvec, nwarps, total, pieces};
     const unsigned grid = (unsigned)((nwarps + kWarpsPerCta - 1) / kWarpsPerCta);
-    if (a.bf16) stream_kernel<true><<<grid, kThreads, 0, stream>>>(sp);
-    else stream_kernel<false><<<grid, kThreads, 0, stream>>>(sp);
+    constexpr size_t kRingBytes = sizeof(uint4) * kWarpsPerCta * kRingSteps * 4 * 32;
+    if (a.bf16) {
+      cudaError_t e0 = allow_dynamic_smem<stream_kernel<true>>(kRingBytes);
+      if (e0 != cudaSuccess) return e0;
+      stream_kernel<true><<<grid, kThreads, kRingBytes, stream>>>(sp);
+    } else {
+      cudaError_t e0 = allow_dynamic_smem<stream_kernel<false>>(kRingBytes);
+      if (e0 != cudaSuccess) return e0;
+      stream_kernel<false><<<grid, kThreads, kRingBytes, stream>>>(sp);
+    }
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
