@@ -151,7 +151,7 @@ size_t kld_full_vocab_workspace_size(int64_t n_rows);
  * Limits and behaviour:
  *   - n_rows <= KLD_NOALLOC_MAX_ROWS; larger n_rows returns
  *     KLD_ERR_UNSUPPORTED and launches nothing (split the batch instead).
- *   - The array takes about 1.2 MB on every GPU that loads the library and
+ *   - The array takes about 1.1 MB on every GPU that loads the library and
  *     stays allocated until the process exits.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current, and so does the first

@@ -3,7 +3,7 @@
 // The rows' 16-byte vectors, flattened in (row, vector) order, are split
 // evenly over a fixed set of persistent warps.  Each warp streams its range
 // two vectors per lane per side per step, copied by the lane itself with
-// 16-byte cp.async into a per-warp shared-memory ring three steps ahead of
+// 16-byte cp.async into a per-warp shared-memory ring five steps ahead of
 // the step it reads (no registers held for loads in flight), and keeps an
 // online log-sum-exp state (kld_common.cuh) whose running maximum and argmax are
 // warp-uniform: one redux.sync finds a step's maximum, and only a step that
@@ -190,9 +190,9 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_two() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_four() { asm volatile("cp.async.wait_group 4;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-constexpr int kRingSteps = 4;  // steps a warp's ring holds: the one read, three in flight
+constexpr int kRingSteps = 6;  // steps a warp's ring holds: the one read, five in flight
 
 template <bool kBF16>
 __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow, int a, int b, int lane,
@@ -256,9 +256,9 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
     if (++since == kFlushSteps) fold();  // warp-uniform
   };
 
-  // full steps: each lane copies its four 16-byte vectors of step st + 3
+  // full steps: each lane copies its four 16-byte vectors of step st + 5
   // into the warp's shared-memory ring (cp.async: no registers held) before
-  // step st is processed, so three steps of loads are in flight per warp
+  // step st is processed, so five steps of loads are in flight per warp
   auto issue = [&](int s) {
     const int64_t o = (int64_t)s * kStepVecs * 16;
     uint4* r = ring + (s % kRingSteps) * 4 * 32 + lane;
@@ -275,14 +275,18 @@ __device__ __forceinline__ Piece stream_piece(const char* xrow, const char* yrow
   cp_async_commit();
   if (nfull > 2) issue(2);
   cp_async_commit();
+  if (nfull > 3) issue(3);
+  cp_async_commit();
+  if (nfull > 4) issue(4);
+  cp_async_commit();
   for (; st < nfull; ++st) {
-    cp_async_wait_two();  // every group but the two newest has landed: step st is in the ring
+    cp_async_wait_four();  // every group but the four newest has landed: step st is in the ring
     const uint4* r = ring + (st % kRingSteps) * 4 * 32 + lane;
     A.x0 = r[0];
     A.y0 = r[32];
     A.x1 = r[64];
     A.y1 = r[96];
-    if (st + 3 < nfull) issue(st + 3);  // into the slot read one step ago
+    if (st + 5 < nfull) issue(st + 5);  // into the slot read one step ago
     cp_async_commit();
     step(A, st);
   }

@@ -26,8 +26,9 @@ struct FullVocabArgs {
   int warps_override;    // 0: choose from the problem size
 };
 // Upper bound on the streaming warps (fixed, so results do not depend on the
-// device): three CTAs of eight warps per SM on 148 SMs.
-constexpr int kStreamCtasPerSm = 3;
+// device): two CTAs of eight warps per SM on 148 SMs (each CTA holds its
+// warps' 96 KB of load rings).
+constexpr int kStreamCtasPerSm = 2;
 constexpr int kFullVocabMaxWarps = 148 * kStreamCtasPerSm * 8;
 // The sparse-reference and capture streams: at most three CTAs of eight
 // persistent warps per SM of a 148-SM part (their row slots are row + warp).
