@@ -73,6 +73,8 @@ def check(res, x, k, targets, rows=None, chunk=64):
     (40, 5000, 1, torch.bfloat16),
     (9, 70_001, 777, torch.float32),     # sampled threshold
     (8, 262_147, 1024, torch.bfloat16),  # sampled threshold, ragged end, K at its limit
+    (6, 90_001, 777, torch.bfloat16),    # 32-bit sort keys with 247 padding slots
+    (10, 4096, 512, torch.bfloat16),     # the whole row fits the buffer, bf16
 ])
 @pytest.mark.parametrize("exact", [False, True])
 def test_shapes_all_rows(cuda_device, n, V, k, dtype, exact):
